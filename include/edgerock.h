@@ -1,0 +1,243 @@
+/*
+ * edgerock.h — C ABI of the B200 (sm_100a) SWA∥RMA hot path of EdgeRock-4B.
+ *
+ * What the layer is (page title, section):
+ *  [F-arch] fluxbbs.com "EdgeRock-4B 开源：72 MiB 固定 KV，AIME 82.9 分",
+ *           §架构：递归、局部窗口与记忆锚点三件套 — hidden 2560; the eight
+ *           sliding-window layers run a 1024-position window in parallel with
+ *           Rock Memory Anchors (RMA); 16 query heads over 4 KV groups, head
+ *           dim 256, learned RMS-norm on q and k, RoPE on 64 of the 256 dims
+ *           with base 1e7, values neither rotated nor normed; a bias-free FP32
+ *           scorer 2560→256→4 gives one retention score per KV group; each
+ *           group keeps its own top records, groups may share positions;
+ *           candidates gather in blocks of 256 and the bank keeps 1024.
+ *  [F-mem]  same page, §72 MiB 是怎么算出来的 — every part of the state has a
+ *           hard capacity: 32 MiB committed anchors, 8 MiB pending block,
+ *           32 MiB window, 72 MiB per sequence whatever its length.
+ *  [N-rma]  neodrop.ai "内存还会跌吗？KV Cache砍掉99%，单卡吞吐飙6倍…",
+ *           §三段记忆，只记值得记的 — a writer makes one candidate per token, a
+ *           scorer rates it; at 256 candidates they are compared with the bank
+ *           and only the 1024 best are kept, for each of the four KV groups;
+ *           kept anchors are independent and never change.
+ *  Readings fixed where the pages are silent: SiLU between the two scorer
+ *  matmuls; the RMA read is its own softmax over committed + pending records
+ *  with its own q/k/v projections, added to the SWA output before one shared
+ *  o_proj; ties in the top-k go to the lower source position.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named in a signature are DEVICE pointers unless marked (host).
+ *    The caller allocates and frees all memory (state, weights, inputs,
+ *    outputs, workspace); the library never allocates or frees device memory
+ *    and never synchronises the stream, except er_last_device_error, which
+ *    reads one word back.
+ *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).
+ *  - Return value: ER_OK, or a negative ER_E* code.  Host-side argument checks
+ *    happen before anything is enqueued; a failed check enqueues nothing.
+ *    Conditions only the device can see (a sequence id out of range, a full
+ *    pending block, a prefill chunk crossing the block boundary) skip the
+ *    affected sequence and record the first such code in the state's device
+ *    error word (read with er_last_device_error).  No kernel traps.
+ *  - BF16 values are raw bfloat16 bit patterns (er_bf16).
+ */
+#ifndef EDGEROCK_H
+#define EDGEROCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t er_bf16;
+typedef struct CUstream_st* er_stream_t; /* same type as cudaStream_t */
+
+/* Layer shape [F-arch], capacities [F-mem]/[N-rma]. */
+#define ER_HIDDEN 2560
+#define ER_Q_HEADS 16
+#define ER_KV_GROUPS 4
+#define ER_HEADS_PER_GROUP 4
+#define ER_HEAD_DIM 256
+#define ER_MAX_LAYERS 8
+#define ER_WINDOW 1024
+#define ER_BANK 1024
+#define ER_PENDING 256
+#define ER_ROPE_DIMS 64
+#define ER_SCORE_HIDDEN 256
+#define ER_QKV_ROWS 12288 /* 4096 + 1024 + 1024 (SWA) + 4096 + 1024 + 1024 (RMA) */
+#define ER_O_IN 4096      /* 16 heads x 256 */
+
+enum {
+  ER_OK = 0,
+  ER_EINVAL = -1,    /* bad argument (null pointer, size or index out of range) */
+  ER_ECAPACITY = -2, /* pending block full, batch above capacity, workspace too small */
+  ER_ECUDA = -3,     /* a CUDA launch or runtime call failed */
+  ER_EDEVICE = -4    /* returned by er_last_device_error when the device word is set */
+};
+
+/* Per-sequence fixed-capacity state, carved out of ONE caller allocation by
+ * er_state_carve.  Layouts ([seq] is the state row, not a batch index):
+ *   win_k, win_v   BF16  [s_max][n_layers][4][1024][256]  ring: position t in slot t % 1024
+ *   bank_k, bank_v BF16  [s_max][n_layers][4][1024][256]  committed anchors, slots [0, bank_count)
+ *   pend_k, pend_v BF16  [s_max][n_layers][4][256][256]   pending block, slots [0, pend_count)
+ *   bank_score     FP32  [s_max][n_layers][4][1024]       score of each committed record
+ *   pend_score     FP32  [s_max][n_layers][4][256]
+ *   bank_pos       INT32 [s_max][n_layers][4][1024]       source position of each record
+ *   pend_pos       INT32 [s_max][n_layers][4][256]
+ *   meta           INT32 [s_max][4] = {pos, pend_count, bank_count, 0}; pos is the
+ *                  position of the next token; the counts are shared by every
+ *                  layer and group because every token appends to each.
+ *   dev_error      INT32 [4]: first device-side error code (0 = none).
+ * K rows are stored already RMS-normed and rotated at their source position.
+ */
+typedef struct er_state {
+  er_bf16 *win_k, *win_v, *bank_k, *bank_v, *pend_k, *pend_v;
+  float *bank_score, *pend_score;
+  int32_t *bank_pos, *pend_pos;
+  int32_t *meta;
+  int32_t *dev_error;
+  int32_t s_max;
+  int32_t n_layers;
+} er_state;
+
+/* One SWA∥RMA layer's weights (device, caller-owned), nn.Linear layout [out][in]:
+ *   w_qkv BF16 [12288][2560]: rows q_swa 0..4095 | k_swa 4096..5119 | v_swa 5120..6143 |
+ *                             q_rma 6144..10239 | k_rma 10240..11263 | v_rma 11264..12287
+ *   w_o   BF16 [2560][4096]  shared o_proj
+ *   q_norm_swa, k_norm_swa, q_norm_rma, k_norm_rma: BF16 [256] RMS-norm gains
+ *                             (one per head dim, shared by all heads of the branch)
+ *   w1    FP32 [256][2560], w2 FP32 [4][256]: the scorer, bias-free. */
+typedef struct er_layer_weights {
+  const er_bf16* w_qkv;
+  const er_bf16* w_o;
+  const er_bf16 *q_norm_swa, *k_norm_swa, *q_norm_rma, *k_norm_rma;
+  const float* w1;
+  const float* w2;
+} er_layer_weights;
+
+/* ---------------------------------------------------------------- state */
+
+/* Bytes er_state_carve needs for s_max sequences of n_layers (1..8) layers:
+ * 72 MiB of K/V per sequence at 8 layers [F-mem], plus scores, positions,
+ * metadata and alignment.  Returns 0 on bad arguments.  Host-only. */
+size_t er_state_bytes(int32_t s_max, int32_t n_layers);
+
+/* Fills *out with pointers into [base, base+bytes) (device memory, caller
+ * owned, 256-byte aligned).  Touches no memory.  ER_EINVAL if bytes is too
+ * small, base is unaligned, or sizes are out of range. */
+int er_state_carve(void* base, size_t bytes, int32_t s_max, int32_t n_layers, er_state* out);
+
+/* Empties the listed sequences: meta := {0, 0, 0, 0}.  seq_ids: device
+ * int32 [n].  Row contents are left as they are (unread until written). */
+int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stream_t stream);
+
+/* End of one step of T tokens for the listed sequences, after every layer's
+ * call: pos += T; pend_count += T, and a block that reached 256 (which every
+ * layer has committed) empties: pend_count := 0, bank_count := min(1024,
+ * bank_count + 256).  T in 1..256. */
+int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
+               er_stream_t stream);
+
+/* Copies the device error word to *code (host) and clears it; synchronises
+ * `stream`.  Returns ER_OK when the word was 0, else ER_EDEVICE. */
+int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream);
+
+/* ------------------------------------------------------- hot-path steps */
+
+/* a2 — RMS-norm with gain, then rotary embedding of dims [0, 64) at each
+ * row's position [F-arch]: y = x / sqrt(mean(x^2) + 1e-6) * gain, then for
+ * i < 32 the pair (i, i+32) turns by pos * 1e7^(-2i/64).  x, y: BF16
+ * [n_rows][256] (may alias); gain: BF16 [256]; pos: INT32 [n_rows]. */
+int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, const er_bf16* gain,
+                    const int32_t* pos, er_stream_t stream);
+
+/* a3 — retention scores [F-arch], [N-rma]: s = W2 · SiLU(W1 · x), FP32
+ * products and sums.  x: BF16 [n][2560]; s: FP32 [n][4] (one per KV group).
+ * n may be 0. */
+int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s,
+                 er_stream_t stream);
+
+/* a4 — appends one candidate record per KV group for each listed sequence at
+ * its pend_count slot of `layer` [N-rma]: k, v BF16 [n][4][256] (k already
+ * normed and rotated), s FP32 [n][4], pos INT32 [n].  Metadata is not
+ * changed (er_advance does that once per step).  A sequence whose block is
+ * already full is skipped and records ER_ECAPACITY on the device. */
+int er_rma_append_pending(const er_state* st, int32_t layer, const int32_t* seq_ids, int32_t n,
+                          const er_bf16* k, const er_bf16* v, const float* s,
+                          const int32_t* pos, er_stream_t stream);
+
+/* a7 — commit [F-arch], [N-rma]: for each listed sequence and each KV group
+ * independently, the bank_count committed and pend_count pending records are
+ * ranked by (score descending, source position ascending; -0 ranks as +0,
+ * NaN below every number) and the top min(1024, bank_count + pend_count)
+ * stay.  Surviving anchors do not move; evicted bank slots in ascending order,
+ * then slots bank_count, bank_count+1, ..., receive the pending winners in
+ * ascending pending order.
+ *   layer >= 0: that layer only; metadata untouched (a decode step commits
+ *               each layer, then er_advance empties the block).
+ *   layer == -1: every layer, then pend_count := 0 and
+ *               bank_count := min(1024, bank_count + pend_count).
+ *   kept (optional, may be NULL): INT32 [n][layers][4][1024], the kept
+ *   records in rank order as indices 0..1023 (bank slot) / 1024+j (pending
+ *   j), -1 padded; `layers` is n_layers for layer == -1, else 1. */
+int er_rma_commit(const er_state* st, int32_t layer, const int32_t* seq_ids, int32_t n,
+                  int32_t* kept, er_stream_t stream);
+
+/* a5 — the two reads of a decode step, for B sequences whose current token
+ * (position pos) has already been written to the window and appended at
+ * pending slot pend_count: for head h of group h/4,
+ *   o_swa = softmax(q_swa·Kᵀ/16)·V over window positions [pos-1023, pos];
+ *   o_rma = softmax(q_rma·Kᵀ/16)·V over bank slots [0, bank_count) and
+ *           pending slots [0, pend_count]  (o = 0 over an empty list).
+ * q_swa, q_rma: BF16 [B][16][256] (normed, rotated); o_swa, o_rma: FP32
+ * [B][16][256].  ws: workspace of er_attend_workspace_bytes(B) bytes. */
+size_t er_attend_workspace_bytes(int32_t B);
+int er_swa_rma_attend(const er_state* st, int32_t layer, const int32_t* seq_ids, int32_t B,
+                      const er_bf16* q_swa, const er_bf16* q_rma, float* o_swa, float* o_rma,
+                      void* ws, size_t ws_bytes, er_stream_t stream);
+
+/* a1–a7 — one decode step of one layer for B sequences (one token each at
+ * its meta pos): q/k/v projections of both branches, norm + RoPE, scores,
+ * window write (slot pos % 1024), pending append, the two reads,
+ * out = W_o · bf16(o_swa + o_rma), and the commit of this layer for every
+ * sequence whose block this token fills (pend_count + 1 == 256), decided on
+ * the device.  x, out: BF16 [B][2560].  ws: er_decode_workspace_bytes(B).
+ * A step is one call per layer followed by one er_advance(T=1). */
+size_t er_decode_workspace_bytes(int32_t B);
+int er_swa_rma_decode(const er_state* st, const er_layer_weights* w, int32_t layer,
+                      const int32_t* seq_ids, int32_t B, const er_bf16* x, er_bf16* out,
+                      void* ws, size_t ws_bytes, er_stream_t stream);
+
+/* a8 — a prefill chunk of T tokens (1..256) of one sequence (state row
+ * seq_id, a host int) at positions pos..pos+T-1.  Requires
+ * pend_count + T <= 256 (checked on the device).  Token i reads, causally,
+ * window positions [t-1023, t] (old ring entries and the chunk's own tokens)
+ * and the bank plus pending slots [0, pend_count + i]; the chunk enters the
+ * ring after every read; the layer commits if the chunk fills the block.
+ * x, out: BF16 [T][2560]; ws: er_prefill_workspace_bytes(T).  Follow the
+ * chunk's calls for every layer with er_advance(T). */
+size_t er_prefill_workspace_bytes(int32_t T);
+int er_swa_rma_prefill_chunk(const er_state* st, const er_layer_weights* w, int32_t layer,
+                             int32_t seq_id, const er_bf16* x, int32_t T, er_bf16* out,
+                             void* ws, size_t ws_bytes, er_stream_t stream);
+
+/* ------------------------------------------------------ instrumentation */
+
+/* Human-readable name of an ER_* code (static string). */
+const char* er_error_string(int code);
+
+/* Number of kernels this library has launched since load (all threads). */
+uint64_t er_launch_count(void);
+
+/* When enabled, the a5 read kernel launches are bracketed by CUDA events on
+ * their own stream; er_profile_read returns the summed milliseconds and the
+ * number of timed launches since the last reset (it synchronises the events).
+ * Host-side bookkeeping only; not thread-safe. */
+int er_profile_enable(int enable);
+int er_profile_read(double* ms_total, int64_t* launches, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EDGEROCK_H */
