@@ -1,0 +1,358 @@
+"""Benchmark: SWA∥RMA decode tok/s at B=512 over 8 layers, commits/s, % of HBM roofline.
+
+Workload (per GPU; weak scaling over GPUs, no data-path collective): 512
+sequences, 8 SWA∥RMA layers, state seeded at position 32768 with window and
+bank full and pending fill U{0..255} per sequence (36 GiB of BF16 K/V, far
+above the 126 MB L2, so no flush is needed between steps).  One step = one
+token for every sequence through all 8 layers (projections, scores, norm +
+RoPE, window write, pending append, both reads, o_proj, device-decided commits)
+plus the metadata advance.  Over 256 steps every sequence commits once.
+
+Usage: python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+Under torchrun each rank runs its own replica on its own GPU; rank 0 prints
+one JSON line with the whole-job throughput (max time over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SWA∥RMA decode tok/s (B=512, 8 layers) + commits/s; % of B200 HBM roofline"
+WORKLOAD = "decode_b512_l8_t32768"
+B, LAYERS, T0 = 512, 8, 32768
+ROW = 1024  # bytes of one K row + one V row
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=4)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- our arm
+
+def algorithmic_read_bytes(fills, steps_from, steps):
+    """State bytes the reads of one layer must touch, summed over the given steps:
+    per (sequence, group) 1024 window rows + 1024 bank rows + (pending + 1) rows,
+    K and V, plus q (2 branches x 4 heads x 512 B) and o (2 x 4 x 1 KiB FP32)."""
+    tot = 0
+    for s in range(steps_from, steps_from + steps):
+        for f in fills:
+            p = (f + s) % 256
+            tot += 4 * ((1024 + 1024 + p + 1) * ROW + 2 * 4 * 512 + 2 * 4 * 1024)
+    return tot
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    seed = wl.seed_of(3)
+    weights = [sab.LayerWeights.from_dict(wl.make_weights(seed, l, device=dev))
+               for l in range(LAYERS)]
+    wdicts = [w.t for w in weights]
+    st = sab.State(B, LAYERS, device=dev)
+
+    def normrope(x, g, pos):
+        return sab.qk_norm_rope(x.contiguous(), g, pos.to(torch.int32).contiguous())
+
+    fills = wl.seed_state(st.arrays(), range(B), LAYERS, T0, "uniform", seed, wdicts, normrope,
+                          device=dev).cpu().tolist()
+    ids = torch.arange(B, dtype=torch.int32, device=dev)
+    ws = torch.empty(sab.decode_workspace_bytes(B), dtype=torch.uint8, device=dev)
+    total = args.warmup + args.steps
+    n_x = min(total, 64)  # distinct per-step inputs, resident before timing
+    xs = [[wl.make_x(seed, l, s, range(B), device=dev) for l in range(LAYERS)] for s in range(n_x)]
+    outs = [torch.empty(B, 2560, dtype=torch.bfloat16, device=dev) for _ in range(LAYERS)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(s):
+        for l in range(LAYERS):
+            sab.swa_rma_decode(st, weights[l], l, ids, xs[s % n_x][l], out=outs[l], ws=ws)
+        sab.advance(st, ids)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize(dev)
+    if sab.last_device_error(st) != 0:
+        raise RuntimeError("device error during warm-up")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sab.profile_read(reset=True)
+    sab.profile_enable(True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    n0 = sab.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(args.warmup, total):
+        step(s)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    launches = sab.launch_count() - n0
+    clk = clocks.stop()
+    sab.profile_enable(False)
+    attend_ms, attend_n = sab.profile_read(reset=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    err = sab.last_device_error(st)
+    if err != 0:
+        raise RuntimeError(f"device error {err} in the timed region")
+    commits = sum(1 for f in fills for s in range(args.warmup, total) if (f + s) % 256 == 255)
+
+    e2e = None
+    if not args.no_e2e:
+        # same steps through the C ABI from pinned host buffers: H2D of every layer's
+        # input and D2H of every layer's output inside the timed region
+        hx = [torch.empty(LAYERS, B, 2560, dtype=torch.bfloat16, pin_memory=True)
+              for _ in range(2)]
+        for i in range(2):
+            for l in range(LAYERS):
+                hx[i][l].copy_(xs[i][l])
+        hout = torch.empty(LAYERS, B, 2560, dtype=torch.bfloat16, pin_memory=True)
+        dx = torch.empty(LAYERS, B, 2560, dtype=torch.bfloat16, device=dev)
+        k_e2e = min(args.steps, 64)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for s in range(k_e2e):
+            dx.copy_(hx[s % 2], non_blocking=True)
+            for l in range(LAYERS):
+                sab.swa_rma_decode(st, weights[l], l, ids, dx[l], out=outs[l], ws=ws)
+            sab.advance(st, ids)
+            for l in range(LAYERS):
+                hout[l].copy_(outs[l], non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = f0.elapsed_time(f1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t)
+        nbytes = LAYERS * B * 2560 * 2
+        e2e = {"value": world * B * k_e2e / (e2e_ms / 1e3), "unit": "tok/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "steps": k_e2e}
+
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t)
+    return dict(ms=ms, launches=launches, clocks=clk, attend_ms=attend_ms, attend_n=attend_n,
+                fills=fills, commits=commits, e2e=e2e)
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def oracle_tokens_per_s(budget_s=12.0, max_threads=8):
+    """The oracle as it stands on the host cores: whole decode steps (8 layers) of
+    independent sequences of the same workload, one sequence per thread."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    from synth import workloads as wl
+
+    seed = wl.seed_of(3)
+    threads = max(1, min(max_threads, os.cpu_count() or 1))
+    ows = []
+    for l in range(LAYERS):
+        w = wl.make_weights(seed, l)
+        ows.append((oracle.OracleWeights(w["w_qkv"], w["w_o"], w["q_norm_swa"], w["k_norm_swa"],
+                                         w["q_norm_rma"], w["k_norm_rma"], w["w1"], w["w2"]), w))
+    wdicts = [w for _, w in ows]
+    states = []
+    for i in range(threads):
+        ost = oracle.OracleState(1, LAYERS)
+        arrays = {n: getattr(ost, n) for n in oracle.OracleState.ARRAYS}
+        wl.seed_state(arrays, [i], LAYERS, T0, "uniform", seed, wdicts, oracle.norm_rope)
+        states.append(ost)
+    xs = [[wl.make_x(seed, l, s, [i])[0] for l in range(LAYERS)] for i in range(threads)
+          for s in range(1)]
+    deadline = time.time() + budget_s
+    counts = [0] * threads
+
+    def work(i):
+        while time.time() < deadline:
+            for l in range(LAYERS):
+                states[i].decode_layer(ows[l][0], l, 0, xs[i][l])
+            states[i].advance(0)
+            counts[i] += 1
+
+    t0 = time.time()
+    with ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, range(threads)))
+    dt = time.time() - t0
+    return sum(counts) / dt, threads, sum(counts), dt
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return
+    budget = max(3.0, min(60.0, 2.0 * (args.steps + args.warmup)))
+    v, cores, toks, dt = oracle_tokens_per_s(budget_s=min(budget, 30.0))
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": B, "layers": LAYERS, "t0": T0,
+                       "pending_fill": "U{0..255}"},
+            "cpu_baseline": {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{toks} whole 8-layer decode steps of {cores} sequences "
+                                       f"of the workload in {dt:.1f} s"},
+            "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        reference_arm(args, rank, world)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    r = run_ours(args, rank, world, local_rank)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    hbm, peak_kind = peaks()
+    fills = r["fills"]
+    alg = algorithmic_read_bytes(fills, args.warmup, args.steps) * LAYERS
+    n_launch = max(r["attend_n"], 1)
+    per_launch = alg / (args.steps * LAYERS)
+    avg_ms = r["attend_ms"] / n_launch
+    achieved = per_launch / (avg_ms / 1e3) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "attend_traffic.json")
+    if os.path.exists(tpath):
+        traffic = json.load(open(tpath)).get("bytes_per_launch_full")
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        v, cores, toks, dt = oracle_tokens_per_s(budget_s=12.0)
+        cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle",
+               "sample": f"{toks} whole 8-layer decode steps of {cores} sequences of the "
+                         f"workload in {dt:.1f} s"}
+    secs = r["ms"] / 1e3
+    toks = world * B * args.steps
+    line = {
+        "metric": METRIC, "value": toks / secs, "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "layers": LAYERS, "t0": T0,
+                   "pending_fill": "U{0..255}", "state_gib_per_gpu": 36.0,
+                   "l2": "inputs larger than L2 (36 GiB state per GPU), no flush",
+                   "parallelism": f"replicas x{world}"},
+        "commits_per_s": world * r["commits"] / secs,
+        "merges_per_s": world * r["commits"] * LAYERS * 4 / secs,
+        "roofline": {"bound": "hbm", "kernel": "k_attend", "achieved": achieved, "peak": hbm,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": traffic, "alg_bytes_per_launch": per_launch,
+                     "avg_launch_ms": avg_ms, "launches": r["attend_n"]},
+        "cpu_baseline": cpu,
+        "e2e": r["e2e"],
+        "gpu_launches": r["launches"],
+        "clocks": r["clocks"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

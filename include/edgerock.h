@@ -72,7 +72,8 @@ enum {
   ER_EINVAL = -1,    /* bad argument (null pointer, size or index out of range) */
   ER_ECAPACITY = -2, /* pending block full, batch above capacity, workspace too small */
   ER_ECUDA = -3,     /* a CUDA launch or runtime call failed */
-  ER_EDEVICE = -4    /* returned by er_last_device_error when the device word is set */
+  ER_EDEVICE = -4,   /* returned by er_last_device_error when the device word is set */
+  ER_ETIMEOUT = -5   /* device word only: a bounded wait inside a kernel gave up */
 };
 
 /* Per-sequence fixed-capacity state, carved out of ONE caller allocation by

@@ -103,16 +103,19 @@ class OracleState:
     """Fixed-capacity per-sequence state, same [seq][layer][group][slot][256] layout
     as the device state so the two can be compared array by array."""
 
-    def __init__(self, s_max: int, n_layers: int = 8):
+    def __init__(self, s_max: int, n_layers: int = 8, kv: bool = True):
+        """kv=False builds a state with scores, positions and metadata only (no K/V
+        rows): enough to rank and place records in a commit."""
         self.s_max, self.n_layers = s_max, n_layers
         g = (s_max, n_layers, NG)
         z = torch.zeros
-        self.win_k = z(g + (WIN, D), dtype=torch.bfloat16)
-        self.win_v = z(g + (WIN, D), dtype=torch.bfloat16)
-        self.bank_k = z(g + (BANK, D), dtype=torch.bfloat16)
-        self.bank_v = z(g + (BANK, D), dtype=torch.bfloat16)
-        self.pend_k = z(g + (PEND, D), dtype=torch.bfloat16)
-        self.pend_v = z(g + (PEND, D), dtype=torch.bfloat16)
+        kvs = (lambda slots: g + (slots, D)) if kv else (lambda slots: (0,))
+        self.win_k = z(kvs(WIN), dtype=torch.bfloat16)
+        self.win_v = z(kvs(WIN), dtype=torch.bfloat16)
+        self.bank_k = z(kvs(BANK), dtype=torch.bfloat16)
+        self.bank_v = z(kvs(BANK), dtype=torch.bfloat16)
+        self.pend_k = z(kvs(PEND), dtype=torch.bfloat16)
+        self.pend_v = z(kvs(PEND), dtype=torch.bfloat16)
         self.bank_score = z(g + (BANK,), dtype=torch.float32)
         self.pend_score = z(g + (PEND,), dtype=torch.float32)
         self.bank_pos = z(g + (BANK,), dtype=torch.int32)
@@ -125,7 +128,8 @@ class OracleState:
 
     def _bind(self):
         self._s = _State(self.s_max, self.n_layers,
-                         *[getattr(self, n).data_ptr() for n in self.ARRAYS])
+                         *[(getattr(self, n).data_ptr() if getattr(self, n).numel() else None)
+                           for n in self.ARRAYS])
 
     def ptr(self):
         return ctypes.byref(self._s)

@@ -304,8 +304,10 @@ static void commit_group(orc_state* st, int s, int l, int g, int c, int p, int32
   for (int j = 0; j < p; ++j) {
     if (!pend_won[j]) continue;
     int slot = targets[t++];
-    memcpy(bank_k_row(st, s, l, g, slot), pend_k_row(st, s, l, g, j), OD * 2);
-    memcpy(bank_v_row(st, s, l, g, slot), pend_v_row(st, s, l, g, j), OD * 2);
+    if (st->bank_k) { /* a state built without K/V rows ranks and places records only */
+      memcpy(bank_k_row(st, s, l, g, slot), pend_k_row(st, s, l, g, j), OD * 2);
+      memcpy(bank_v_row(st, s, l, g, slot), pend_v_row(st, s, l, g, j), OD * 2);
+    }
     st->bank_score[gi * OBANK + slot] = st->pend_score[gi * OPEND + j];
     st->bank_pos[gi * OBANK + slot] = st->pend_pos[gi * OPEND + j];
   }

@@ -1,0 +1,272 @@
+// commit.cu — a7, the RMA anchor-bank commit, and a4's standalone append.
+//
+// EdgeRock-4B 开源：72 MiB 固定 KV, §架构：… and neodrop.ai "内存还会跌吗？…",
+// §三段记忆，只记值得记的: pending candidates are merged with the committed bank
+// once 256 have gathered; each KV group independently keeps the 1024 records
+// with the highest scores (groups may keep the same source positions); kept
+// anchors are never rewritten.  Ties go to the lower source position (the
+// reading fixed for this library), -0 ranks as +0 and NaN below every number.
+//
+// One 1024-thread block per (sequence, layer, group):
+//  1. 64-bit keys (ordered score << 32 | ~position) for the ≤1280 records,
+//     padded to 2048 with key 0, which ranks below every real record;
+//  2. bitonic sort in shared memory (descending), carrying the source index;
+//  3. flags for the top min(1024, c+p); two block scans give the evicted
+//     bank slots (ascending) and the pending winners (ascending);
+//  4. each warp moves winners' K and V rows (512 B each, 16 B per lane) into
+//     their target slots, with the score and position.
+// Surviving anchors are not touched, so the write traffic is only the moved
+// records.
+#include "common.cuh"
+#include "params.cuh"
+
+namespace er {
+namespace {
+
+constexpr int NSORT = 2048;
+constexpr int CT = 1024;  // threads per commit block
+
+__device__ __forceinline__ uint32_t ordered_score(float s) {
+  uint32_t u = __float_as_uint(s);
+  if ((u & 0x7FFFFFFFu) == 0) u = 0;             // -0 -> +0
+  if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu)) return 0;  // NaN: lowest
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t rec_key(float s, int32_t pos) {
+  return ((uint64_t)ordered_score(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)pos);
+}
+
+// Exclusive scan over the 1024 threads of a block; *total gets the sum.
+__device__ int block_scan_excl(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sums[lane] = w;  // inclusive
+  }
+  __syncthreads();
+  const int base = warp ? warp_sums[warp - 1] : 0;
+  *total = warp_sums[31];
+  __syncthreads();
+  return base + x - v;
+}
+
+}  // namespace
+
+
+__global__ void __launch_bounds__(CT) k_commit(CommitParams P) {
+  __shared__ uint64_t key[NSORT];
+  __shared__ uint16_t src[NSORT];
+  __shared__ uint8_t flag[BANK + PEND];
+  __shared__ int16_t evict_list[BANK];
+  __shared__ int32_t move_src[PEND], move_dst[PEND];
+  __shared__ int warp_sums[32];
+
+  const int b = blockIdx.x;
+  const int l = P.layer0 + blockIdx.y / NG;
+  const int g = blockIdx.y % NG;
+  const int tid = threadIdx.x;
+  const int seq = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b];
+  if (seq < 0 || seq >= P.s_max) {
+    if (tid == 0 && blockIdx.y == 0) set_dev_error(P.err, ER_EINVAL);
+    return;
+  }
+  const int c = P.meta[seq * 4 + 2];
+  const int p = P.meta[seq * 4 + 1] + P.p_add;
+  if (P.only_if_full && p != PEND) return;
+  if (c < 0 || c > BANK || p < 0 || p > PEND) {
+    if (tid == 0) set_dev_error(P.err, ER_ECAPACITY);
+    return;
+  }
+  const size_t gi = grp(seq, l, g, P.L);
+
+  for (int i = tid; i < NSORT; i += CT) {
+    uint64_t k = 0;
+    if (i < c) k = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
+    else if (i >= BANK && i < BANK + p)
+      k = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
+    key[i] = k;
+    src[i] = (uint16_t)i;
+  }
+  for (int i = tid; i < BANK + PEND; i += CT) flag[i] = 0;
+  __syncthreads();
+
+  // bitonic sort, descending
+  for (int k = 2; k <= NSORT; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const int i = ((tid & ~(j - 1)) << 1) | (tid & (j - 1));
+      const int m = i | j;
+      const uint64_t a = key[i], bb = key[m];
+      const bool desc = (i & k) == 0;
+      if (desc ? (a < bb) : (a > bb)) {
+        key[i] = bb;
+        key[m] = a;
+        const uint16_t t = src[i];
+        src[i] = src[m];
+        src[m] = t;
+      }
+      __syncthreads();
+    }
+  }
+
+  const int K = min(BANK, c + p);
+  if (tid < K) flag[src[tid]] = 1;
+  if (P.kept) {
+    int32_t* kp = P.kept + (((size_t)b * P.nlayers + (l - P.layer0)) * NG + g) * BANK;
+    kp[tid] = tid < K ? (int32_t)src[tid] : -1;
+  }
+  __syncthreads();
+
+  // evicted bank slots, ascending
+  int total_evict = 0;
+  const int ev = (tid < c && !flag[tid]) ? 1 : 0;
+  const int ev_rank = block_scan_excl(ev, warp_sums, &total_evict);
+  if (ev) evict_list[ev_rank] = (int16_t)tid;
+  // pending winners, ascending pending index
+  int total_win = 0;
+  const int wn = (tid < p && flag[BANK + tid]) ? 1 : 0;
+  const int w_rank = block_scan_excl(wn, warp_sums, &total_win);
+  __syncthreads();
+  if (wn) {
+    const int dst = w_rank < total_evict ? (int)evict_list[w_rank] : c + (w_rank - total_evict);
+    move_src[w_rank] = tid;
+    move_dst[w_rank] = dst;
+  }
+  __syncthreads();
+
+  // move rows: one warp per winner, 16 bytes per lane per row
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int w = warp; w < total_win; w += CT / 32) {
+    const int j = move_src[w], d = move_dst[w];
+    const uint4* sk = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + j) * D);
+    const uint4* sv = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + j) * D);
+    uint4* dk = reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + d) * D);
+    uint4* dv = reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + d) * D);
+    const uint4 a = sk[lane], a2 = sv[lane];
+    dk[lane] = a;
+    dv[lane] = a2;
+    if (lane == 0) {
+      P.bank_score[gi * BANK + d] = P.pend_score[gi * PEND + j];
+      P.bank_pos[gi * BANK + d] = P.pend_pos[gi * PEND + j];
+    }
+  }
+}
+
+__global__ void k_commit_finish(int32_t* meta, const int32_t* seq_ids, int n, int s_max) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= n) return;
+  const int s = seq_ids[b];
+  if (s < 0 || s >= s_max) return;
+  int32_t* m = meta + (size_t)s * 4;
+  m[2] = min(BANK, m[2] + m[1]);
+  m[1] = 0;
+}
+
+int launch_commit(const CommitParams& P, cudaStream_t st) {
+  if (P.n <= 0) return ER_OK;
+  k_commit<<<dim3(P.n, P.nlayers * NG), CT, 0, st>>>(P);
+  count_launches(1);
+  return launch_status();
+}
+
+// ------------------------------------------------------------- a4: append
+
+struct AppendParams {
+  uint16_t *pend_k, *pend_v;
+  float* pend_score;
+  int32_t* pend_pos;
+  const int32_t* meta;
+  const int32_t* seq_ids;
+  int n, s_max, L, layer;
+  const uint16_t *k, *v;
+  const float* s;
+  const int32_t* pos;
+  int32_t* err;
+};
+
+// block per sequence, warp w: rows k0..k3 (w < 4), v0..v3 (w >= 4)
+__global__ void __launch_bounds__(256) k_append(AppendParams P) {
+  const int b = blockIdx.x, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seq = P.seq_ids[b];
+  if (seq < 0 || seq >= P.s_max) {
+    if (threadIdx.x == 0) set_dev_error(P.err, ER_EINVAL);
+    return;
+  }
+  const int p = P.meta[seq * 4 + 1];
+  if (p >= PEND) {
+    if (threadIdx.x == 0) set_dev_error(P.err, ER_ECAPACITY);
+    return;
+  }
+  const int g = w & 3;
+  const size_t gi = grp(seq, P.layer, g, P.L);
+  const uint4* srcp =
+      reinterpret_cast<const uint4*>((w < 4 ? P.k : P.v) + ((size_t)b * NG + g) * D);
+  uint4* dstp = reinterpret_cast<uint4*>((w < 4 ? P.pend_k : P.pend_v) + (gi * PEND + p) * D);
+  dstp[lane] = srcp[lane];
+  if (w < 4 && lane == 0) {
+    P.pend_score[gi * PEND + p] = P.s[b * NG + g];
+    P.pend_pos[gi * PEND + p] = P.pos[b];
+  }
+}
+
+}  // namespace er
+
+using namespace er;
+
+extern "C" {
+
+int er_rma_commit(const er_state* st, int32_t layer, const int32_t* seq_ids, int32_t n,
+                  int32_t* kept, er_stream_t stream) {
+  if (!st || n < 0 || (n > 0 && !seq_ids) || layer < -1 || layer >= st->n_layers)
+    return ER_EINVAL;
+  if (n == 0) return ER_OK;
+  CommitParams P;
+  P.bank_k = st->bank_k; P.bank_v = st->bank_v;
+  P.pend_k = st->pend_k; P.pend_v = st->pend_v;
+  P.bank_score = st->bank_score; P.pend_score = st->pend_score;
+  P.bank_pos = st->bank_pos; P.pend_pos = st->pend_pos;
+  P.meta = st->meta; P.seq_ids = seq_ids; P.seq_fixed = -1;
+  P.n = n; P.s_max = st->s_max; P.L = st->n_layers;
+  P.layer0 = layer < 0 ? 0 : layer;
+  P.nlayers = layer < 0 ? st->n_layers : 1;
+  P.p_add = 0; P.only_if_full = 0;
+  P.kept = kept; P.err = st->dev_error;
+  cudaStream_t s = (cudaStream_t)stream;
+  int rc = launch_commit(P, s);
+  if (rc != ER_OK || layer >= 0) return rc;
+  k_commit_finish<<<(n + 127) / 128, 128, 0, s>>>(st->meta, seq_ids, n, st->s_max);
+  count_launches(1);
+  return launch_status();
+}
+
+int er_rma_append_pending(const er_state* st, int32_t layer, const int32_t* seq_ids, int32_t n,
+                          const er_bf16* k, const er_bf16* v, const float* s,
+                          const int32_t* pos, er_stream_t stream) {
+  if (!st || n < 0 || layer < 0 || layer >= st->n_layers) return ER_EINVAL;
+  if (n > 0 && (!seq_ids || !k || !v || !s || !pos)) return ER_EINVAL;
+  if (n == 0) return ER_OK;
+  AppendParams P;
+  P.pend_k = st->pend_k; P.pend_v = st->pend_v;
+  P.pend_score = st->pend_score; P.pend_pos = st->pend_pos;
+  P.meta = st->meta; P.seq_ids = seq_ids;
+  P.n = n; P.s_max = st->s_max; P.L = st->n_layers; P.layer = layer;
+  P.k = k; P.v = v; P.s = s; P.pos = pos; P.err = st->dev_error;
+  k_append<<<n, 256, 0, (cudaStream_t)stream>>>(P);
+  count_launches(1);
+  return launch_status();
+}
+
+}  // extern "C"

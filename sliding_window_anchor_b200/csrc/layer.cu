@@ -1,0 +1,167 @@
+// layer.cu — one SWA∥RMA layer step: decode (a1–a7) and a prefill chunk (a8).
+//
+// Order of a decode step (the reading fixed for this library, consistent with
+// EdgeRock-4B 开源：72 MiB 固定 KV §架构 and neodrop.ai §三段记忆): project, score,
+// norm + RoPE, write the window slot and append the pending record, read both
+// branches, o_proj, then commit this layer for sequences whose block the token
+// filled.  A prefill chunk writes its window rows only after every token read,
+// because the chunk's early tokens still see ring positions its late tokens
+// would overwrite.
+#include "common.cuh"
+#include "params.cuh"
+
+namespace er {
+
+int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
+                  cudaStream_t st);
+int launch_score(const float* w1, const float* w2, const uint16_t* x, int n, float* s,
+                 cudaStream_t st);
+int launch_post_proj(const PostParams& P, cudaStream_t st);
+int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
+                  cudaStream_t st);
+int launch_commit(const CommitParams& P, cudaStream_t st);
+size_t attend_part_floats(int nq);
+size_t attend_ml_floats(int nq);
+
+}  // namespace er
+
+namespace er {
+namespace {
+
+struct LayerWs {
+  uint16_t* proj;
+  float* s;
+  uint16_t *q_swa, *q_rma;
+  uint16_t *chunk_k, *chunk_v;
+  float *part_o, *part_ml;
+  uint16_t* o_sum;
+  size_t bytes;
+};
+
+LayerWs carve_ws(void* base, int nq, bool prefill) {
+  Carver c(base);
+  LayerWs w;
+  w.proj = c.take<uint16_t>((size_t)nq * QKV);
+  w.s = c.take<float>((size_t)nq * NG);
+  w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
+  w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
+  w.chunk_k = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
+  w.chunk_v = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
+  w.part_o = c.take<float>(attend_part_floats(nq));
+  w.part_ml = c.take<float>(attend_ml_floats(nq));
+  w.o_sum = c.take<uint16_t>((size_t)nq * OIN);
+  w.bytes = c.used();
+  return w;
+}
+
+bool weights_ok(const er_layer_weights* w) {
+  return w && w->w_qkv && w->w_o && w->q_norm_swa && w->k_norm_swa && w->q_norm_rma &&
+         w->k_norm_rma && w->w1 && w->w2;
+}
+
+// The chunk's window rows enter the ring after all of its reads.
+__global__ void k_ring_write(const uint16_t* chunk_k, const uint16_t* chunk_v, uint16_t* win_k,
+                             uint16_t* win_v, const int32_t* meta, int seq, int s_max, int L,
+                             int layer, int T) {
+  const int i = blockIdx.x, g = blockIdx.y, lane = threadIdx.x & 31, is_v = threadIdx.x >> 5;
+  if (seq < 0 || seq >= s_max) return;
+  const int t = meta[seq * 4 + 0] + i;
+  const size_t row = grp(seq, layer, g, L) * WIN + (size_t)(t % WIN);
+  const uint4* src =
+      reinterpret_cast<const uint4*>((is_v ? chunk_v : chunk_k) + ((size_t)g * T + i) * D);
+  uint4* dst = reinterpret_cast<uint4*>((is_v ? win_v : win_k) + row * D);
+  dst[lane] = src[lane];
+}
+
+int run_layer(const er_state* st, const er_layer_weights* w, int layer, const int32_t* seq_ids,
+              int seq_fixed, int nq, const uint16_t* x, uint16_t* out, void* ws, size_t ws_bytes,
+              cudaStream_t s) {
+  const bool prefill = seq_fixed >= 0;
+  LayerWs W = carve_ws(ws, nq, prefill);
+  if (ws_bytes < W.bytes) return ER_ECAPACITY;
+  int rc;
+  // a1: all six projections in one GEMM
+  if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
+  // a3: FP32 scores
+  if ((rc = launch_score(w->w1, w->w2, x, nq, W.s, s)) != ER_OK) return rc;
+  // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
+  PostParams pp{};
+  pp.proj = W.proj; pp.s = W.s; pp.nq = nq;
+  pp.gq_swa = w->q_norm_swa; pp.gk_swa = w->k_norm_swa;
+  pp.gq_rma = w->q_norm_rma; pp.gk_rma = w->k_norm_rma;
+  pp.q_swa = W.q_swa; pp.q_rma = W.q_rma;
+  pp.win_k = st->win_k; pp.win_v = st->win_v; pp.pend_k = st->pend_k; pp.pend_v = st->pend_v;
+  pp.pend_score = st->pend_score; pp.pend_pos = st->pend_pos;
+  pp.meta = st->meta; pp.seq_ids = seq_ids; pp.s_max = st->s_max; pp.L = st->n_layers;
+  pp.layer = layer; pp.prefill = prefill ? 1 : 0; pp.seq_fixed = seq_fixed;
+  pp.chunk_k = W.chunk_k; pp.chunk_v = W.chunk_v; pp.err = st->dev_error;
+  if ((rc = launch_post_proj(pp, s)) != ER_OK) return rc;
+  // a5: both reads, merged into bf16(o_swa + o_rma)
+  AttendParams ap{};
+  ap.win_k = st->win_k; ap.win_v = st->win_v; ap.bank_k = st->bank_k; ap.bank_v = st->bank_v;
+  ap.pend_k = st->pend_k; ap.pend_v = st->pend_v; ap.meta = st->meta; ap.seq_ids = seq_ids;
+  ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
+  ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
+  ap.prefill = prefill ? 1 : 0; ap.seq_fixed = seq_fixed;
+  ap.chunk_k = W.chunk_k; ap.chunk_v = W.chunk_v;
+  ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.err = st->dev_error;
+  if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, s)) != ER_OK) return rc;
+  // a6: shared o_proj
+  if ((rc = gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s)) != ER_OK) return rc;
+  if (prefill) {
+    k_ring_write<<<dim3(nq, NG), 64, 0, s>>>(W.chunk_k, W.chunk_v, st->win_k, st->win_v,
+                                             st->meta, seq_fixed, st->s_max, st->n_layers,
+                                             layer, nq);
+    count_launches(1);
+    if ((rc = launch_status()) != ER_OK) return rc;
+  }
+  // a7: commit this layer where the block is now full (decided on the device)
+  CommitParams cp{};
+  cp.bank_k = st->bank_k; cp.bank_v = st->bank_v; cp.pend_k = st->pend_k; cp.pend_v = st->pend_v;
+  cp.bank_score = st->bank_score; cp.pend_score = st->pend_score;
+  cp.bank_pos = st->bank_pos; cp.pend_pos = st->pend_pos;
+  cp.meta = st->meta; cp.seq_ids = seq_ids; cp.seq_fixed = seq_fixed;
+  cp.n = prefill ? 1 : nq; cp.s_max = st->s_max; cp.L = st->n_layers;
+  cp.layer0 = layer; cp.nlayers = 1; cp.p_add = prefill ? nq : 1; cp.only_if_full = 1;
+  cp.kept = nullptr; cp.err = st->dev_error;
+  return launch_commit(cp, s);
+}
+
+}  // namespace
+}  // namespace er
+
+using namespace er;
+
+extern "C" {
+
+size_t er_decode_workspace_bytes(int32_t B) {
+  if (B < 0) return 0;
+  return carve_ws(nullptr, B, false).bytes;
+}
+
+size_t er_prefill_workspace_bytes(int32_t T) {
+  if (T < 0 || T > PEND) return 0;
+  return carve_ws(nullptr, T, true).bytes;
+}
+
+int er_swa_rma_decode(const er_state* st, const er_layer_weights* w, int32_t layer,
+                      const int32_t* seq_ids, int32_t B, const er_bf16* x, er_bf16* out,
+                      void* ws, size_t ws_bytes, er_stream_t stream) {
+  if (!st || B < 0 || layer < 0 || layer >= st->n_layers) return ER_EINVAL;
+  if (B == 0) return ER_OK;
+  if (B > st->s_max) return ER_ECAPACITY;
+  if (!weights_ok(w) || !seq_ids || !x || !out || !ws) return ER_EINVAL;
+  return run_layer(st, w, layer, seq_ids, -1, B, x, out, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+int er_swa_rma_prefill_chunk(const er_state* st, const er_layer_weights* w, int32_t layer,
+                             int32_t seq_id, const er_bf16* x, int32_t T, er_bf16* out,
+                             void* ws, size_t ws_bytes, er_stream_t stream) {
+  if (!st || layer < 0 || layer >= st->n_layers || T < 1 || T > PEND) return ER_EINVAL;
+  if (seq_id < 0 || seq_id >= st->s_max) return ER_EINVAL;
+  if (!weights_ok(w) || !x || !out || !ws) return ER_EINVAL;
+  return run_layer(st, w, layer, nullptr, seq_id, T, x, out, ws, ws_bytes,
+                   (cudaStream_t)stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// norm_rope.cu — a2 (q/k RMS-norm + partial RoPE) and the a4 state writes
+// that follow the projections.
+//
+// EdgeRock-4B 开源：72 MiB 固定 KV, §架构：递归、局部窗口与记忆锚点三件套:
+// q and k carry a learned RMS-norm; rotary embedding covers 64 of the 256
+// dims with base 1e7; v is neither normed nor rotated.  Pairing (i, i+32),
+// eps 1e-6 and the directly applied gain are this library's reading.
+//
+// One warp owns one 256-wide head vector, 8 BF16 values per lane (one 16-byte
+// load); lanes 0..7 hold the rotated dims and exchange pairs with xor 4.  The
+// rotation angle pos * 1e7^(-2i/64) is formed and reduced in float64 so that
+// positions up to 2^18 keep full angle accuracy; the rotation itself is fp32.
+#include "common.cuh"
+#include "params.cuh"
+
+namespace er {
+namespace {
+
+__device__ __forceinline__ void load8(const uint16_t* src, float v[8]) {
+  uint4 w = *reinterpret_cast<const uint4*>(src);
+  v[0] = bf_lo(w.x); v[1] = bf_hi(w.x); v[2] = bf_lo(w.y); v[3] = bf_hi(w.y);
+  v[4] = bf_lo(w.z); v[5] = bf_hi(w.z); v[6] = bf_lo(w.w); v[7] = bf_hi(w.w);
+}
+
+__device__ __forceinline__ void store8(uint16_t* dst, const float v[8]) {
+  uint4 w;
+  w.x = pack_bf2(v[0], v[1]); w.y = pack_bf2(v[2], v[3]);
+  w.z = pack_bf2(v[4], v[5]); w.w = pack_bf2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(dst) = w;
+}
+
+// y = x / sqrt(mean(x^2) + 1e-6) * gain, then rotate (i, i+32), i < 32.
+__device__ __forceinline__ void norm_rope_lane(float v[8], const uint16_t* gain, int32_t pos,
+                                               int lane) {
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss * (1.0f / D) + 1e-6f);
+  float g[8];
+  load8(gain + lane * 8, g);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = (v[e] * inv) * g[e];
+  float partner[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, v[e], 4);
+  if (lane < 8) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = (lane & 3) * 8 + e;  // frequency index 0..31
+      const double inv_freq = pow(1.0e7, -2.0 * (double)i / (double)ROPE);
+      double sn, cs;
+      sincos((double)pos * inv_freq, &sn, &cs);
+      const float c = (float)cs, s = (float)sn;
+      if (lane < 4) v[e] = v[e] * c - partner[e] * s;        // dim i:    a cos - b sin
+      else v[e] = v[e] * c + partner[e] * s;                 // dim i+32: b cos + a sin
+    }
+  }
+}
+
+__global__ void k_norm_rope(const uint16_t* x, uint16_t* y, int64_t n_rows, const uint16_t* gain,
+                            const int32_t* pos) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= n_rows) return;
+  float v[8];
+  load8(x + row * D + lane * 8, v);
+  norm_rope_lane(v, gain, pos[row], lane);
+  store8(y + row * D + lane * 8, v);
+}
+
+}  // namespace
+
+
+// Grid (nq, 6) x 256 threads: warp slot hs = 0..47 covers, per token,
+// q_swa 0..15 | k_swa 16..19 | v_swa 20..23 | q_rma 24..39 | k_rma 40..43 | v_rma 44..47.
+__global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
+  const int lane = threadIdx.x & 31;
+  const int hs = blockIdx.y * 8 + (threadIdx.x >> 5);
+  const int qi = blockIdx.x;
+  const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
+  if (seq < 0 || seq >= P.s_max) {
+    if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);
+    return;
+  }
+  const int32_t pos0 = P.meta[seq * 4 + 0];
+  const int32_t pend0 = P.meta[seq * 4 + 1];
+  const int32_t t = pos0 + (P.prefill ? qi : 0);
+  const int p_idx = pend0 + (P.prefill ? qi : 0);
+  const bool state_ok = p_idx < PEND;
+  if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
+
+  int col;
+  const uint16_t* gain = nullptr;
+  if (hs < 16) { col = OFF_Q_SWA + hs * D; gain = P.gq_swa; }
+  else if (hs < 20) { col = OFF_K_SWA + (hs - 16) * D; gain = P.gk_swa; }
+  else if (hs < 24) { col = OFF_V_SWA + (hs - 20) * D; }
+  else if (hs < 40) { col = OFF_Q_RMA + (hs - 24) * D; gain = P.gq_rma; }
+  else if (hs < 44) { col = OFF_K_RMA + (hs - 40) * D; gain = P.gk_rma; }
+  else { col = OFF_V_RMA + (hs - 44) * D; }
+
+  float v[8];
+  load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
+  if (gain) norm_rope_lane(v, gain, t, lane);
+
+  uint16_t* dst = nullptr;
+  if (hs < 16) {
+    dst = P.q_swa + ((size_t)qi * NH + hs) * D;
+  } else if (hs < 24) {
+    const int g = (hs < 20) ? hs - 16 : hs - 20;
+    const bool is_k = hs < 20;
+    if (P.prefill) {
+      dst = (is_k ? P.chunk_k : P.chunk_v) + ((size_t)g * P.nq + qi) * D;
+    } else {
+      const size_t row = grp(seq, P.layer, g, P.L) * WIN + (size_t)(t % WIN);
+      dst = (is_k ? P.win_k : P.win_v) + row * D;
+    }
+  } else if (hs < 40) {
+    dst = P.q_rma + ((size_t)qi * NH + (hs - 24)) * D;
+  } else {
+    if (!state_ok) return;
+    const int g = (hs < 44) ? hs - 40 : hs - 44;
+    const size_t gi = grp(seq, P.layer, g, P.L);
+    dst = ((hs < 44) ? P.pend_k : P.pend_v) + (gi * PEND + p_idx) * D;
+    if (hs < 44 && lane == 0) {
+      P.pend_score[gi * PEND + p_idx] = P.s[qi * NG + g];
+      P.pend_pos[gi * PEND + p_idx] = t;
+    }
+  }
+  store8(dst + lane * 8, v);
+}
+
+int launch_post_proj(const PostParams& P, cudaStream_t st) {
+  if (P.nq <= 0) return ER_OK;
+  k_post_proj<<<dim3(P.nq, 6), 256, 0, st>>>(P);
+  count_launches(1);
+  return launch_status();
+}
+
+}  // namespace er
+
+using namespace er;
+
+extern "C" int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, const er_bf16* gain,
+                               const int32_t* pos, er_stream_t stream) {
+  if (n_rows < 0 || (n_rows > 0 && (!x || !y || !gain || !pos))) return ER_EINVAL;
+  if (n_rows == 0) return ER_OK;
+  const int64_t blocks = (n_rows + 7) / 8;
+  if (blocks > 0x7FFFFFFF) return ER_EINVAL;
+  k_norm_rope<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(x, y, n_rows, gain, pos);
+  count_launches(1);
+  return launch_status();
+}

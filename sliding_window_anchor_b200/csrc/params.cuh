@@ -1,0 +1,62 @@
+// params.cuh — launch parameters shared between the kernels and the layer
+// orchestration (layer.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace er {
+
+struct PostParams {
+  const uint16_t* proj;  // [nq][12288]
+  const float* s;        // [nq][4]
+  int nq;
+  const uint16_t *gq_swa, *gk_swa, *gq_rma, *gk_rma;
+  uint16_t *q_swa, *q_rma;  // [nq][16][256] each
+  uint16_t *win_k, *win_v, *pend_k, *pend_v;
+  float* pend_score;
+  int32_t* pend_pos;
+  const int32_t* meta;
+  const int32_t* seq_ids;
+  int s_max, L, layer;
+  int prefill;                 // 0: token b of sequence seq_ids[b]; 1: token i of seq_fixed
+  int seq_fixed;
+  uint16_t *chunk_k, *chunk_v; // prefill: [4][nq][256] window rows of the chunk
+  int32_t* err;
+};
+
+struct AttendParams {
+  const uint16_t *win_k, *win_v, *bank_k, *bank_v, *pend_k, *pend_v;
+  const int32_t* meta;
+  const int32_t* seq_ids;
+  int s_max, L, layer;
+  const uint16_t* q_swa;  // [nq][16][256], normed and rotated
+  const uint16_t* q_rma;  // [nq][16][256]
+  int nq;
+  int prefill;        // 0: query b = sequence seq_ids[b] at meta pos; 1: token b of seq_fixed
+  int seq_fixed;
+  const uint16_t *chunk_k, *chunk_v;  // prefill: [4][nq][256]
+  int splits;
+  float* part_o;   // [items][4][256]
+  float* part_ml;  // [items][4][2]
+  int32_t* err;
+};
+
+struct CommitParams {
+  uint16_t *bank_k, *bank_v;
+  const uint16_t *pend_k, *pend_v;
+  float* bank_score;
+  const float* pend_score;
+  int32_t* bank_pos;
+  const int32_t* pend_pos;
+  const int32_t* meta;
+  const int32_t* seq_ids;  // [n], or ignored when seq_fixed >= 0 (then n == 1)
+  int seq_fixed;
+  int n, s_max, L;
+  int layer0, nlayers;
+  int p_add;         // pending records = meta.pend + p_add
+  int only_if_full;  // commit only when that count is 256
+  int32_t* kept;     // optional [n][nlayers][4][1024]
+  int32_t* err;
+};
+
+}  // namespace er

@@ -1,0 +1,255 @@
+// state.cu — state carving, per-sequence metadata kernels, error word,
+// launch accounting and the optional timing of the read kernel.
+//
+// The state's capacities are hard limits (EdgeRock-4B 开源：72 MiB 固定 KV,
+// §72 MiB 是怎么算出来的): window 1024, bank 1024 and pending 256 rows per
+// (layer, group), K and V in BF16, so a sequence holds 72 MiB at 8 layers
+// whatever its length.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace er {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launches(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+int launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? ER_OK : ER_ECUDA;
+}
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+namespace {
+
+struct StateLayout {
+  size_t win, bank, pend, bscore, pscore, bpos, ppos, meta, err, total;
+};
+
+bool layout_of(int32_t s_max, int32_t n_layers, StateLayout* L) {
+  if (s_max < 1 || s_max > (1 << 20) || n_layers < 1 || n_layers > ER_MAX_LAYERS) return false;
+  Carver c(nullptr);
+  size_t g = (size_t)s_max * n_layers * NG;
+  L->win = (size_t)c.take<uint16_t>(g * WIN * D);
+  size_t win_v = (size_t)c.take<uint16_t>(g * WIN * D);
+  L->bank = (size_t)c.take<uint16_t>(g * BANK * D);
+  size_t bank_v = (size_t)c.take<uint16_t>(g * BANK * D);
+  L->pend = (size_t)c.take<uint16_t>(g * PEND * D);
+  size_t pend_v = (size_t)c.take<uint16_t>(g * PEND * D);
+  (void)win_v; (void)bank_v; (void)pend_v;
+  L->bscore = (size_t)c.take<float>(g * BANK);
+  L->pscore = (size_t)c.take<float>(g * PEND);
+  L->bpos = (size_t)c.take<int32_t>(g * BANK);
+  L->ppos = (size_t)c.take<int32_t>(g * PEND);
+  L->meta = (size_t)c.take<int32_t>((size_t)s_max * 4);
+  L->err = (size_t)c.take<int32_t>(64);
+  L->total = c.used();
+  return true;
+}
+
+__global__ void k_state_init(int32_t* meta, const int32_t* seq_ids, int n, int s_max,
+                             int32_t* err) {
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= n) return;
+  int s = seq_ids[b];
+  if (s < 0 || s >= s_max) {
+    set_dev_error(err, ER_EINVAL);
+    return;
+  }
+  meta[s * 4 + 0] = 0;
+  meta[s * 4 + 1] = 0;
+  meta[s * 4 + 2] = 0;
+  meta[s * 4 + 3] = 0;
+}
+
+// End of a step of T tokens: the position moves on; a block that reached 256
+// was committed by every layer during the step and empties.
+__global__ void k_advance(int32_t* meta, const int32_t* seq_ids, int n, int T, int s_max,
+                          int32_t* err) {
+  int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= n) return;
+  int s = seq_ids[b];
+  if (s < 0 || s >= s_max) {
+    set_dev_error(err, ER_EINVAL);
+    return;
+  }
+  int32_t* m = meta + (size_t)s * 4;
+  int pend = m[1] + T;
+  if (pend > PEND) {
+    set_dev_error(err, ER_ECAPACITY);
+    return;
+  }
+  m[0] += T;
+  if (pend == PEND) {
+    m[1] = 0;
+    m[2] = min(BANK, m[2] + PEND);
+  } else {
+    m[1] = pend;
+  }
+}
+
+// ------------------------------------------------------ read-kernel timing
+struct ProfileState {
+  std::mutex mu;
+  bool enabled = false;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending;
+  std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pool;
+  double ms = 0.0;
+  int64_t launches = 0;
+};
+ProfileState& prof() {
+  static ProfileState p;
+  return p;
+}
+
+}  // namespace
+
+bool profile_begin(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t>* ev) {
+  ProfileState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  if (!p.enabled) return false;
+  if (p.pool.empty()) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess) return false;
+    if (cudaEventCreate(&b) != cudaSuccess) {
+      cudaEventDestroy(a);
+      return false;
+    }
+    p.pool.push_back({a, b});
+  }
+  *ev = p.pool.back();
+  p.pool.pop_back();
+  cudaEventRecord(ev->first, st);
+  return true;
+}
+
+void profile_end(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t> ev) {
+  ProfileState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  cudaEventRecord(ev.second, st);
+  p.pending.push_back(ev);
+}
+
+}  // namespace er
+
+using namespace er;
+
+extern "C" {
+
+size_t er_state_bytes(int32_t s_max, int32_t n_layers) {
+  StateLayout L;
+  return layout_of(s_max, n_layers, &L) ? L.total : 0;
+}
+
+int er_state_carve(void* base, size_t bytes, int32_t s_max, int32_t n_layers, er_state* out) {
+  StateLayout L;
+  if (!base || !out || !layout_of(s_max, n_layers, &L)) return ER_EINVAL;
+  if (((uintptr_t)base & 255u) != 0 || bytes < L.total) return ER_EINVAL;
+  char* b = (char*)base;
+  size_t g = (size_t)s_max * n_layers * NG;
+  out->win_k = (er_bf16*)(b + L.win);
+  out->win_v = out->win_k + g * WIN * D;
+  out->bank_k = (er_bf16*)(b + L.bank);
+  out->bank_v = out->bank_k + g * BANK * D;
+  out->pend_k = (er_bf16*)(b + L.pend);
+  out->pend_v = out->pend_k + g * PEND * D;
+  out->bank_score = (float*)(b + L.bscore);
+  out->pend_score = (float*)(b + L.pscore);
+  out->bank_pos = (int32_t*)(b + L.bpos);
+  out->pend_pos = (int32_t*)(b + L.ppos);
+  out->meta = (int32_t*)(b + L.meta);
+  out->dev_error = (int32_t*)(b + L.err);
+  out->s_max = s_max;
+  out->n_layers = n_layers;
+  return ER_OK;
+}
+
+int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stream_t stream) {
+  if (!st || !st->meta || (n > 0 && !seq_ids) || n < 0) return ER_EINVAL;
+  if (n == 0) return ER_OK;
+  k_state_init<<<(n + 127) / 128, 128, 0, (cudaStream_t)stream>>>(st->meta, seq_ids, n,
+                                                                   st->s_max, st->dev_error);
+  count_launches(1);
+  return launch_status();
+}
+
+int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
+               er_stream_t stream) {
+  if (!st || !st->meta || (n > 0 && !seq_ids) || n < 0 || T < 1 || T > PEND) return ER_EINVAL;
+  if (n == 0) return ER_OK;
+  k_advance<<<(n + 127) / 128, 128, 0, (cudaStream_t)stream>>>(st->meta, seq_ids, n, T,
+                                                               st->s_max, st->dev_error);
+  count_launches(1);
+  return launch_status();
+}
+
+int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream) {
+  if (!st || !st->dev_error || !code) return ER_EINVAL;
+  int32_t h = 0;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&h, st->dev_error, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return ER_ECUDA;
+  if (cudaMemsetAsync(st->dev_error, 0, sizeof(int32_t), s) != cudaSuccess) return ER_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ER_ECUDA;
+  *code = h;
+  return h == 0 ? ER_OK : ER_EDEVICE;
+}
+
+const char* er_error_string(int code) {
+  switch (code) {
+    case ER_OK: return "ok";
+    case ER_EINVAL: return "invalid argument";
+    case ER_ECAPACITY: return "capacity exceeded";
+    case ER_ECUDA: return "CUDA error";
+    case ER_EDEVICE: return "device-side error recorded";
+    case ER_ETIMEOUT: return "bounded device wait timed out";
+    default: return "unknown error";
+  }
+}
+
+uint64_t er_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int er_profile_enable(int enable) {
+  ProfileState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  p.enabled = enable != 0;
+  return ER_OK;
+}
+
+int er_profile_read(double* ms_total, int64_t* launches, int reset) {
+  ProfileState& p = prof();
+  std::lock_guard<std::mutex> g(p.mu);
+  for (auto& ev : p.pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(ev.second) != cudaSuccess) return ER_ECUDA;
+    if (cudaEventElapsedTime(&ms, ev.first, ev.second) != cudaSuccess) return ER_ECUDA;
+    p.ms += ms;
+    p.launches += 1;
+    p.pool.push_back(ev);
+  }
+  p.pending.clear();
+  if (ms_total) *ms_total = p.ms;
+  if (launches) *launches = p.launches;
+  if (reset) {
+    p.ms = 0.0;
+    p.launches = 0;
+  }
+  return ER_OK;
+}
+
+}  // extern "C"

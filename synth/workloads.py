@@ -102,8 +102,11 @@ def window_positions(t0: int, device="cpu") -> torch.Tensor:
     return (t0 - WIN + torch.remainder(s - t0, WIN)).to(torch.int32).to(device)
 
 
-def pend_fill(seed: int, mode: str, seqs, device="cpu") -> torch.Tensor:
+def pend_fill(seed: int, mode, seqs, device="cpu") -> torch.Tensor:
+    """Pending fill per sequence: "zero", "full", "uniform" (U{0..255}), or explicit values."""
     seqs = list(seqs)
+    if not isinstance(mode, str):
+        return torch.as_tensor(mode, dtype=torch.int32).reshape(len(seqs)).to(device)
     if mode == "zero":
         return torch.zeros(len(seqs), dtype=torch.int32, device=device)
     if mode == "full":

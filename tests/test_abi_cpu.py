@@ -1,0 +1,103 @@
+"""The C-ABI library builds, loads and exports every declared symbol (CPU only).
+
+Only host-side logic is exercised here: sizes, carving, argument checks that
+return before anything is enqueued.  No kernel is launched.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sliding_window_anchor_b200 import build, _lib
+    build.build()
+    return _lib.lib()
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(er_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    from sliding_window_anchor_b200 import _lib
+    assert set(names) == set(_lib.EXPORTS)
+
+
+def test_state_bytes_and_carve(L):
+    from sliding_window_anchor_b200._lib import CState
+    n = L.er_state_bytes(2, 8)
+    kv = 2 * 75497472
+    meta = 2 * 8 * 4 * (1024 + 256) * 8
+    assert kv + meta <= n <= kv + meta + 64 * 1024
+    assert L.er_state_bytes(0, 8) == 0 and L.er_state_bytes(1, 9) == 0
+    st = CState()
+    fake = 1 << 40  # carving only computes pointers
+    assert L.er_state_carve(ctypes.c_void_p(fake), n, 2, 8, ctypes.byref(st)) == 0
+    assert st.win_v - st.win_k == 2 * 8 * 4 * 1024 * 256 * 2
+    assert st.pend_v - st.pend_k == 2 * 8 * 4 * 256 * 256 * 2
+    for f in ("win_k", "bank_k", "pend_k", "bank_score", "pend_score", "bank_pos", "pend_pos",
+              "meta", "dev_error"):
+        assert getattr(st, f) % 256 == 0
+    assert st.dev_error + 64 * 4 <= fake + n
+    assert L.er_state_carve(ctypes.c_void_p(fake), n - 1, 2, 8, ctypes.byref(st)) == -1
+    assert L.er_state_carve(ctypes.c_void_p(fake + 8), n, 2, 8, ctypes.byref(st)) == -1
+
+
+def test_workspace_sizes_monotone(L):
+    prev = 0
+    for B in (1, 2, 8, 64, 512):
+        n = L.er_decode_workspace_bytes(B)
+        assert n > prev
+        prev = n
+    assert L.er_prefill_workspace_bytes(1) > 0 and L.er_prefill_workspace_bytes(0) == 0
+    assert L.er_prefill_workspace_bytes(257) == 0
+    assert L.er_attend_workspace_bytes(512) < L.er_decode_workspace_bytes(512)
+
+
+def test_host_validation_rejects_before_enqueue(L):
+    from sliding_window_anchor_b200._lib import CState, CWeights
+    st = CState()
+    n = L.er_state_bytes(4, 8)
+    L.er_state_carve(ctypes.c_void_p(1 << 40), n, 4, 8, ctypes.byref(st))
+    w = CWeights()
+    nul = None
+    # null state / weights / pointers, bad layer, bad sizes: all return before any launch
+    assert L.er_swa_rma_decode(None, ctypes.byref(w), 0, nul, 1, nul, nul, nul, 0, nul) == -1
+    assert L.er_swa_rma_decode(ctypes.byref(st), ctypes.byref(w), 0, nul, 1, nul, nul, nul, 0,
+                               nul) == -1
+    assert L.er_swa_rma_decode(ctypes.byref(st), ctypes.byref(w), 8, nul, 1, nul, nul, nul, 0,
+                               nul) == -1
+    assert L.er_swa_rma_decode(ctypes.byref(st), ctypes.byref(w), 0, nul, 5, nul, nul, nul, 0,
+                               nul) == -2  # batch above the state's capacity
+    assert L.er_swa_rma_prefill_chunk(ctypes.byref(st), ctypes.byref(w), 0, 0, nul, 257, nul,
+                                      nul, 0, nul) == -1
+    assert L.er_swa_rma_prefill_chunk(ctypes.byref(st), ctypes.byref(w), 0, 4, nul, 16, nul,
+                                      nul, 0, nul) == -1
+    assert L.er_rma_commit(ctypes.byref(st), 8, nul, 1, nul, nul) == -1
+    assert L.er_rma_commit(ctypes.byref(st), -2, nul, 1, nul, nul) == -1
+    assert L.er_rma_append_pending(ctypes.byref(st), 0, nul, 1, nul, nul, nul, nul, nul) == -1
+    assert L.er_advance(ctypes.byref(st), nul, 1, 0, nul) == -1
+    assert L.er_advance(ctypes.byref(st), nul, 1, 257, nul) == -1
+    assert L.er_rma_score(None, nul, 1, nul, nul) == -1
+    assert L.er_qk_norm_rope(nul, nul, 4, nul, nul, nul) == -1
+    # empty work is fine and launches nothing
+    before = L.er_launch_count()
+    assert L.er_rma_score(ctypes.byref(w), nul, 0, nul, nul) == 0
+    assert L.er_qk_norm_rope(nul, nul, 0, nul, nul, nul) == 0
+    assert L.er_launch_count() == before
+    assert L.er_error_string(-2) == b"capacity exceeded"

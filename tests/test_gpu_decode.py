@@ -1,0 +1,197 @@
+"""GPU parity of whole decode steps (a1–a7) and prefill chunks (a8) against the oracle.
+
+Workloads follow the synthetic recipe of synth/workloads.py.  The device
+seeds its own state (its norm/RoPE kernel) and the oracle seeds its own, from
+the same generator numbers.  Bars: the stated |Δ| <= 1e-2 + 1e-2·|oracle| on
+every layer output, and kept anchor sets equal except where two records'
+scores differ by less than 1e-5 relative at the keep/evict boundary.
+"""
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+import torch
+
+import oracle
+from synth import workloads as wl
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sab():
+    from sliding_window_anchor_b200 import build
+    build.build()
+    import sliding_window_anchor_b200 as m
+    return m
+
+
+def _kept_sets_agree(gpu_row, ost_row, n_layers):
+    """Bank position sets per (layer, group) match, up to near-ties at the boundary."""
+    for l in range(n_layers):
+        for g in range(4):
+            c = int(ost_row["meta"][2])
+            gp = set(gpu_row["bank_pos"][l, g, :c].tolist())
+            op = set(ost_row["bank_pos"][l, g, :c].tolist())
+            if gp == op:
+                continue
+            # records only one side kept must sit at the boundary score within 1e-5 relative
+            ob = ost_row["bank_score"][l, g, :c].double()
+            smin = float(ob.min())
+            for side, pos_set, other, scores, poss in (
+                    ("gpu", gp, op, gpu_row["bank_score"][l, g, :c], gpu_row["bank_pos"][l, g, :c]),
+                    ("oracle", op, gp, ost_row["bank_score"][l, g, :c], ost_row["bank_pos"][l, g, :c])):
+                for pos in pos_set - other:
+                    s = float(scores[(poss == pos).nonzero()[0, 0]])
+                    assert abs(s - smin) <= 1e-5 * max(abs(smin), 1e-30) + 1e-12, (side, l, g, pos)
+    return True
+
+
+def _run_oracle_seq(ow_list, ost, row, steps, layers, seed, gseq, x_of):
+    outs = {}
+    for step in range(steps):
+        for l in layers:
+            outs[(step, l)] = ost.decode_layer(ow_list[l], l, row, x_of(step, l, gseq))
+        ost.advance(row)
+    return outs
+
+
+def test_decode_single_layer_256_steps_with_commit(sab):
+    """B=1, one layer, state at 4096, empty pending: 256 steps, one commit at the last."""
+    cfg, seed = wl.CONFIGS[0], wl.seed_of(0)
+    L = cfg["n_layers"]
+    ow, wdict = H.oracle_weights(seed, 0)
+    gw, gdict = H.gpu_weights(seed, 0)
+    ost = oracle.OracleState(1, L)
+    H.seed_oracle_state(ost, [0], L, cfg["t0"], cfg["pend"], seed, [wdict])
+    st = sab.State(1, L)
+    H.seed_gpu_state(st, L, cfg["t0"], cfg["pend"], seed, [gdict])
+    ws = torch.empty(sab.decode_workspace_bytes(1), dtype=torch.uint8, device="cuda")
+    gouts = []
+    for step in range(cfg["steps"]):
+        x = wl.make_x(seed, 0, step, [0], device="cuda")
+        gouts.append(sab.swa_rma_decode(st, gw, 0, [0], x, ws=ws).cpu())
+        sab.advance(st, [0])
+    assert sab.last_device_error(st) == 0
+    worst = 0.0
+    for step in range(cfg["steps"]):
+        ref = ost.decode_layer(ow, 0, 0, wl.make_x(seed, 0, step, [0])[0])
+        ost.advance(0)
+        assert H.tol_ok(gouts[step][0], ref), (step, H.max_err(gouts[step][0], ref))
+        worst = max(worst, H.max_err(gouts[step][0], ref) / float(ref.double().abs().max()))
+    print(f"config0 worst |Δ|/max|ref| = {worst:.3e}")
+    assert worst < 2e-2
+    grow, orow = H.download_row(st, 0), {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
+    assert torch.equal(grow["meta"], orow["meta"])
+    assert int(orow["meta"][1]) == 0 and int(orow["meta"][0]) == cfg["t0"] + 256
+    _kept_sets_agree(grow, orow, L)
+
+
+@pytest.mark.parametrize("cfg_index,steps", [(2, 4), (3, 2)])
+def test_decode_batched_sampled_sequences(sab, cfg_index, steps):
+    """Full batch on the device (B=64 or 512, 8 layers, t0=32768, random fills);
+    the oracle follows two sampled sequences, one of which commits first."""
+    cfg, seed = wl.CONFIGS[cfg_index], wl.seed_of(cfg_index)
+    B, L = cfg["B"], cfg["n_layers"]
+    gws, gdicts = zip(*[H.gpu_weights(seed, l) for l in range(L)])
+    st = sab.State(B, L)
+    fills = H.seed_gpu_state(st, L, cfg["t0"], cfg["pend"], seed, list(gdicts)).cpu()
+    ws = torch.empty(sab.decode_workspace_bytes(B), dtype=torch.uint8, device="cuda")
+    ids = torch.arange(B, dtype=torch.int32, device="cuda")
+    gouts = {}
+    for step in range(steps):
+        for l in range(L):
+            x = wl.make_x(seed, l, step, range(B), device="cuda")
+            gouts[(step, l)] = sab.swa_rma_decode(st, gws[l], l, ids, x, ws=ws)
+        sab.advance(st, ids)
+    assert sab.last_device_error(st) == 0
+    sampled = [int(torch.argmax(fills)), 1 if int(torch.argmax(fills)) != 1 else 2]
+    assert int(fills[sampled[0]]) + steps >= 256, "the sampled set must include a commit"
+
+    ows, wdicts = zip(*[H.oracle_weights(seed, l) for l in range(L)])
+
+    def run(gseq):
+        ost = oracle.OracleState(1, L)
+        H.seed_oracle_state(ost, [gseq], L, cfg["t0"], cfg["pend"], seed, list(wdicts))
+        x_of = lambda step, l, s: wl.make_x(seed, l, step, [s])[0]
+        return ost, _run_oracle_seq(ows, ost, 0, steps, range(L), seed, gseq, x_of)
+
+    with ThreadPoolExecutor(len(sampled)) as ex:
+        results = list(ex.map(run, sampled))
+    for gseq, (ost, outs) in zip(sampled, results):
+        for (step, l), ref in outs.items():
+            got = gouts[(step, l)][gseq].cpu()
+            assert H.tol_ok(got, ref), (gseq, step, l, H.max_err(got, ref))
+        grow = H.download_row(st, gseq)
+        orow = {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
+        assert torch.equal(grow["meta"], orow["meta"])
+        _kept_sets_agree(grow, orow, L)
+
+
+def test_prefill_chunks_match_oracle_and_decode(sab):
+    """Seeded state at 4096 (the ring wraps for every query), one layer: a full chunk of
+    256 (fills the block, commits) then a ragged chunk of 37."""
+    seed = wl.seed_of(4)
+    L = 1
+    ow, wdict = H.oracle_weights(seed, 0)
+    gw, gdict = H.gpu_weights(seed, 0)
+    ost = oracle.OracleState(1, L)
+    H.seed_oracle_state(ost, [0], L, 4096, "zero", seed, [wdict])
+    st = sab.State(2, L)
+    H.seed_gpu_state(st, L, 4096, [0, 0], seed, [gdict])
+    # row 1 replays the same stream token by token through the decode path
+    for n in oracle.OracleState.ARRAYS:
+        getattr(st, n)[1].copy_(getattr(st, n)[0])
+    for ci, T in enumerate((256, 37)):
+        x = wl.make_x(seed, 0, 1000 + ci, range(T), big_every=4096, first_pos=4096)
+        got = sab.swa_rma_prefill_chunk(st, gw, 0, 0, x.cuda())
+        sab.advance(st, [0], T)
+        dec = []
+        for i in range(T):
+            dec.append(sab.swa_rma_decode(st, gw, 0, [1], x[i:i + 1].cuda()))
+            sab.advance(st, [1])
+        dec = torch.cat(dec).cpu()
+        ref = ost.prefill_chunk(ow, 0, 0, x)
+        ost.advance(0, T)
+        assert H.tol_ok(got.cpu(), ref), (ci, H.max_err(got.cpu(), ref))
+        assert H.tol_ok(got.cpu(), dec), (ci, H.max_err(got.cpu(), dec))
+    assert sab.last_device_error(st) == 0
+    g0, g1 = H.download_row(st, 0), H.download_row(st, 1)
+    orow = {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
+    assert torch.equal(g0["meta"], orow["meta"]) and torch.equal(g1["meta"], orow["meta"])
+    _kept_sets_agree(g0, orow, L)
+    _kept_sets_agree(g1, orow, L)
+
+
+def test_snapshot_restore_is_bit_identical(sab):
+    """The state is flat fixed-size memory: a copy taken mid-stream replays exactly."""
+    seed = 77
+    gw, gdict = H.gpu_weights(seed, 0)
+    st = sab.State(3, 1)
+    H.seed_gpu_state(st, 1, 4096, [250, 0, 17], seed, [gdict])
+    snap = st.blob.clone()
+    runs = []
+    for rep in range(2):
+        st.blob.copy_(snap)
+        outs = []
+        for step in range(8):
+            x = wl.make_x(seed, 0, step, range(3), device="cuda")
+            outs.append(sab.swa_rma_decode(st, gw, 0, [0, 1, 2], x))
+            sab.advance(st, [0, 1, 2])
+        runs.append((torch.stack(outs), st.blob.clone()))
+    assert torch.equal(runs[0][0], runs[1][0])
+    assert torch.equal(runs[0][1], runs[1][1])
+
+
+def test_out_of_range_sequence_is_recorded_not_faulted(sab):
+    gw, gdict = H.gpu_weights(5, 0)
+    st = sab.State(2, 1)
+    H.seed_gpu_state(st, 1, 4096, [3, 4], 5, [gdict])
+    x = wl.make_x(5, 0, 0, range(2), device="cuda")
+    sab.swa_rma_decode(st, gw, 0, torch.tensor([0, 7], dtype=torch.int32, device="cuda"), x)
+    torch.cuda.synchronize()
+    assert sab.last_device_error(st) == -1
+    # a block that is already full cannot take the token's record
+    st.meta[1, 1] = 256
+    sab.swa_rma_decode(st, gw, 0, [0, 1], x)
+    assert sab.last_device_error(st) == -2

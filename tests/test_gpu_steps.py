@@ -1,0 +1,230 @@
+"""GPU parity of the individual steps (a2, a3, a4, a5, a7) against the oracle.
+
+All calls go through the C ABI (libedgerock.so via ctypes).  Bars:
+  - integer / byte work (append, commit indices, moved rows): bit-exact;
+  - FP32 scores: |Δs| <= 1e-4·(|s| + Σ_j |W2_gj|·|h_j|);
+  - normed/rotated BF16 rows: at most one BF16 ulp, ≥ 99% identical;
+  - attention branch outputs: the stated |Δ| <= 1e-2 + 1e-2·|oracle|, plus a
+    tighter |Δ| <= 2e-5 + 1e-4·|oracle| derived from FP32 accumulation, which
+    a single dropped or duplicated row (weight ≈ 1/2000) would break.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads as wl
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sab():
+    from sliding_window_anchor_b200 import build
+    build.build()
+    import sliding_window_anchor_b200 as m
+    return m
+
+
+# ----------------------------------------------------------------- a2
+
+def test_norm_rope_matches_oracle(sab):
+    n = 4096
+    x = synth.normal((n, 256), 3, synth.MISC, torch.bfloat16)
+    g = synth.normal((256,), 3, synth.MISC + 1, torch.bfloat16, scale=0.1, offset=1.0)
+    pos = torch.empty(n, dtype=torch.int32)
+    synth.fill_uniform_(pos, 3, synth.MISC + 2, 262144)
+    pos[:8] = torch.tensor([0, 1, 2, 1023, 4095, 131071, 262142, 262143], dtype=torch.int32)
+    ref = oracle.norm_rope(x, g, pos)
+    got = sab.qk_norm_rope(x.cuda(), g.cuda(), pos.cuda()).cpu()
+    ulp = 2.0 ** (torch.floor(torch.log2(ref.double().abs().clamp_min(1e-30))) - 7)
+    diff = (got.double() - ref.double()).abs()
+    assert bool((diff <= ulp + 1e-30).all()), float((diff / ulp).max())
+    assert (got == ref).double().mean() > 0.99
+    # in place
+    xc = x.cuda()
+    sab.qk_norm_rope(xc, g.cuda(), pos.cuda(), out=xc)
+    assert torch.equal(xc.cpu(), got)
+
+
+# ----------------------------------------------------------------- a3
+
+@pytest.mark.parametrize("n", [0, 1, 7, 64, 515])
+def test_score_matches_oracle(sab, n):
+    seed = 100 + n
+    w = wl.make_weights(seed, 0)
+    x = synth.normal((max(n, 1), 2560), seed, synth.MISC, torch.bfloat16)[:n]
+    gw, _ = H.gpu_weights(seed, 0)
+    got = sab.rma_score(gw, x.cuda()).cpu()
+    if n == 0:
+        assert got.shape == (0, 4)
+        return
+    ref = oracle.score(w["w1"], w["w2"], x)
+    h = torch.nn.functional.silu(x.double() @ w["w1"].double().T).abs()
+    cond = ref.double().abs() + h @ w["w2"].double().abs().T
+    assert bool(((got.double() - ref.double()).abs() <= 1e-4 * cond).all())
+
+
+# ----------------------------------------------------------------- a4
+
+def test_append_bit_exact(sab):
+    S, L = 5, 2
+    st = sab.State(S, L)
+    ost = oracle.OracleState(S, L)
+    ost.meta[:, 1] = torch.tensor([0, 3, 255, 17, 100], dtype=torch.int32)
+    st.meta.copy_(ost.meta)
+    seqs = [4, 0, 2]
+    k = synth.normal((3, 4, 256), 9, synth.MISC, torch.bfloat16)
+    v = synth.normal((3, 4, 256), 9, synth.MISC + 1, torch.bfloat16)
+    s = synth.normal((3, 4), 9, synth.MISC + 2)
+    pos = torch.tensor([77, 5, 9999], dtype=torch.int32)
+    ost.append_pending(1, seqs, k, v, s, pos)
+    sab.rma_append_pending(st, 1, seqs, k.cuda(), v.cuda(), s.cuda(), pos.cuda())
+    for n in ("pend_k", "pend_v", "pend_score", "pend_pos", "meta"):
+        assert torch.equal(getattr(st, n).cpu(), getattr(ost, n)), n
+    assert sab.last_device_error(st) == 0
+    # a full block is refused on the device: recorded, nothing written
+    before = st.pend_k.clone()
+    st.meta[1, 1] = 256
+    sab.rma_append_pending(st, 0, [1], k[:1].cuda(), v[:1].cuda(), s[:1].cuda(), pos[:1].cuda())
+    assert sab.last_device_error(st) == -2
+    assert torch.equal(st.pend_k, before)
+    # an out-of-range sequence id is recorded too
+    sab.rma_append_pending(st, 0, [9], k[:1].cuda(), v[:1].cuda(), s[:1].cuda(), pos[:1].cuda())
+    assert sab.last_device_error(st) == -1
+    assert sab.last_device_error(st) == 0
+
+
+# ----------------------------------------------------------------- a7
+
+def _commit_state(seed, c, p, S=1, tweak=None):
+    ost = oracle.OracleState(S, 1)
+    gen = np.random.default_rng(seed)
+    for sq in range(S):
+        for g in range(4):
+            ost.bank_score[sq, 0, g] = torch.from_numpy(gen.standard_normal(1024).astype(np.float32))
+            ost.pend_score[sq, 0, g] = torch.from_numpy(gen.standard_normal(256).astype(np.float32))
+            ost.bank_pos[sq, 0, g] = torch.from_numpy(gen.permutation(30000)[:1024].astype(np.int32))
+            ost.pend_pos[sq, 0, g] = torch.arange(40000, 40256, dtype=torch.int32)
+    for n, st_ in (("bank_k", 1), ("bank_v", 2), ("pend_k", 3), ("pend_v", 4)):
+        synth.fill_normal_(getattr(ost, n), seed, st_)
+    if tweak:
+        tweak(ost)
+    ost.meta[:] = torch.tensor([40256, p, c, 0], dtype=torch.int32)
+    return ost
+
+
+def _tweak_ties(ost):
+    bs, ps = ost.bank_score[0, 0], ost.pend_score[0, 0]
+    bs[0, :] = torch.from_numpy(np.linspace(5, 1, 1024).astype(np.float32))
+    ps[0, :] = bs[0, 700]
+    bs[1, 5] = -0.0
+    ps[1, 9] = 0.0
+    bs[1, 6] = float("nan")
+    ps[1, 10] = float("-inf")
+    ps[1, 11] = float("inf")
+    bs[2, :] = -1.0
+    ps[2, :] = -1.0
+    for g in range(4):
+        ost.pend_pos[0, 0, g, 3] = 123
+        ps[g, 3] = 100.0
+
+
+@pytest.mark.parametrize("c,p,tweak", [(1024, 256, None), (1024, 256, _tweak_ties),
+                                       (700, 256, None), (0, 256, None), (1024, 37, None),
+                                       (1000, 100, None), (1024, 0, None)])
+def test_commit_bit_exact(sab, c, p, tweak):
+    ost = _commit_state(50 + c + p, c, p, tweak=tweak)
+    st = sab.State(1, 1)
+    H.upload_state(st, ost)
+    ref_kept = ost.commit(-1, 0, want_kept=True)
+    kept = sab.rma_commit(st, -1, [0], want_kept=True).cpu()
+    assert torch.equal(kept[0], ref_kept)
+    for n in oracle.OracleState.ARRAYS:
+        assert torch.equal(getattr(st, n).cpu(), getattr(ost, n)), n
+    assert sab.last_device_error(st) == 0
+
+
+def test_commit_single_layer_leaves_metadata(sab):
+    ost = oracle.OracleState(2, 3)
+    for n, sid in (("bank_score", 1), ("pend_score", 2)):
+        synth.fill_normal_(getattr(ost, n), 8, sid)
+    for sq in range(2):
+        for l in range(3):
+            for g in range(4):
+                ost.bank_pos[sq, l, g] = torch.arange(1024, dtype=torch.int32) * 3
+                ost.pend_pos[sq, l, g] = torch.arange(5000, 5256, dtype=torch.int32)
+    for n, sid in (("bank_k", 3), ("bank_v", 4), ("pend_k", 5), ("pend_v", 6)):
+        synth.fill_normal_(getattr(ost, n), 8, sid)
+    ost.meta[:] = torch.tensor([5256, 256, 1024, 0], dtype=torch.int32)
+    st = sab.State(2, 3)
+    H.upload_state(st, ost)
+    ost.commit(1, 1)
+    sab.rma_commit(st, 1, [1])
+    for n in oracle.OracleState.ARRAYS:
+        assert torch.equal(getattr(st, n).cpu(), getattr(ost, n)), n
+
+
+# ----------------------------------------------------------------- a5
+
+def _attend_case(sab, B, t0s, fills, n_layers=1, layer=0, seed=70):
+    """Oracle runs one decode step per sequence; the device reads the same
+    post-append state with the same q and must reproduce both branches."""
+    ow, w = H.oracle_weights(seed, layer)
+    ost = oracle.OracleState(B, n_layers)
+    wd = [wl.make_weights(seed, l) for l in range(n_layers)]
+    for b in range(B):
+        if t0s[b] >= 1024:
+            one = oracle.OracleState(1, n_layers)
+            H.seed_oracle_state(one, [b], n_layers, t0s[b], [fills[b]], seed, wd)
+            for n in oracle.OracleState.ARRAYS:
+                getattr(ost, n)[b].copy_(getattr(one, n)[0])
+        else:  # early stream: build it token by token
+            for i in range(t0s[b]):
+                ost.decode_layer(ow, layer, b, synth.normal((2560,), seed, synth.MISC + i,
+                                                           torch.bfloat16))
+                ost.advance(b)
+    refs, qs = [], []
+    before = ost.clone()
+    for b in range(B):
+        x = synth.normal((2560,), seed + 1, synth.MISC + b, torch.bfloat16)
+        t = int(ost.meta[b, 0])
+        _, o_swa, o_rma = ost.decode_layer(ow, layer, b, x, want_branches=True)
+        proj = oracle.linear_bf16(w["w_qkv"], x)
+        q_swa = oracle.norm_rope(proj[:4096].view(16, 256), w["q_norm_swa"], t)
+        q_rma = oracle.norm_rope(proj[6144:10240].view(16, 256), w["q_norm_rma"], t)
+        refs.append((o_swa, o_rma))
+        qs.append((q_swa, q_rma))
+    # the device sees the state after the window write and pending append, before a commit
+    st = sab.State(B, n_layers)
+    H.upload_state(st, ost)
+    st.meta.copy_(before.meta)
+    for b in range(B):
+        p = int(before.meta[b, 1])
+        assert p + 1 < 256
+    q_swa = torch.stack([q[0] for q in qs]).cuda()
+    q_rma = torch.stack([q[1] for q in qs]).cuda()
+    o_swa, o_rma = sab.swa_rma_attend(st, layer, list(range(B)), q_swa, q_rma)
+    assert sab.last_device_error(st) == 0
+    for b in range(B):
+        for got, ref in ((o_swa[b], refs[b][0]), (o_rma[b], refs[b][1])):
+            assert H.tol_ok(got, ref, 1e-2, 1e-2)
+            assert H.tol_ok(got, ref, 2e-5, 1e-4), H.max_err(got, ref)
+
+
+def test_attend_full_state_single_query(sab):
+    # B=1 uses 16 splits per branch; fill 200 gives a ragged pending tail
+    _attend_case(sab, 1, [4096], [200])
+
+
+def test_attend_mixed_batch(sab):
+    # steady state with empty / ragged pending blocks, plus early-stream sequences
+    # (window not yet full, bank empty or partly filled by a first commit)
+    _attend_case(sab, 4, [4096, 4096, 3, 300], [0, 254, 0, 0])
+
+
+def test_attend_many_queries_one_split(sab):
+    B = 40  # 320 items: one split per branch
+    _attend_case(sab, B, [4096] * B, [(37 * b) % 250 for b in range(B)])
