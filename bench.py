@@ -168,10 +168,12 @@ def run_ours(args, rank, world, local_rank):
     clocks.start()
     n0 = sab.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
     e0.record(stream)
     for s in range(args.warmup, total):
         step(s)
     e1.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
     launches = sab.launch_count() - n0

@@ -118,7 +118,7 @@ typedef struct er_layer_weights {
 
 /* ---------------------------------------------------------------- state */
 
-/* Bytes er_state_carve needs for s_max sequences of n_layers (1..8) layers:
+/* Bytes er_state_carve needs for s_max (1..4096) sequences of n_layers (1..8) layers:
  * 72 MiB of K/V per sequence at 8 layers [F-mem], plus scores, positions,
  * metadata and alignment.  Returns 0 on bad arguments.  Host-only. */
 size_t er_state_bytes(int32_t s_max, int32_t n_layers);
@@ -153,10 +153,13 @@ int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, const er_bf16*
                     const int32_t* pos, er_stream_t stream);
 
 /* a3 — retention scores [F-arch], [N-rma]: s = W2 · SiLU(W1 · x), FP32
- * products and sums.  x: BF16 [n][2560]; s: FP32 [n][4] (one per KV group).
- * n may be 0. */
-int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s,
-                 er_stream_t stream);
+ * products and sums (split over K, summed in a fixed order: deterministic).
+ * x: BF16 [n][2560]; s: FP32 [n][4] (one per KV group); n may be 0.
+ * ws: scratch of er_score_workspace_bytes(n) bytes (the K-split partial sums;
+ * contents on return are unspecified). */
+size_t er_score_workspace_bytes(int32_t n);
+int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
+                 size_t ws_bytes, er_stream_t stream);
 
 /* a4 — appends one candidate record per KV group for each listed sequence at
  * its pend_count slot of `layer` [N-rma]: k, v BF16 [n][4][256] (k already

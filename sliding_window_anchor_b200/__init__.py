@@ -25,7 +25,7 @@ __all__ = ["State", "LayerWeights", "qk_norm_rope", "rma_score", "rma_append_pen
            "rma_commit", "swa_rma_attend", "swa_rma_decode", "swa_rma_prefill_chunk",
            "advance", "state_init", "last_device_error", "launch_count", "profile_enable",
            "profile_read", "decode_workspace_bytes", "prefill_workspace_bytes",
-           "attend_workspace_bytes", "ERError"]
+           "attend_workspace_bytes", "score_workspace_bytes", "ERError"]
 
 
 class State:
@@ -135,11 +135,17 @@ def qk_norm_rope(x: torch.Tensor, gain: torch.Tensor, pos: torch.Tensor, out=Non
     return out
 
 
-def rma_score(w: LayerWeights, x: torch.Tensor, stream=None):
+def score_workspace_bytes(n: int) -> int:
+    return int(lib().er_score_workspace_bytes(n))
+
+
+def rma_score(w: LayerWeights, x: torch.Tensor, ws=None, stream=None):
     n = x.numel() // HIDDEN
     s = torch.empty(n, NG, dtype=torch.float32, device=x.device)
+    ws = _ws(score_workspace_bytes(n), x.device, ws)
     check("er_rma_score", lib().er_rma_score(w.ptr(), dev_ptr(x, torch.bfloat16, "x"), n,
-                                             dev_ptr(s), stream_handle(stream, x.device)))
+                                             dev_ptr(s), dev_ptr(ws), ws.numel(),
+                                             stream_handle(stream, x.device)))
     return s
 
 

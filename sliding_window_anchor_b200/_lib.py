@@ -52,8 +52,10 @@ EXPORTS = {
                                             ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
     "er_qk_norm_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "er_score_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "er_rma_score": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p, ctypes.c_int32,
-                                    ctypes.c_void_p, ctypes.c_void_p]),
+                                    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                    ctypes.c_void_p]),
     "er_rma_append_pending": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_int32,
                                              ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,

@@ -11,21 +11,35 @@
 // the chunk's own rows in prefill, bank, pending); they stream through shared
 // memory in 64-row tiles.
 //
-// Persistent kernel, one 288-thread CTA per SM:
-//   warp 8 (producer): lane 0 walks the CTA's items and issues one bulk copy
-//     (cp.async.bulk, the TMA engine, no tensor map, no multicast) for the K
-//     rows and one for the V rows of each tile into a 3-stage ring, with
-//     completion counted as transaction bytes on the stage's mbarrier;
-//   warps 0..7 (consumers): each takes 8 rows of every tile.  K·q for the
-//     group's 4 heads uses packed FP32 FMA (FFMA2) with the logits reduced by
-//     a 5-step transpose butterfly in which lane L ends with (row L/4, head
-//     L%4); lane-dependent XOR indexing of rows and heads removes every select
-//     from the butterfly.  Online softmax in base 2 (q pre-scaled by
-//     log2(e)/16), P·V again with FFMA2.  At the item's last tile the 8 warps
-//     merge through shared memory and write one partial (m, l, o).
-// A second kernel merges the splits of both branches: o = o_swa + o_rma.
+// Persistent kernel, one 160-thread CTA per SM:
+//   warp 4 (producer): lane 0 walks the CTA's items; for each tile it arms the
+//     stage's mbarrier with the transaction bytes and issues TMA tensor copies
+//     (cp.async.bulk.tensor.2d, no multicast) of four 64x64 boxes of K rows and
+//     four of V rows, 128-byte swizzled, plus the item's 4 query heads (one
+//     plain bulk copy) with its first tile; 3-stage ring.
+//   warps 0..3 (consumers): each takes 16 rows (keys) of every tile.  The
+//     group's 4 heads share every K and V row, so the two contractions are
+//     small dense matrix products and run on the tensor cores with
+//     mma.m16n8k16 (BF16 in, FP32 accumulate), fragments read by ldmatrix from
+//     the swizzled tiles without bank conflicts:
+//       Sᵀ[16 keys x 8] = K[16 x 256] · Qᵀ  (heads 4..7 are zero padding)
+//       Oᵀ[256 x 8]    += Vᵀ[256 x 16 keys] · Pᵀ[16 keys x 8]
+//     P = exp2(S·log2e/16 - m) is split into a BF16 high part and a BF16
+//     remainder, and both are multiplied (two MMAs), so P·V keeps ~16
+//     significant bits instead of BF16's 8.  Online softmax in base 2 with the
+//     rescale skipped while the running maximum holds.  At the item's last
+//     tile the 4 warps merge through shared memory (their own rows of the
+//     tile's K boxes) and write either the final output or one partial
+//     (m, l, o) per split.
+// Measured on B200 before this design: the same pipeline with CUDA-core FMAs
+// reached 80% of the measured copy bandwidth, and 105% with the math removed,
+// so the math, not the data path, was the limit.
+// A second kernel merges the splits of both branches when there are several.
 // Every wait is bounded (≈2 s) and records ER_ETIMEOUT instead of hanging.
+#include <cudaTypedefs.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "params.cuh"
@@ -37,10 +51,12 @@ void profile_end(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t> ev);
 
 namespace {
 
-constexpr int TR = 64;        // rows per tile
-constexpr int NCW = 8;        // consumer warps (8 rows each)
+constexpr int TR = 64;                  // rows per tile
+constexpr int NCW = 4;                  // consumer warps, 16 rows each
 constexpr int STAGES = 3;
 constexpr int NTHREADS = (NCW + 1) * 32;
+constexpr int BOX = 64 * 128;           // one 64-row x 64-dim box (8 KB, 128 B per row)
+constexpr int TILE_BYTES = 4 * BOX;     // a 64-row K (or V) tile: four boxes
 constexpr float kLog2eOver16 = 1.4426950408889634f / 16.0f;
 constexpr int F_FIRST = 1, F_LAST = 2;
 
@@ -49,12 +65,12 @@ struct TileDesc {
   int flags;
 };
 
-struct __align__(128) AttnSmem {
-  uint16_t k[STAGES][TR * D];
-  uint16_t v[STAGES][TR * D];
-  float merge_acc[NCW][HPG][D];
+struct __align__(1024) AttnSmem {
+  unsigned char k[STAGES][TILE_BYTES];  // the item's last K tile doubles as the merge area
+  unsigned char v[STAGES][TILE_BYTES];
+  uint16_t q[STAGES][HPG * D];         // the item's 4 query heads, sent with its first tile
+  uint16_t pt[NCW][2][8][16];          // Pᵀ staging per warp: [hi/lo][head][key]
   float merge_ml[NCW][HPG][2];
-  float2 pbuf[NCW][8][HPG];
   TileDesc desc[STAGES];
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
@@ -62,50 +78,48 @@ struct __align__(128) AttnSmem {
   volatile int abort_flag;
 };
 
-}  // namespace
+static_assert(sizeof(AttnSmem) + 1024 <= 232448,
+              "shared memory above the 227 KB per-block limit");
 
-
-namespace {
-
+// Rows [row, row + rows) of one of the tensor-mapped arrays.
 struct Range {
-  const uint16_t* k;
-  const uint16_t* v;
+  int map;
+  int row;
   int rows;
 };
 
-// Row ranges of one item; returns the number of ranges (0..3).
+// Row ranges of one item; returns the number of ranges (0..3), none empty.
 __device__ int item_ranges(const AttendParams& P, int qi, int g, int br, Range r[3]) {
   const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
   if (seq < 0 || seq >= P.s_max) return 0;
   const int32_t pos0 = P.meta[seq * 4 + 0];
   const int pend = P.meta[seq * 4 + 1];
   const int bank = min(max(P.meta[seq * 4 + 2], 0), BANK);
-  const size_t gi = grp(seq, P.layer, g, P.L);
+  const int gi = (int)grp(seq, P.layer, g, P.L);
   int n = 0;
   if (br == 0) {
-    const uint16_t* wk = P.win_k + gi * WIN * D;
-    const uint16_t* wv = P.win_v + gi * WIN * D;
+    const int w0 = gi * WIN;  // first ring row of this (sequence, layer, group)
     if (!P.prefill) {
       // window positions [t-1023, t], t = pos0, all already in the ring
       const int nwin = min(pos0 + 1, WIN);
-      r[n++] = Range{wk, wv, nwin};
+      if (nwin > 0) r[n++] = Range{TM_WIN, w0, nwin};
     } else {
       const int t = pos0 + qi;
+      if (t < 0) return 0;
       const int lo = max(0, t - (WIN - 1));
       const int count = pos0 - lo;  // old ring positions lo..pos0-1
       if (count > 0) {
         const int s0 = lo % WIN;
         const int n1 = min(count, WIN - s0);
-        r[n++] = Range{wk + (size_t)s0 * D, wv + (size_t)s0 * D, n1};
-        if (count > n1) r[n++] = Range{wk, wv, count - n1};
+        r[n++] = Range{TM_WIN, w0 + s0, n1};
+        if (count > n1) r[n++] = Range{TM_WIN, w0, count - n1};
       }
-      r[n++] = Range{P.chunk_k + (size_t)g * P.nq * D, P.chunk_v + (size_t)g * P.nq * D, qi + 1};
+      r[n++] = Range{TM_CHUNK, g * P.nq, qi + 1};
     }
   } else {
-    if (bank > 0)
-      r[n++] = Range{P.bank_k + gi * BANK * D, P.bank_v + gi * BANK * D, bank};
+    if (bank > 0) r[n++] = Range{TM_BANK, gi * BANK, bank};
     const int np = min(pend + (P.prefill ? qi : 0) + 1, PEND);
-    if (np > 0) r[n++] = Range{P.pend_k + gi * PEND * D, P.pend_v + gi * PEND * D, np};
+    if (np > 0) r[n++] = Range{TM_PEND, gi * PEND, np};
   }
   return n;
 }
@@ -120,9 +134,117 @@ __device__ __forceinline__ void item_coords(const AttendParams& P, int item, int
   *qi = rest >> 2;
 }
 
-__global__ void __launch_bounds__(NTHREADS, 1) k_attend(AttendParams P) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  AttnSmem& S = *reinterpret_cast<AttnSmem*>(smem_raw);
+struct Tile {
+  int map, row;
+  int rows, flags, qi, g, br;
+};
+
+// The CTA's tile sequence: items item_begin..item_end-1, each the tiles of its
+// split (or one empty tile when the split has no rows).
+struct TileIter {
+  const AttendParams* P;
+  int item, item_end;
+  Range r[3];
+  int nr, ri, tile_in_range, e, emit, qi, g, br;
+  bool has_rows;
+
+  __device__ void init(const AttendParams* p, int begin, int end) {
+    P = p;
+    item = begin;
+    item_end = end;
+    start_item();
+  }
+  __device__ void start_item() {
+    if (item >= item_end) return;
+    int split;
+    item_coords(*P, item, &qi, &g, &br, &split);
+    nr = item_ranges(*P, qi, g, br, r);
+    int nt = 0;
+    for (int i = 0; i < nr; ++i) nt += (r[i].rows + TR - 1) / TR;
+    const int t0 = (int)((long)split * nt / P->splits);
+    const int t1 = (int)((long)(split + 1) * nt / P->splits);
+    ri = 0;
+    int tix = 0;
+    while (ri < nr && tix + (r[ri].rows + TR - 1) / TR <= t0) {
+      tix += (r[ri].rows + TR - 1) / TR;
+      ++ri;
+    }
+    tile_in_range = t0 - tix;
+    has_rows = t1 > t0;
+    emit = has_rows ? t1 - t0 : 1;
+    e = 0;
+  }
+  __device__ bool next(Tile* t) {
+    if (item >= item_end) return false;
+    t->qi = qi;
+    t->g = g;
+    t->br = br;
+    t->rows = 0;
+    t->map = 0;
+    t->row = 0;
+    if (has_rows) {
+      const int off = tile_in_range * TR;
+      t->rows = min(TR, r[ri].rows - off);
+      t->map = r[ri].map;
+      t->row = r[ri].row + off;
+      if (++tile_in_range * TR >= r[ri].rows) {
+        ++ri;
+        tile_in_range = 0;
+      }
+    }
+    t->flags = (e == 0 ? F_FIRST : 0) | (e == emit - 1 ? F_LAST : 0);
+    if (++e == emit) {
+      ++item;
+      start_item();
+    }
+    return true;
+  }
+};
+
+// ------------------------------------------------------- tensor-core helpers
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t r[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t r[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// D = A·B + D, m16n8k16, BF16 operands, FP32 accumulators.
+__device__ __forceinline__ void mma_bf16(float d[4], const uint32_t a[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// One 64x64 box of a 2-D tensor map into shared memory (x: dims, y: rows).
+// x is a multiple of 64 elements (128 B), as TMA requires.
+__device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x, int y,
+                                        uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ AttendParams P) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // the swizzled boxes need 1024-byte aligned destinations
+  AttnSmem& S = *reinterpret_cast<AttnSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = P.nq * NG * 2 * P.splits;
 
@@ -137,99 +259,89 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(AttendParams P) {
   }
   __syncthreads();
 
+  // contiguous, even-length item ranges per CTA: a (query, group)'s two branch
+  // items are read back to back by the same CTA
+  int per = (n_items + gridDim.x - 1) / gridDim.x;
+  per += per & 1;
+  const int item_begin = min(n_items, (int)blockIdx.x * per);
+  const int item_end = min(n_items, item_begin + per);
+
   if (warp == NCW) {
     // ------------------------------------------------------------ producer
-    if (lane != 0) return;
+    TileIter ld;
+    ld.init(&P, item_begin, item_end);
+    Tile t;
     uint32_t tc = 0;
-    for (int item = blockIdx.x; item < n_items && !S.abort_flag; item += gridDim.x) {
-      int qi, g, br, split;
-      item_coords(P, item, &qi, &g, &br, &split);
-      Range r[3];
-      const int nr = item_ranges(P, qi, g, br, r);
-      int nt = 0;
-      for (int i = 0; i < nr; ++i) nt += (r[i].rows + TR - 1) / TR;
-      const int t0 = (int)((long)split * nt / P.splits);
-      const int t1 = (int)((long)(split + 1) * nt / P.splits);
-      int ri = 0, tile_in_range = 0, tix = 0;
-      // advance to tile t0
-      while (ri < nr && tix + (r[ri].rows + TR - 1) / TR <= t0) {
-        tix += (r[ri].rows + TR - 1) / TR;
-        ++ri;
-      }
-      tile_in_range = t0 - tix;
-      const int emit = (t1 > t0) ? (t1 - t0) : 1;  // an empty item still sends one tile
-      for (int e = 0; e < emit; ++e) {
-        const int stage = tc % STAGES;
-        const uint32_t phase = (tc / STAGES) & 1;
-        if (!mbar_wait(&S.empty[stage], phase ^ 1, P.err)) {
-          S.abort_flag = 1;
-          break;
-        }
-        int rows = 0;
-        const uint16_t *ks = nullptr, *vs = nullptr;
-        if (t1 > t0) {
-          const int off = tile_in_range * TR;
-          rows = min(TR, r[ri].rows - off);
-          ks = r[ri].k + (size_t)off * D;
-          vs = r[ri].v + (size_t)off * D;
-          if (++tile_in_range * TR >= r[ri].rows) {
-            ++ri;
-            tile_in_range = 0;
+    while (ld.next(&t)) {
+      const int stage = tc % STAGES;
+      const uint32_t phase = (tc / STAGES) & 1;
+      if (lane == 0 && !mbar_wait(&S.empty[stage], phase ^ 1, P.err)) S.abort_flag = 1;
+      __syncwarp();
+      if (S.abort_flag) break;
+      if (lane == 0) {
+        const uint32_t qbytes = (t.flags & F_FIRST) ? HPG * ROW_BYTES : 0;
+        // whole boxes always land (rows past the range are masked by the consumers,
+        // rows past the array are zero-filled by TMA)
+        const uint32_t bytes = (t.rows > 0 ? 2u * TILE_BYTES : 0u) + qbytes;
+        S.desc[stage].rows = t.rows;
+        S.desc[stage].flags = t.flags;
+        if (bytes) mbar_arrive_expect_tx(&S.full[stage], bytes);
+        else mbar_arrive(&S.full[stage]);
+        if (qbytes)
+          bulk_g2s(S.q[stage], (t.br ? P.q_rma : P.q_swa) + ((size_t)t.qi * NH + t.g * HPG) * D,
+                   qbytes, &S.full[stage]);
+        if (t.rows > 0) {
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            tma_box(S.k[stage] + b * BOX, &P.tmap_k[t.map], 64 * b, t.row, &S.full[stage]);
+            tma_box(S.v[stage] + b * BOX, &P.tmap_v[t.map], 64 * b, t.row, &S.full[stage]);
           }
         }
-        S.desc[stage].rows = rows;
-        S.desc[stage].flags = (e == 0 ? F_FIRST : 0) | (e == emit - 1 ? F_LAST : 0);
-        if (rows > 0) {
-          const uint32_t bytes = (uint32_t)rows * ROW_BYTES;
-          mbar_arrive_expect_tx(&S.full[stage], 2 * bytes);
-          bulk_g2s(S.k[stage], ks, bytes, &S.full[stage]);
-          bulk_g2s(S.v[stage], vs, bytes, &S.full[stage]);
-        } else {
-          mbar_arrive(&S.full[stage]);
-        }
-        ++tc;
       }
+      ++tc;
     }
     // drain: the last tile of each stage must have landed before exit
-    for (uint32_t i = (tc > STAGES ? tc - STAGES : 0); i < tc; ++i)
-      mbar_wait(&S.full[i % STAGES], (i / STAGES) & 1, P.err);
+    if (lane == 0)
+      for (uint32_t i = (tc > STAGES ? tc - STAGES : 0); i < tc; ++i)
+        mbar_wait(&S.full[i % STAGES], (i / STAGES) & 1, P.err);
     return;
   }
 
   // -------------------------------------------------------------- consumers
-  const int rx = (lane >> 2) & 7;  // row XOR of this lane
-  const int hx = lane & 3;         // head XOR of this lane
-  const int lr = lane >> 2;        // logit row held after the butterfly
+  const int gq = lane >> 2;   // fragment row group: keys gq, gq+8 / head gq (B operands)
+  const int cq = lane & 3;    // fragment column quad: heads 2cq, 2cq+1 / keys 2cq.. (B)
+  const bool real_heads = cq < 2;   // lanes holding heads 0..3 of the C fragments
+  const int row0 = 16 * warp;       // this warp's 16 rows of a tile
+  // ldmatrix rows of this lane: QK reads keys row0 + (lane&7) + 8*((lane>>3)&1) at dim
+  // chunk 2kk + (lane>>4); PV reads keys row0 + (lane&7) + 8*(lane>>4) at dim chunk
+  // 2mt + ((lane>>3)&1).  In a 128B-swizzled box, 16-byte chunk c of row r sits at
+  // chunk position c ^ (r & 7), and r & 7 == lane & 7 here.
+  const int sw = lane & 7;
+  const uint32_t row_qk = (uint32_t)(row0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * 128u;
+  const int chunk_qk = lane >> 4;
+  const uint32_t row_pv = (uint32_t)(row0 + (lane & 7) + 8 * (lane >> 4)) * 128u;
+  const int chunk_pv = (lane >> 3) & 1;
+
   uint32_t tc = 0;
   uint32_t mphase = 0;
   bool aborted = false;
+  float keep[8];  // normalized SWA output of the pair's first item (direct mode)
+#pragma unroll
+  for (int i = 0; i < 8; ++i) keep[i] = 0.f;
 
-  for (int item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (int item = item_begin; item < item_end; ++item) {
     int qi, g, br, split;
     item_coords(P, item, &qi, &g, &br, &split);
-    // q for the group's 4 heads: dims 8*lane..8*lane+7, heads XOR-permuted, duplicated pairs
-    float2 qd[HPG][8];
-    {
-      const uint16_t* qb = (br ? P.q_rma : P.q_swa) + ((size_t)qi * NH + g * HPG) * D + lane * 8;
+    uint32_t qb[16][2];  // Qᵀ B fragments for the 16 k-steps (heads >= 4 are zero)
+    float o[16][4];      // Oᵀ accumulators: dims 16mt + gq (+8) x heads 2cq (+1)
 #pragma unroll
-      for (int h = 0; h < HPG; ++h) {
-        const uint4 w = *reinterpret_cast<const uint4*>(qb + (size_t)(h ^ hx) * D);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (int mt = 0; mt < 16; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = bf_lo(ws[e]) * kLog2eOver16, b = bf_hi(ws[e]) * kLog2eOver16;
-          qd[h][2 * e] = make_float2(a, a);
-          qd[h][2 * e + 1] = make_float2(b, b);
-        }
-      }
-    }
-    float m_run = -INFINITY, l_run = 0.f;
-    float2 accv[HPG][4];
-#pragma unroll
-    for (int h = 0; h < HPG; ++h)
-#pragma unroll
-      for (int wd = 0; wd < 4; ++wd) accv[h][wd] = make_float2(0.f, 0.f);
+      for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};  // heads 2cq, 2cq+1
+    float l_run[2] = {0.f, 0.f};              // this lane's partial sums
 
+    int last_stage = 0;
     while (true) {
       const int stage = tc % STAGES;
       const uint32_t phase = (tc / STAGES) & 1;
@@ -238,150 +350,202 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(AttendParams P) {
         S.abort_flag = 1;
       }
       const TileDesc d = S.desc[stage];
-      const int nrows = aborted ? 0 : min(8, d.rows - 8 * warp);
+      const int nrows = aborted ? 0 : min(16, d.rows - row0);
+      if (d.flags & F_FIRST) {
+        const uint16_t* q = S.q[stage];
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          qb[kk][0] = gq < HPG ? *reinterpret_cast<const uint32_t*>(q + gq * D + 16 * kk + 2 * cq)
+                               : 0u;
+          qb[kk][1] = gq < HPG
+                          ? *reinterpret_cast<const uint32_t*>(q + gq * D + 16 * kk + 8 + 2 * cq)
+                          : 0u;
+        }
+      }
       if (nrows > 0) {
-        // ---- K phase: logits of 8 rows x 4 heads
-        const char* kt = reinterpret_cast<const char*>(S.k[stage]) + (8 * warp) * ROW_BYTES +
-                         lane * 16;
-        float2 acc[4][HPG];
+        const uint32_t kbase = smem_u32(S.k[stage]);
+        const uint32_t vbase = smem_u32(S.v[stage]);
+        if (nrows < 16) {
+          // rows past the tile's end hold stale bytes: zero this warp's V rows there so
+          // that p = 0 times them stays 0 in the tensor-core sum
+          for (int r = nrows; r < 16; ++r)  // a whole row: 4 boxes x 8 chunks = 32 lanes
+            *reinterpret_cast<uint4*>(S.v[stage] + (lane >> 3) * BOX + (row0 + r) * 128 +
+                                      (lane & 7) * 16) = make_uint4(0, 0, 0, 0);
+          __syncwarp();
+        }
+        // ---- Sᵀ = K · Qᵀ over 256 dims (two accumulators to halve the chain)
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int ip = 0; ip < 4; ++ip)
+        for (int kk = 0; kk < 16; kk += 2) {
+          uint32_t a[4], a2[4];
+          const int c0 = 2 * kk + chunk_qk, c1 = 2 * (kk + 1) + chunk_qk;  // 0..31
+          ldsm_x4(kbase + (c0 >> 3) * BOX + row_qk + (((c0 & 7) ^ sw) << 4), a);
+          ldsm_x4(kbase + (c1 >> 3) * BOX + row_qk + (((c1 & 7) ^ sw) << 4), a2);
+          mma_bf16(sa, a, qb[kk][0], qb[kk][1]);
+          mma_bf16(sb, a2, qb[kk + 1][0], qb[kk + 1][1]);
+        }
+        // s[i]: keys gq (i<2) / gq+8 (i>=2), heads 2cq + (i&1); base-2 logits
+        float s[4];
 #pragma unroll
-          for (int h = 0; h < HPG; ++h) acc[ip][h] = make_float2(0.f, 0.f);
+        for (int i = 0; i < 4; ++i) {
+          const int key = (i < 2) ? gq : gq + 8;
+          s[i] = (key < nrows) ? (sa[i] + sb[i]) * kLog2eOver16 : -INFINITY;
+        }
+        // ---- online softmax for this lane's two heads (8 lanes share each pair)
+        float alpha[2], pv[4];
 #pragma unroll
-        for (int ip = 0; ip < 4; ++ip) {
-          const uint4 ka = lds128(kt + ((2 * ip) ^ rx) * ROW_BYTES);
-          const uint4 kb = lds128(kt + ((2 * ip + 1) ^ rx) * ROW_BYTES);
-          const uint32_t wa[4] = {ka.x, ka.y, ka.z, ka.w};
-          const uint32_t wb[4] = {kb.x, kb.y, kb.z, kb.w};
+        for (int j = 0; j < 2; ++j) {
+          float mt = fmaxf(s[j], s[j + 2]);
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 4));
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
+          mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+          const float m_new = fmaxf(m_run[j], mt);
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          alpha[j] = exp2f(m_run[j] - m_use);
+          pv[j] = exp2f(s[j] - m_use);
+          pv[j + 2] = exp2f(s[j + 2] - m_use);
+          l_run[j] = l_run[j] * alpha[j] + pv[j] + pv[j + 2];
+          m_run[j] = m_new;
+        }
+        if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-          for (int wd = 0; wd < 4; ++wd) {
-            const float2 lo = make_float2(bf_lo(wa[wd]), bf_lo(wb[wd]));
-            const float2 hi = make_float2(bf_hi(wa[wd]), bf_hi(wb[wd]));
-#pragma unroll
-            for (int h = 0; h < HPG; ++h) {
-              acc[ip][h] = __ffma2_rn(qd[h][2 * wd], lo, acc[ip][h]);
-              acc[ip][h] = __ffma2_rn(qd[h][2 * wd + 1], hi, acc[ip][h]);
-            }
+          for (int mt = 0; mt < 16; ++mt) {
+            o[mt][0] *= alpha[0];
+            o[mt][1] *= alpha[1];
+            o[mt][2] *= alpha[0];
+            o[mt][3] *= alpha[1];
           }
         }
-        // transpose butterfly: lane L ends with (row L>>2, head L&3)
+        // ---- Pᵀ to shared memory as BF16 high part + BF16 remainder
+        if (real_heads) {
 #pragma unroll
-        for (int ip = 0; ip < 2; ++ip)
-#pragma unroll
-          for (int h = 0; h < HPG; ++h) {
-            acc[ip][h].x += __shfl_xor_sync(0xffffffffu, acc[ip + 2][h].x, 16);
-            acc[ip][h].y += __shfl_xor_sync(0xffffffffu, acc[ip + 2][h].y, 16);
-          }
-#pragma unroll
-        for (int h = 0; h < HPG; ++h) {
-          acc[0][h].x += __shfl_xor_sync(0xffffffffu, acc[1][h].x, 8);
-          acc[0][h].y += __shfl_xor_sync(0xffffffffu, acc[1][h].y, 8);
-        }
-        float rr[HPG];
-#pragma unroll
-        for (int h = 0; h < HPG; ++h)
-          rr[h] = acc[0][h].x + __shfl_xor_sync(0xffffffffu, acc[0][h].y, 4);
-        rr[0] += __shfl_xor_sync(0xffffffffu, rr[2], 2);
-        rr[1] += __shfl_xor_sync(0xffffffffu, rr[3], 2);
-        rr[0] += __shfl_xor_sync(0xffffffffu, rr[1], 1);
-
-        // ---- online softmax (base 2) for head hx
-        const float s = (lr < nrows) ? rr[0] : -INFINITY;
-        float mt = fmaxf(s, __shfl_xor_sync(0xffffffffu, s, 4));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 8));
-        mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
-        const float m_new = fmaxf(m_run, mt);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = exp2f(m_run - m_use);
-        const float pr = exp2f(s - m_use);
-        l_run = l_run * alpha + pr;
-        m_run = m_new;
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-#pragma unroll
-          for (int h = 0; h < HPG; ++h) {
-            const float ah = __shfl_sync(0xffffffffu, alpha, h);
-            const float2 a2 = make_float2(ah, ah);
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) accv[h][wd] = __fmul2_rn(accv[h][wd], a2);
+          for (int i = 0; i < 4; ++i) {
+            const int key = (i < 2) ? gq : gq + 8;
+            const int head = 2 * cq + (i & 1);
+            const __nv_bfloat16 hi = __float2bfloat16_rn(pv[i]);
+            const __nv_bfloat16 lo = __float2bfloat16_rn(pv[i] - __bfloat162float(hi));
+            S.pt[warp][0][head][key] = __bfloat16_as_ushort(hi);
+            S.pt[warp][1][head][key] = __bfloat16_as_ushort(lo);
           }
         }
-        S.pbuf[warp][lr][hx] = make_float2(pr, pr);
         __syncwarp();
-
-        // ---- V phase
-        const char* vt = reinterpret_cast<const char*>(S.v[stage]) + (8 * warp) * ROW_BYTES +
-                         lane * 16;
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          if (r < nrows) {
-            const uint4 vv = lds128(vt + r * ROW_BYTES);
-            const float4 pa = lds128f(&S.pbuf[warp][r][0]);
-            const float4 pb = lds128f(&S.pbuf[warp][r][2]);
-            const float2 p2[HPG] = {make_float2(pa.x, pa.y), make_float2(pa.z, pa.w),
-                                    make_float2(pb.x, pb.y), make_float2(pb.z, pb.w)};
-            const uint32_t ws[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-              const float2 val = make_float2(bf_lo(ws[wd]), bf_hi(ws[wd]));
-#pragma unroll
-              for (int h = 0; h < HPG; ++h) accv[h][wd] = __ffma2_rn(p2[h], val, accv[h][wd]);
-            }
-          }
+        uint32_t bh0 = 0, bh1 = 0, bl0 = 0, bl1 = 0;
+        if (gq < HPG) {
+          bh0 = *reinterpret_cast<const uint32_t*>(&S.pt[warp][0][gq][2 * cq]);
+          bh1 = *reinterpret_cast<const uint32_t*>(&S.pt[warp][0][gq][2 * cq + 8]);
+          bl0 = *reinterpret_cast<const uint32_t*>(&S.pt[warp][1][gq][2 * cq]);
+          bl1 = *reinterpret_cast<const uint32_t*>(&S.pt[warp][1][gq][2 * cq + 8]);
         }
+        // ---- Oᵀ += Vᵀ · Pᵀ, 16 dim tiles of 16
+#pragma unroll
+        for (int mt = 0; mt < 16; ++mt) {
+          uint32_t a[4];
+          const int c = 2 * mt + chunk_pv;  // 0..31
+          ldsm_x4_t(vbase + (c >> 3) * BOX + row_pv + (((c & 7) ^ sw) << 4), a);
+          mma_bf16(o[mt], a, bh0, bh1);
+          mma_bf16(o[mt], a, bl0, bl1);
+        }
+        __syncwarp();  // Pᵀ staging is rewritten by the next tile
+        if (nrows < 16) fence_proxy_async_smem();  // zeroed rows are refilled by TMA later
+      }
+      ++tc;
+      if (aborted || (d.flags & F_LAST)) {
+        last_stage = stage;  // released after the merge, which reuses its K buffer
+        break;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[stage]);
-      ++tc;
-      if (aborted || (d.flags & F_LAST)) break;
     }
 
-    // ---- merge the 8 warps' partials of this item
-    float lt = l_run;
-    lt += __shfl_xor_sync(0xffffffffu, lt, 4);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 8);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 16);
-    if (lane < HPG) {
-      S.merge_ml[warp][lane][0] = m_run;
-      S.merge_ml[warp][lane][1] = lt;
-    }
+    // ---- merge the 4 warps' partials of this item
+    // merge slot of (warp, head): 1 KB inside this warp's own rows of K box `head`
+    unsigned char* kl = S.k[last_stage];
+    auto slot = [&](int w, int h) { return reinterpret_cast<float*>(kl + h * BOX + w * 2048); };
+    float lt[2] = {l_run[0], l_run[1]};
 #pragma unroll
-    for (int h = 0; h < HPG; ++h) {
-      float4* dst = reinterpret_cast<float4*>(&S.merge_acc[warp][h][lane * 8]);
-      dst[0] = make_float4(accv[h][0].x, accv[h][0].y, accv[h][1].x, accv[h][1].y);
-      dst[1] = make_float4(accv[h][2].x, accv[h][2].y, accv[h][3].x, accv[h][3].y);
+    for (int j = 0; j < 2; ++j) {
+      lt[j] += __shfl_xor_sync(0xffffffffu, lt[j], 4);
+      lt[j] += __shfl_xor_sync(0xffffffffu, lt[j], 8);
+      lt[j] += __shfl_xor_sync(0xffffffffu, lt[j], 16);
+    }
+    if (lane < 2) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        S.merge_ml[warp][2 * lane + j][0] = m_run[j];
+        S.merge_ml[warp][2 * lane + j][1] = lt[j];
+      }
+    }
+    if (real_heads) {
+#pragma unroll
+      for (int mt = 0; mt < 16; ++mt) {
+        const int d0 = 16 * mt + gq;
+        slot(warp, 2 * cq)[d0] = o[mt][0];
+        slot(warp, 2 * cq + 1)[d0] = o[mt][1];
+        slot(warp, 2 * cq)[d0 + 8] = o[mt][2];
+        slot(warp, 2 * cq + 1)[d0 + 8] = o[mt][3];
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.merge_bar);
     if (!mbar_wait(&S.merge_bar, mphase, P.err)) aborted = true;
     mphase ^= 1;
     {
-      const int ct = warp * 32 + lane;
-      const int h = ct >> 6, d0 = (ct & 63) * 4;
+      const int ct = warp * 32 + lane;        // 128 threads: head ct/32, dims 8*(ct%32)..
+      const int h = ct >> 5, d0 = (ct & 31) * 8;
       float M = -INFINITY;
 #pragma unroll
       for (int w = 0; w < NCW; ++w) M = fmaxf(M, S.merge_ml[w][h][0]);
-      float Ls = 0.f;
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      float Ls = 0.f, acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
       if (M != -INFINITY) {
 #pragma unroll
         for (int w = 0; w < NCW; ++w) {
           const float f = exp2f(S.merge_ml[w][h][0] - M);
           Ls += S.merge_ml[w][h][1] * f;
-          const float4 a = *reinterpret_cast<const float4*>(&S.merge_acc[w][h][d0]);
-          o.x += a.x * f; o.y += a.y * f; o.z += a.z * f; o.w += a.w * f;
+          const float* sl = slot(w, h);
+          const float4 a = *reinterpret_cast<const float4*>(sl + d0);
+          const float4 b = *reinterpret_cast<const float4*>(sl + d0 + 4);
+          acc[0] += a.x * f; acc[1] += a.y * f; acc[2] += a.z * f; acc[3] += a.w * f;
+          acc[4] += b.x * f; acc[5] += b.y * f; acc[6] += b.z * f; acc[7] += b.w * f;
         }
       }
-      *reinterpret_cast<float4*>(P.part_o + ((size_t)item * HPG + h) * D + d0) = o;
-      if (d0 == 0) {
-        P.part_ml[((size_t)item * HPG + h) * 2 + 0] = M;
-        P.part_ml[((size_t)item * HPG + h) * 2 + 1] = Ls;
+      if (P.direct) {
+        const float rcp = Ls > 0.f ? 1.0f / Ls : 0.f;
+        const size_t oi = ((size_t)qi * NH + g * HPG + h) * D + d0;
+        if (P.o_sum == nullptr) {
+          float* dst = (br ? P.o_rma : P.o_swa) + oi;
+          *reinterpret_cast<float4*>(dst) =
+              make_float4(acc[0] * rcp, acc[1] * rcp, acc[2] * rcp, acc[3] * rcp);
+          *reinterpret_cast<float4*>(dst + 4) =
+              make_float4(acc[4] * rcp, acc[5] * rcp, acc[6] * rcp, acc[7] * rcp);
+        } else if (br == 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) keep[i] = acc[i] * rcp;
+        } else {
+          uint4 packed;
+          packed.x = pack_bf2(keep[0] + acc[0] * rcp, keep[1] + acc[1] * rcp);
+          packed.y = pack_bf2(keep[2] + acc[2] * rcp, keep[3] + acc[3] * rcp);
+          packed.z = pack_bf2(keep[4] + acc[4] * rcp, keep[5] + acc[5] * rcp);
+          packed.w = pack_bf2(keep[6] + acc[6] * rcp, keep[7] + acc[7] * rcp);
+          *reinterpret_cast<uint4*>(P.o_sum + oi) = packed;
+        }
+      } else {
+        float* dst = P.part_o + ((size_t)item * HPG + h) * D + d0;
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        if (d0 == 0) {
+          P.part_ml[((size_t)item * HPG + h) * 2 + 0] = M;
+          P.part_ml[((size_t)item * HPG + h) * 2 + 1] = Ls;
+        }
       }
     }
+    fence_proxy_async_smem();  // the merge wrote the K buffer that TMA refills next
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.merge_bar);
     if (!mbar_wait(&S.merge_bar, mphase, P.err)) aborted = true;
     mphase ^= 1;
+    if (lane == 0) mbar_arrive(&S.empty[last_stage]);
     if (aborted) break;
   }
 }
@@ -434,29 +598,80 @@ size_t attend_part_floats(int nq) {
 }
 size_t attend_ml_floats(int nq) { return (size_t)nq * NG * 2 * attend_splits(nq) * HPG * 2; }
 
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D map of `rows` contiguous 512-byte BF16 rows; 64x64 boxes, 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows) {
+  auto fn = encode_fn();
+  if (!fn || rows == 0 || ((uintptr_t)base & 15u)) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)ROW_BYTES};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+}  // namespace
+
 int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* o_sum,
                   cudaStream_t st) {
   if (P0.nq <= 0) return ER_OK;
   AttendParams P = P0;
   P.splits = attend_splits(P.nq);
+  const uint64_t groups = (uint64_t)P.s_max * P.L * NG;
+  bool ok = encode_rows(&P.tmap_k[TM_WIN], P.win_k, groups * WIN) &&
+            encode_rows(&P.tmap_v[TM_WIN], P.win_v, groups * WIN) &&
+            encode_rows(&P.tmap_k[TM_BANK], P.bank_k, groups * BANK) &&
+            encode_rows(&P.tmap_v[TM_BANK], P.bank_v, groups * BANK) &&
+            encode_rows(&P.tmap_k[TM_PEND], P.pend_k, groups * PEND) &&
+            encode_rows(&P.tmap_v[TM_PEND], P.pend_v, groups * PEND);
+  if (P.prefill) {
+    ok = ok && encode_rows(&P.tmap_k[TM_CHUNK], P.chunk_k, (uint64_t)NG * P.nq) &&
+         encode_rows(&P.tmap_v[TM_CHUNK], P.chunk_v, (uint64_t)NG * P.nq);
+  } else {
+    P.tmap_k[TM_CHUNK] = P.tmap_k[TM_WIN];
+    P.tmap_v[TM_CHUNK] = P.tmap_v[TM_WIN];
+  }
+  if (!ok) return ER_ECUDA;
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     if (cudaFuncSetAttribute(k_attend, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(AttnSmem)) != cudaSuccess)
+                             (int)sizeof(AttnSmem) + 1024) != cudaSuccess)
       return ER_ECUDA;
     attr_done[dev] = true;
   }
   const int n_items = P.nq * NG * 2 * P.splits;
   const int grid = min(n_items, num_sms());
+  P.direct = P.splits == 1 ? 1 : 0;
+  P.o_swa = o_swa;
+  P.o_rma = o_rma;
+  P.o_sum = o_sum;
   std::pair<cudaEvent_t, cudaEvent_t> ev;
   const bool timed = profile_begin(st, &ev);
-  k_attend<<<grid, NTHREADS, sizeof(AttnSmem), st>>>(P);
+  k_attend<<<grid, NTHREADS, sizeof(AttnSmem) + 1024, st>>>(P);
   if (timed) profile_end(st, ev);
   count_launches(1);
   int rc = launch_status();
-  if (rc != ER_OK) return rc;
+  if (rc != ER_OK || P.direct) return rc;
   k_attend_merge<<<dim3(P.nq, NH), 256, 0, st>>>(P.part_o, P.part_ml, P.splits, o_swa, o_rma,
                                                   o_sum);
   count_launches(1);
@@ -483,6 +698,9 @@ int er_swa_rma_attend(const er_state* st, int32_t layer, const int32_t* seq_ids,
   if (!st || B < 0 || layer < 0 || layer >= st->n_layers) return ER_EINVAL;
   if (B == 0) return ER_OK;
   if (!seq_ids || !q_swa || !q_rma || !o_swa || !o_rma || !ws) return ER_EINVAL;
+  if (!aligned16(q_swa) || !aligned16(q_rma) || !aligned16(o_swa) || !aligned16(o_rma) ||
+      !aligned16(ws))
+    return ER_EINVAL;
   if (ws_bytes < er_attend_workspace_bytes(B)) return ER_ECAPACITY;
   Carver c(ws);
   AttendParams P{};

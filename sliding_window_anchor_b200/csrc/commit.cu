@@ -25,6 +25,7 @@ namespace {
 
 constexpr int NSORT = 2048;
 constexpr int CT = 1024;  // threads per commit block
+constexpr int SPB = 32;   // most sequences one block looks after (decode path)
 
 __device__ __forceinline__ uint32_t ordered_score(float s) {
   uint32_t u = __float_as_uint(s);
@@ -74,22 +75,38 @@ __global__ void __launch_bounds__(CT) k_commit(CommitParams P) {
   __shared__ int16_t evict_list[BANK];
   __shared__ int32_t move_src[PEND], move_dst[PEND];
   __shared__ int warp_sums[32];
+  __shared__ int blk_seq[SPB], blk_c[SPB], blk_p[SPB];
 
-  const int b = blockIdx.x;
   const int l = P.layer0 + blockIdx.y / NG;
   const int g = blockIdx.y % NG;
   const int tid = threadIdx.x;
-  const int seq = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b];
+  // each block owns a run of `per_block` listed sequences; their metadata is read
+  // in one parallel load, so the (many) sequences with nothing to commit cost
+  // no serial global-memory latency
+  const int b0 = blockIdx.x * P.per_block;
+  const int nb = min(P.per_block, P.n - b0);
+  if (tid < nb) {
+    const int seq = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b0 + tid];
+    blk_seq[tid] = seq;
+    if (seq >= 0 && seq < P.s_max) {
+      blk_c[tid] = P.meta[seq * 4 + 2];
+      blk_p[tid] = P.meta[seq * 4 + 1] + P.p_add;
+    }
+  }
+  __syncthreads();
+  for (int bi = 0; bi < nb; ++bi) {
+  const int b = b0 + bi;
+  const int seq = blk_seq[bi];
   if (seq < 0 || seq >= P.s_max) {
     if (tid == 0 && blockIdx.y == 0) set_dev_error(P.err, ER_EINVAL);
-    return;
+    continue;
   }
-  const int c = P.meta[seq * 4 + 2];
-  const int p = P.meta[seq * 4 + 1] + P.p_add;
-  if (P.only_if_full && p != PEND) return;
+  const int c = blk_c[bi];
+  const int p = blk_p[bi];
+  if (P.only_if_full && p != PEND) continue;
   if (c < 0 || c > BANK || p < 0 || p > PEND) {
     if (tid == 0) set_dev_error(P.err, ER_ECAPACITY);
-    return;
+    continue;
   }
   const size_t gi = grp(seq, l, g, P.L);
 
@@ -163,6 +180,8 @@ __global__ void __launch_bounds__(CT) k_commit(CommitParams P) {
       P.bank_pos[gi * BANK + d] = P.pend_pos[gi * PEND + j];
     }
   }
+  __syncthreads();  // shared arrays are reused by the next sequence
+  }
 }
 
 __global__ void k_commit_finish(int32_t* meta, const int32_t* seq_ids, int n, int s_max) {
@@ -177,7 +196,10 @@ __global__ void k_commit_finish(int32_t* meta, const int32_t* seq_ids, int n, in
 
 int launch_commit(const CommitParams& P, cudaStream_t st) {
   if (P.n <= 0) return ER_OK;
-  k_commit<<<dim3(P.n, P.nlayers * NG), CT, 0, st>>>(P);
+  CommitParams Q = P;
+  Q.per_block = P.only_if_full ? SPB : 1;
+  const int gx = (P.n + Q.per_block - 1) / Q.per_block;
+  k_commit<<<dim3(gx, P.nlayers * NG), CT, 0, st>>>(Q);
   count_launches(1);
   return launch_status();
 }
@@ -258,6 +280,7 @@ int er_rma_append_pending(const er_state* st, int32_t layer, const int32_t* seq_
   if (!st || n < 0 || layer < 0 || layer >= st->n_layers) return ER_EINVAL;
   if (n > 0 && (!seq_ids || !k || !v || !s || !pos)) return ER_EINVAL;
   if (n == 0) return ER_OK;
+  if (!aligned16(k) || !aligned16(v)) return ER_EINVAL;
   AppendParams P;
   P.pend_k = st->pend_k; P.pend_v = st->pend_v;
   P.pend_score = st->pend_score; P.pend_pos = st->pend_pos;

@@ -146,19 +146,24 @@ __device__ __forceinline__ float4 lds128f(const void* p) {
 
 // ------------------------------------------------------------ host side
 
+// Vector loads and bulk copies need 16-byte aligned rows; entry points reject
+// pointers that are not (ER_EINVAL) instead of letting a kernel fault.
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
 void count_launches(int n);                 // bookkeeping for er_launch_count
 int launch_status();                        // ER_OK or ER_ECUDA after a launch
 int num_sms();                              // SMs of the current device (cached)
 
-// Workspace carving: 256-byte aligned sub-buffers.
+// Workspace carving: 256-byte aligned sub-buffers.  With a null base the
+// returned "pointers" are the byte offsets themselves (layout computation).
 struct Carver {
-  char* base;
+  uintptr_t base;
   size_t off = 0;
-  explicit Carver(void* b) : base((char*)b) {}
+  explicit Carver(void* b) : base((uintptr_t)b) {}
   template <class T>
   T* take(size_t count) {
     off = (off + 255) & ~(size_t)255;
-    T* p = base ? (T*)(base + off) : nullptr;
+    T* p = reinterpret_cast<T*>(base + off);
     off += count * sizeof(T);
     return p;
   }

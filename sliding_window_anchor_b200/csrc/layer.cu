@@ -15,7 +15,8 @@ namespace er {
 int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
                   cudaStream_t st);
 int launch_score(const float* w1, const float* w2, const uint16_t* x, int n, float* s,
-                 cudaStream_t st);
+                 float* part, cudaStream_t st);
+size_t score_part_floats(int n);
 int launch_post_proj(const PostParams& P, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
                   cudaStream_t st);
@@ -31,6 +32,7 @@ namespace {
 struct LayerWs {
   uint16_t* proj;
   float* s;
+  float* score_part;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
   float *part_o, *part_ml;
@@ -43,6 +45,7 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   LayerWs w;
   w.proj = c.take<uint16_t>((size_t)nq * QKV);
   w.s = c.take<float>((size_t)nq * NG);
+  w.score_part = c.take<float>(score_part_floats(nq));
   w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
   w.chunk_k = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
@@ -56,7 +59,9 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
 
 bool weights_ok(const er_layer_weights* w) {
   return w && w->w_qkv && w->w_o && w->q_norm_swa && w->k_norm_swa && w->q_norm_rma &&
-         w->k_norm_rma && w->w1 && w->w2;
+         w->k_norm_rma && w->w1 && w->w2 && aligned16(w->w_qkv) && aligned16(w->w_o) &&
+         aligned16(w->q_norm_swa) && aligned16(w->k_norm_swa) && aligned16(w->q_norm_rma) &&
+         aligned16(w->k_norm_rma) && aligned16(w->w1) && aligned16(w->w2);
 }
 
 // The chunk's window rows enter the ring after all of its reads.
@@ -66,6 +71,7 @@ __global__ void k_ring_write(const uint16_t* chunk_k, const uint16_t* chunk_v, u
   const int i = blockIdx.x, g = blockIdx.y, lane = threadIdx.x & 31, is_v = threadIdx.x >> 5;
   if (seq < 0 || seq >= s_max) return;
   const int t = meta[seq * 4 + 0] + i;
+  if (t < 0) return;
   const size_t row = grp(seq, layer, g, L) * WIN + (size_t)(t % WIN);
   const uint4* src =
       reinterpret_cast<const uint4*>((is_v ? chunk_v : chunk_k) + ((size_t)g * T + i) * D);
@@ -83,7 +89,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   // a1: all six projections in one GEMM
   if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
   // a3: FP32 scores
-  if ((rc = launch_score(w->w1, w->w2, x, nq, W.s, s)) != ER_OK) return rc;
+  if ((rc = launch_score(w->w1, w->w2, x, nq, W.s, W.score_part, s)) != ER_OK) return rc;
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
   pp.proj = W.proj; pp.s = W.s; pp.nq = nq;
@@ -151,6 +157,7 @@ int er_swa_rma_decode(const er_state* st, const er_layer_weights* w, int32_t lay
   if (B == 0) return ER_OK;
   if (B > st->s_max) return ER_ECAPACITY;
   if (!weights_ok(w) || !seq_ids || !x || !out || !ws) return ER_EINVAL;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(ws)) return ER_EINVAL;
   return run_layer(st, w, layer, seq_ids, -1, B, x, out, ws, ws_bytes, (cudaStream_t)stream);
 }
 
@@ -160,6 +167,7 @@ int er_swa_rma_prefill_chunk(const er_state* st, const er_layer_weights* w, int3
   if (!st || layer < 0 || layer >= st->n_layers || T < 1 || T > PEND) return ER_EINVAL;
   if (seq_id < 0 || seq_id >= st->s_max) return ER_EINVAL;
   if (!weights_ok(w) || !x || !out || !ws) return ER_EINVAL;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(ws)) return ER_EINVAL;
   return run_layer(st, w, layer, nullptr, seq_id, T, x, out, ws, ws_bytes,
                    (cudaStream_t)stream);
 }

@@ -29,6 +29,16 @@ __device__ __forceinline__ void store8(uint16_t* dst, const float v[8]) {
   *reinterpret_cast<uint4*>(dst) = w;
 }
 
+// cos/sin of pos * 1e7^(-2i/64) for i = lane (0..31): the angle is formed and
+// reduced in float64 (one evaluation per lane), then rounded to float.
+__device__ __forceinline__ float2 rope_cs_lane(int32_t pos, int lane) {
+  const double kLog2Theta = 23.253496664211536;  // log2(1e7)
+  const double inv_freq = exp2(-(double)lane * (kLog2Theta / 32.0));
+  double sn, cs;
+  sincos((double)pos * inv_freq, &sn, &cs);
+  return make_float2((float)cs, (float)sn);
+}
+
 // y = x / sqrt(mean(x^2) + 1e-6) * gain, then rotate (i, i+32), i < 32.
 __device__ __forceinline__ void norm_rope_lane(float v[8], const uint16_t* gain, int32_t pos,
                                                int lane) {
@@ -42,20 +52,16 @@ __device__ __forceinline__ void norm_rope_lane(float v[8], const uint16_t* gain,
   load8(gain + lane * 8, g);
 #pragma unroll
   for (int e = 0; e < 8; ++e) v[e] = (v[e] * inv) * g[e];
+  const float2 mycs = rope_cs_lane(pos, lane);
   float partner[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(0xffffffffu, v[e], 4);
-  if (lane < 8) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = (lane & 3) * 8 + e;  // frequency index 0..31
-      const double inv_freq = pow(1.0e7, -2.0 * (double)i / (double)ROPE);
-      double sn, cs;
-      sincos((double)pos * inv_freq, &sn, &cs);
-      const float c = (float)cs, s = (float)sn;
-      if (lane < 4) v[e] = v[e] * c - partner[e] * s;        // dim i:    a cos - b sin
-      else v[e] = v[e] * c + partner[e] * s;                 // dim i+32: b cos + a sin
-    }
+  for (int e = 0; e < 8; ++e) {
+    partner[e] = __shfl_xor_sync(0xffffffffu, v[e], 4);
+    // frequency index of this lane's element e (lanes 0..7): 8*(lane&3) + e
+    const float c = __shfl_sync(0xffffffffu, mycs.x, (lane & 3) * 8 + e);
+    const float sn = __shfl_sync(0xffffffffu, mycs.y, (lane & 3) * 8 + e);
+    if (lane < 4) v[e] = v[e] * c - partner[e] * sn;        // dim i:    a cos - b sin
+    else if (lane < 8) v[e] = v[e] * c + partner[e] * sn;   // dim i+32: b cos + a sin
   }
 }
 
@@ -88,7 +94,7 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   const int32_t pend0 = P.meta[seq * 4 + 1];
   const int32_t t = pos0 + (P.prefill ? qi : 0);
   const int p_idx = pend0 + (P.prefill ? qi : 0);
-  const bool state_ok = p_idx < PEND;
+  const bool state_ok = p_idx >= 0 && p_idx < PEND && t >= 0;
   if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
 
   int col;
@@ -113,6 +119,7 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
     if (P.prefill) {
       dst = (is_k ? P.chunk_k : P.chunk_v) + ((size_t)g * P.nq + qi) * D;
     } else {
+      if (t < 0) return;
       const size_t row = grp(seq, P.layer, g, P.L) * WIN + (size_t)(t % WIN);
       dst = (is_k ? P.win_k : P.win_v) + row * D;
     }
@@ -146,6 +153,7 @@ extern "C" int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, con
                                const int32_t* pos, er_stream_t stream) {
   if (n_rows < 0 || (n_rows > 0 && (!x || !y || !gain || !pos))) return ER_EINVAL;
   if (n_rows == 0) return ER_OK;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(gain)) return ER_EINVAL;
   const int64_t blocks = (n_rows + 7) / 8;
   if (blocks > 0x7FFFFFFF) return ER_EINVAL;
   k_norm_rope<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(x, y, n_rows, gain, pos);

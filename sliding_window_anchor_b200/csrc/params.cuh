@@ -2,6 +2,8 @@
 // orchestration (layer.cu).
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace er {
@@ -24,7 +26,13 @@ struct PostParams {
   int32_t* err;
 };
 
+// Tensor maps of the row arrays the reads stream (2-D views [rows][256] BF16,
+// 64x64 boxes, 128-byte swizzle): K and V of window, bank, pending, chunk.
+enum { TM_WIN = 0, TM_BANK = 1, TM_PEND = 2, TM_CHUNK = 3, TM_COUNT = 4 };
+
 struct AttendParams {
+  CUtensorMap tmap_k[TM_COUNT];
+  CUtensorMap tmap_v[TM_COUNT];
   const uint16_t *win_k, *win_v, *bank_k, *bank_v, *pend_k, *pend_v;
   const int32_t* meta;
   const int32_t* seq_ids;
@@ -38,6 +46,11 @@ struct AttendParams {
   int splits;
   float* part_o;   // [items][4][256]
   float* part_ml;  // [items][4][2]
+  // direct output (splits == 1): the CTA that reads a (query, group)'s SWA item
+  // reads its RMA item next and writes the final result itself
+  int direct;
+  float *o_swa, *o_rma;  // FP32 [nq][16][256] (standalone read), or
+  uint16_t* o_sum;       // BF16 [nq][4096] = bf16(o_swa + o_rma) (layer path)
   int32_t* err;
 };
 
@@ -55,6 +68,7 @@ struct CommitParams {
   int layer0, nlayers;
   int p_add;         // pending records = meta.pend + p_add
   int only_if_full;  // commit only when that count is 256
+  int per_block;     // sequences per block (set at launch)
   int32_t* kept;     // optional [n][nlayers][4][1024]
   int32_t* err;
 };

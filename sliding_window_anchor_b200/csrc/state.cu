@@ -41,7 +41,9 @@ struct StateLayout {
 };
 
 bool layout_of(int32_t s_max, int32_t n_layers, StateLayout* L) {
-  if (s_max < 1 || s_max > (1 << 20) || n_layers < 1 || n_layers > ER_MAX_LAYERS) return false;
+  // row indices of every array stay below 2^31 (TMA coordinates are 32-bit): 4096
+  // sequences are 288 GiB of state, more than one GPU holds
+  if (s_max < 1 || s_max > 4096 || n_layers < 1 || n_layers > ER_MAX_LAYERS) return false;
   Carver c(nullptr);
   size_t g = (size_t)s_max * n_layers * NG;
   L->win = (size_t)c.take<uint16_t>(g * WIN * D);

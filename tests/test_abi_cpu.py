@@ -54,6 +54,16 @@ def test_state_bytes_and_carve(L):
               "meta", "dev_error"):
         assert getattr(st, f) % 256 == 0
     assert st.dev_error + 64 * 4 <= fake + n
+    # the carved arrays are disjoint, in order, inside the allocation
+    g = 2 * 8 * 4
+    sizes = {"win_k": g * 1024 * 512, "win_v": g * 1024 * 512, "bank_k": g * 1024 * 512,
+             "bank_v": g * 1024 * 512, "pend_k": g * 256 * 512, "pend_v": g * 256 * 512,
+             "bank_score": g * 1024 * 4, "pend_score": g * 256 * 4, "bank_pos": g * 1024 * 4,
+             "pend_pos": g * 256 * 4, "meta": 2 * 16, "dev_error": 16}
+    spans = sorted((getattr(st, f), getattr(st, f) + b) for f, b in sizes.items())
+    assert spans[0][0] >= fake and spans[-1][1] <= fake + n
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0
     assert L.er_state_carve(ctypes.c_void_p(fake), n - 1, 2, 8, ctypes.byref(st)) == -1
     assert L.er_state_carve(ctypes.c_void_p(fake + 8), n, 2, 8, ctypes.byref(st)) == -1
 
@@ -93,11 +103,19 @@ def test_host_validation_rejects_before_enqueue(L):
     assert L.er_rma_append_pending(ctypes.byref(st), 0, nul, 1, nul, nul, nul, nul, nul) == -1
     assert L.er_advance(ctypes.byref(st), nul, 1, 0, nul) == -1
     assert L.er_advance(ctypes.byref(st), nul, 1, 257, nul) == -1
-    assert L.er_rma_score(None, nul, 1, nul, nul) == -1
+    assert L.er_rma_score(None, nul, 1, nul, nul, 0, nul) == -1
     assert L.er_qk_norm_rope(nul, nul, 4, nul, nul, nul) == -1
+    # misaligned rows are refused (16-byte vector loads and bulk copies need alignment)
+    fake = ctypes.c_void_p((1 << 40) + 2)
+    ok = ctypes.c_void_p(1 << 40)
+    before = L.er_launch_count()
+    assert L.er_qk_norm_rope(fake, ok, 4, ok, ok, nul) == -1
+    assert L.er_swa_rma_attend(ctypes.byref(st), 0, ok, 1, fake, ok, ok, ok, ok, 1 << 30,
+                               nul) == -1
+    assert L.er_launch_count() == before
     # empty work is fine and launches nothing
     before = L.er_launch_count()
-    assert L.er_rma_score(ctypes.byref(w), nul, 0, nul, nul) == 0
+    assert L.er_rma_score(ctypes.byref(w), nul, 0, nul, nul, 0, nul) == 0
     assert L.er_qk_norm_rope(nul, nul, 0, nul, nul, nul) == 0
     assert L.er_launch_count() == before
     assert L.er_error_string(-2) == b"capacity exceeded"
