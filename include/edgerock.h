@@ -161,6 +161,28 @@ size_t er_score_workspace_bytes(int32_t n);
 int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
                  size_t ws_bytes, er_stream_t stream);
 
+/* a3 without caller scratch.  The pages describe nothing like this; it exists
+ * for callers that cannot hand the library any device memory beyond the
+ * inputs and outputs, so cannot provide er_rma_score's workspace: for example
+ * a host program whose device memory is all owned by another framework's
+ * caching allocator, or a plugin interface that only receives tensor pointers
+ * and may not call cudaMalloc itself.  Same result as er_rma_score.
+ *  - The split-K partial sums live in one fixed device array inside the
+ *    library (ER_SCORE_NOALLOC_MAX_TOKENS x 16 x 256 floats = 4 MiB), which
+ *    every GPU that loads the library holds until the process exits.
+ *  - n above ER_SCORE_NOALLOC_MAX_TOKENS returns ER_ECAPACITY; nothing runs.
+ *  - The first call on a device (with that device current) looks the array's
+ *    device address up with cudaGetSymbolAddress and caches it; make that
+ *    first call before any stream capture on the device.
+ *  - Nothing is allocated or freed: no cudaMalloc, no cudaFree.
+ *  - Every call shares the one array: calls whose work overlaps on the GPU
+ *    (different streams, or different threads on one device) race and give
+ *    wrong scores; serialise them.  The array keeps the last call's contents;
+ *    no part of it needs to start at zero. */
+#define ER_SCORE_NOALLOC_MAX_TOKENS 256
+int er_rma_score_noalloc(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s,
+                         er_stream_t stream);
+
 /* a4 — appends one candidate record per KV group for each listed sequence at
  * its pend_count slot of `layer` [N-rma]: k, v BF16 [n][4][256] (k already
  * normed and rotated), s FP32 [n][4], pos INT32 [n].  Metadata is not

@@ -25,7 +25,7 @@ __all__ = ["State", "LayerWeights", "qk_norm_rope", "rma_score", "rma_append_pen
            "rma_commit", "swa_rma_attend", "swa_rma_decode", "swa_rma_prefill_chunk",
            "advance", "state_init", "last_device_error", "launch_count", "profile_enable",
            "profile_read", "decode_workspace_bytes", "prefill_workspace_bytes",
-           "attend_workspace_bytes", "score_workspace_bytes", "ERError"]
+           "attend_workspace_bytes", "score_workspace_bytes", "rma_score_noalloc", "ERError"]
 
 
 class State:
@@ -146,6 +146,16 @@ def rma_score(w: LayerWeights, x: torch.Tensor, ws=None, stream=None):
     check("er_rma_score", lib().er_rma_score(w.ptr(), dev_ptr(x, torch.bfloat16, "x"), n,
                                              dev_ptr(s), dev_ptr(ws), ws.numel(),
                                              stream_handle(stream, x.device)))
+    return s
+
+
+def rma_score_noalloc(w: LayerWeights, x: torch.Tensor, stream=None):
+    """er_rma_score without a workspace: the scratch is a fixed array inside the
+    library (at most ER_SCORE_NOALLOC_MAX_TOKENS = 256 tokens per call)."""
+    n = x.numel() // HIDDEN
+    s = torch.empty(n, NG, dtype=torch.float32, device=x.device)
+    check("er_rma_score_noalloc", lib().er_rma_score_noalloc(
+        w.ptr(), dev_ptr(x, torch.bfloat16, "x"), n, dev_ptr(s), stream_handle(stream, x.device)))
     return s
 
 

@@ -56,6 +56,8 @@ EXPORTS = {
     "er_rma_score": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p, ctypes.c_int32,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                     ctypes.c_void_p]),
+    "er_rma_score_noalloc": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p,
+                                            ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     "er_rma_append_pending": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_int32,
                                              ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,

@@ -14,6 +14,8 @@
 //  stage 2: per token, the splits are summed in a fixed order, SiLU, and the
 //    256→4 contraction is a block reduction.
 // The partials live in caller-provided workspace (er_score_workspace_bytes).
+#include <mutex>
+
 #include "common.cuh"
 
 namespace er {
@@ -153,9 +155,55 @@ int launch_score(const float* w1, const float* w2, const uint16_t* x, int n, flo
 
 }  // namespace er
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant.  The split-K partial sums normally live in scratch
+// the caller passes in; here they live in this fixed array, which every GPU
+// that loads the library keeps for the life of the process (ER_SCORE_NOALLOC_
+// MAX_TOKENS x 16 splits x 256 floats = 4 MiB).  Host code must not hand the
+// array's name to a kernel: on the host it only stands in for the symbol, so
+// its device address is looked up with cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) float g_score_noalloc_scratch[(size_t)16 *
+                                                               ER_SCORE_NOALLOC_MAX_TOKENS *
+                                                               er::SH];
+
+namespace er {
+namespace {
+
+static_assert(KSPLIT == 16, "the allocation-free scratch is sized for 16 K splits");
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[64] = {nullptr};
+
+}  // namespace
+}  // namespace er
+
 using namespace er;
 
 extern "C" {
+
+int er_rma_score_noalloc(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s,
+                         er_stream_t stream) {
+  if (!w || n < 0 || (n > 0 && (!w->w1 || !w->w2 || !x || !s))) return ER_EINVAL;
+  if (n > ER_SCORE_NOALLOC_MAX_TOKENS) return ER_ECAPACITY;
+  if (n == 0) return ER_OK;
+  if (!aligned16(w->w1) || ((uintptr_t)x & 3u)) return ER_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ER_ECUDA;
+  float* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      // first call on this device (which is current): find the array's device address
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_score_noalloc_scratch) != cudaSuccess || !p)
+        return ER_ECUDA;
+      g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  // every split's partial sums are written before they are read: nothing to clear
+  return launch_score(w->w1, w->w2, x, n, s, scratch, (cudaStream_t)stream);
+}
 
 size_t er_score_workspace_bytes(int32_t n) {
   if (n < 0) return 0;
