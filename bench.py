@@ -41,6 +41,11 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-commit-bench", action="store_true")
+    ap.add_argument("--kernel", default="step", choices=["step", "attend", "commit"],
+                    help="step: the benchmark; attend/commit: one kernel alone at --batch "
+                         "sequences (profiling driver)")
+    ap.add_argument("--batch", type=int, default=256)
     return ap.parse_args()
 
 
@@ -105,6 +110,26 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
                 "samples": len(sm)}
+
+
+# ------------------------------------------------------------ multi-rank
+
+def reduce_max(value: float, device) -> float:
+    """Max of a float over all ranks (identity without a process group).  Every
+    rank calls it at the same points, in warm-up, timing and error paths alike."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_per_s(world: int, batch: int, steps: int, max_ms: float) -> float:
+    """Weak scaling: every rank decodes its own batch; the job's rate uses the
+    slowest rank's time."""
+    return world * batch * steps / (max_ms / 1e3)
 
 
 # --------------------------------------------------------------- our arm
@@ -214,21 +239,116 @@ def run_ours(args, rank, world, local_rank):
                 hout[l].copy_(outs[l], non_blocking=True)
         f1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = f0.elapsed_time(f1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t)
+        e2e_ms = reduce_max(f0.elapsed_time(f1), dev)
         nbytes = LAYERS * B * 2560 * 2
-        e2e = {"value": world * B * k_e2e / (e2e_ms / 1e3), "unit": "tok/s",
+        e2e = {"value": whole_job_tokens_per_s(world, B, k_e2e, e2e_ms), "unit": "tok/s",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "steps": k_e2e}
 
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t)
+    ms = reduce_max(ms, dev)
+    cm = None
+    if not args.no_commit_bench and rank == 0:
+        # the commit microbench reuses the decode state's memory (B=512 x 8 layers)
+        cm = commit_microbench(st, dev)
     return dict(ms=ms, launches=launches, clocks=clk, attend_ms=attend_ms, attend_n=attend_n,
-                fills=fills, commits=commits, e2e=e2e)
+                fills=fills, commits=commits, e2e=e2e, commit_microbench=cm)
+
+
+# ------------------------------------------------------- commit microbench
+
+def seed_commit_workload(st, seed, rep, dev):
+    """The commit workload: every (sequence, layer, group) holds a full bank and a
+    full pending block; scores N(0,1) with ~5% exact ties inside each merge; K/V
+    rows N(0,1).  Repetition r re-seeds the pending block (scores, positions
+    t0+256r+j) on top of the bank the previous repetition left."""
+    import torch
+    import synth
+    from synth import workloads as wl
+    n, L = st.s_max, st.n_layers
+    if rep == 0:
+        wl.seed_state(st.arrays(), range(n), L, T0, "full", seed, [None] * L, None, device=dev,
+                      plain_keys=True, dup_scores=True)
+    else:
+        synth.fill_normal_dup_(st.pend_score, seed + rep, synth.PEND_SCORE, 256, 20)
+    j = torch.arange(256, dtype=torch.int32, device=dev)
+    st.pend_pos.copy_((T0 + 256 * rep + j).view(1, 1, 1, 256).expand_as(st.pend_pos))
+    st.meta[:, 0] = T0 + 256 * (rep + 1)
+    st.meta[:, 1] = 256
+    st.meta[:, 2] = 1024
+
+
+def commit_microbench(st, dev, reps=3):
+    """Times er_rma_commit(layer=-1) over every sequence: B x 8 layers x 4 groups
+    independent top-1024-of-1280 merges.  Algorithmic bytes per merge: the 1280
+    keys (score + position, 8 B each) read, plus each moved record's K and V row
+    read and written (2 x 1 KiB) with its score and position (2 x 8 B)."""
+    import torch
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+    seed = wl.seed_of(1)
+    ids = torch.arange(st.s_max, dtype=torch.int32, device=dev)
+    merges = st.s_max * st.n_layers * 4
+    times, moved = [], []
+    for rep in range(reps + 1):
+        seed_commit_workload(st, seed, rep, dev)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        sab.rma_commit(st, -1, ids)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        if sab.last_device_error(st) != 0:
+            raise RuntimeError("device error in the commit microbench")
+        if rep > 0:  # the first repetition is the warm-up
+            times.append(e0.elapsed_time(e1))
+            moved.append(int((st.bank_pos >= T0 + 256 * rep).sum()))
+    i = sorted(range(reps), key=lambda k: times[k])[reps // 2]
+    ms, m = times[i], moved[i]
+    alg = merges * 1280 * 8 + m * (2 * 1024 + 16)
+    hbm, kind = peaks()
+    return {"workload": f"commit_b{st.s_max}_l{st.n_layers}", "merges": merges, "ms": ms,
+            "merges_per_s": merges / (ms / 1e3),
+            "sequence_commits_per_s": st.s_max / (ms / 1e3),
+            "moved_records": m, "alg_bytes": alg, "achieved_gbs": alg / (ms / 1e3) / 1e9,
+            "frac": alg / (ms / 1e3) / 1e9 / hbm, "peak_gbs": hbm, "peak_kind": kind}
+
+
+def single_kernel(args):
+    """Profiling driver: one kernel alone on a --batch workload, three launches."""
+    import torch
+    import synth
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+    dev = torch.device("cuda", 0)
+    B = args.batch
+    if args.kernel == "attend":
+        seed = 5
+        w = wl.make_weights(seed, 0, device=dev)
+        st = sab.State(B, 1)
+        nr = lambda x, g, p: sab.qk_norm_rope(x.contiguous(), g, p.to(torch.int32).contiguous())
+        fills = wl.seed_state(st.arrays(), range(B), 1, T0, "uniform", seed, [w], nr, device=dev)
+        q1 = synth.normal((B, 16, 256), seed, 900, torch.bfloat16, dev)
+        q2 = synth.normal((B, 16, 256), seed, 901, torch.bfloat16, dev)
+        ids = torch.arange(B, dtype=torch.int32, device=dev)
+        ws = torch.empty(sab.attend_workspace_bytes(B), dtype=torch.uint8, device=dev)
+        ms = []
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sab.swa_rma_attend(st, 0, ids, q1, q2, ws=ws)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        alg = sum(4 * ((2048 + int(f) + 1) * ROW + 2 * 4 * 512 + 2 * 4 * 1024)
+                  for f in fills.tolist())
+        if sab.last_device_error(st) != 0:
+            raise RuntimeError("device error")
+        out = {"kernel": "k_attend", "batch": B, "layers": 1, "ms": ms[-1], "alg_bytes": alg,
+               "gbs": alg / (ms[-1] / 1e3) / 1e9}
+    else:
+        st = sab.State(B, LAYERS)
+        r = commit_microbench(st, dev, reps=2)
+        out = {"kernel": "k_commit", "batch": B, **r}
+    print(json.dumps(out), flush=True)
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -303,6 +423,9 @@ def main():
     if args.impl == "reference":
         reference_arm(args, rank, world)
         return
+    if args.kernel != "step":
+        single_kernel(args)
+        return
     import torch
     import torch.distributed as dist
     if world > 1:
@@ -324,7 +447,12 @@ def main():
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "attend_traffic.json")
     if os.path.exists(tpath):
-        traffic = json.load(open(tpath)).get("bytes_per_launch_full")
+        # DRAM traffic from the committed ncu capture; null once the kernel source has changed
+        import hashlib
+        rec = json.load(open(tpath))
+        src = os.path.join(ROOT, rec["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest() == rec.get("source_sha256"):
+            traffic = rec.get("bytes_per_launch_full")
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         v, cores, toks, dt = oracle_tokens_per_s(budget_s=12.0)
@@ -332,9 +460,9 @@ def main():
                "sample": f"{toks} whole 8-layer decode steps of {cores} sequences of the "
                          f"workload in {dt:.1f} s"}
     secs = r["ms"] / 1e3
-    toks = world * B * args.steps
     line = {
-        "metric": METRIC, "value": toks / secs, "unit": "tok/s", "n_gpus": world,
+        "metric": METRIC, "value": whole_job_tokens_per_s(world, B, args.steps, r["ms"]),
+        "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -352,6 +480,7 @@ def main():
         "e2e": r["e2e"],
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
+        "commit_microbench": r["commit_microbench"],
     }
     print(json.dumps(line), flush=True)
 
