@@ -7,10 +7,13 @@
 // anchors are never rewritten.  Ties go to the lower source position (the
 // reading fixed for this library), -0 ranks as +0 and NaN below every number.
 //
-// One 1024-thread block per (sequence, layer, group):
+// One 256-thread block per (sequence, layer, group), up to 4 blocks per SM:
 //  1. 64-bit keys (ordered score << 32 | ~position) for the ≤1280 records,
-//     padded to 2048 with key 0, which ranks below every real record;
-//  2. bitonic sort in shared memory (descending), carrying the source index;
+//     padded to 2048 with key 0, which ranks below every real record; each
+//     thread holds 8 consecutive keys (and their source indices) in registers;
+//  2. bitonic sort, descending: partner strides below 8 inside a thread, 8..128
+//     between the lanes of a warp (shuffles), 256 and up through shared memory
+//     (12 block barriers in all);
 //  3. flags for the top min(1024, c+p); two block scans give the evicted
 //     bank slots (ascending) and the pending winners (ascending);
 //  4. each warp moves winners' K and V rows (512 B each, 16 B per lane) into
@@ -24,7 +27,9 @@ namespace er {
 namespace {
 
 constexpr int NSORT = 2048;
-constexpr int CT = 1024;  // threads per commit block
+constexpr int CT = 256;   // threads per commit block
+constexpr int EPT = NSORT / CT;  // 8 keys per thread
+constexpr int CW = CT / 32;      // warps per block
 constexpr int SPB = 32;   // most sequences one block looks after (decode path)
 
 __device__ __forceinline__ uint32_t ordered_score(float s) {
@@ -38,7 +43,7 @@ __device__ __forceinline__ uint64_t rec_key(float s, int32_t pos) {
   return ((uint64_t)ordered_score(s) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)pos);
 }
 
-// Exclusive scan over the 1024 threads of a block; *total gets the sum.
+// Exclusive scan over the CT threads of a block; *total gets the sum.
 __device__ int block_scan_excl(int v, int* warp_sums, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
@@ -50,32 +55,167 @@ __device__ int block_scan_excl(int v, int* warp_sums, int* total) {
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_sums[lane];
+    int w = lane < CW ? warp_sums[lane] : 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
+    for (int o = 1; o < CW; o <<= 1) {
       int y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    warp_sums[lane] = w;  // inclusive
+    if (lane < CW) warp_sums[lane] = w;  // inclusive
   }
   __syncthreads();
   const int base = warp ? warp_sums[warp - 1] : 0;
-  *total = warp_sums[31];
+  *total = warp_sums[CW - 1];
   __syncthreads();
   return base + x - v;
+}
+
+// Compare-exchange toward descending order when `desc`, ascending otherwise.
+__device__ __forceinline__ void cas(uint64_t& ka, uint32_t& sa, uint64_t& kb, uint32_t& sb,
+                                    bool desc) {
+  if (desc ? (ka < kb) : (ka > kb)) {
+    const uint64_t tk = ka;
+    ka = kb;
+    kb = tk;
+    const uint32_t ts = sa;
+    sa = sb;
+    sb = ts;
+  }
+}
+
+// Bitonic sort (descending) of 2048 keys held 8 per thread: element i = 8*tid + e.
+__device__ void sort2048(uint64_t (&key)[EPT], uint32_t (&src)[EPT], uint64_t* skey,
+                         uint16_t* ssrc) {
+  const int tid = threadIdx.x, lane = tid & 31;
+#pragma unroll
+  for (int k = 2; k <= NSORT; k <<= 1) {
+    int j = k >> 1;
+    if (j >= 256) {
+      // strides that cross warps: through shared memory, disjoint pairs per thread
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        skey[tid * EPT + e] = key[e];
+        ssrc[tid * EPT + e] = (uint16_t)src[e];
+      }
+      __syncthreads();
+#pragma unroll
+      for (; j >= 256; j >>= 1) {
+#pragma unroll
+        for (int q = 0; q < (NSORT / 2) / CT; ++q) {
+          const int pr = q * CT + tid;  // pair index 0..1023
+          const int i = ((pr & ~(j - 1)) << 1) | (pr & (j - 1));
+          const int m = i | j;
+          uint64_t a = skey[i], b = skey[m];
+          uint32_t sa = ssrc[i], sb = ssrc[m];
+          cas(a, sa, b, sb, (i & k) == 0);
+          skey[i] = a;
+          skey[m] = b;
+          ssrc[i] = (uint16_t)sa;
+          ssrc[m] = (uint16_t)sb;
+        }
+        __syncthreads();
+      }
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        key[e] = skey[tid * EPT + e];
+        src[e] = ssrc[tid * EPT + e];
+      }
+    }
+#pragma unroll
+    for (; j >= EPT; j >>= 1) {
+      // partner element i ^ j is element e of lane lane ^ (j / 8)
+      const int pl = j / EPT;
+      const bool lower = (lane & pl) == 0;
+      const bool desc = ((tid * EPT) & k) == 0;
+      const bool keep_max = lower == desc;
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        const uint64_t b = __shfl_xor_sync(0xffffffffu, key[e], pl);
+        const uint32_t sb = __shfl_xor_sync(0xffffffffu, src[e], pl);
+        const bool take = keep_max ? (b > key[e]) : (b < key[e]);
+        if (take) {
+          key[e] = b;
+          src[e] = sb;
+        }
+      }
+    }
+#pragma unroll
+    for (; j >= 1; j >>= 1) {
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        if ((e & j) == 0)
+          cas(key[e], src[e], key[e | j], src[e | j], ((tid * EPT + e) & k) == 0);
+      }
+    }
+  }
 }
 
 }  // namespace
 
 
-__global__ void __launch_bounds__(CT) k_commit(CommitParams P) {
-  __shared__ uint64_t key[NSORT];
-  __shared__ uint16_t src[NSORT];
+// K-th largest of the block's keys (keys unique, 0 = padding), by radix select on
+// 8-bit digits from the top: each pass histograms the digit of the keys that
+// still match the chosen prefix, and a suffix scan over the 256 bins finds the
+// bin holding rank K.  Returns a (prefix, shift) pair such that a key is among
+// the top K exactly when (key >> shift) >= (prefix >> shift).
+__device__ void radix_select(const uint64_t (&key)[5], int K, int* hist, int* warp_sums,
+                             int* sel, uint64_t* out_prefix, int* out_shift) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint64_t prefix = 0, mask = 0;
+  int need = K;
+  int shift = 64;
+  while (shift > 0) {
+    shift -= 8;
+    hist[tid] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < 5; ++q)
+      if (key[q] != 0 && (key[q] & mask) == prefix)
+        atomicAdd(&hist[(int)((key[q] >> shift) & 255u)], 1);
+    __syncthreads();
+    // inclusive suffix sum S(i) = sum_{d >= i} hist[d], thread i = bin 255 - tid
+    const int bin = 255 - tid;
+    int x = hist[bin];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_sums[w];
+    const int S = base + x;              // keys with digit >= bin
+    const int above = S - hist[bin];     // keys with digit > bin
+    if (S >= need && above < need) {
+      sel[0] = bin;
+      sel[1] = above;
+      sel[2] = hist[bin];
+    }
+    __syncthreads();
+    const int b = sel[0];
+    need -= sel[1];
+    prefix |= (uint64_t)b << shift;
+    mask |= (uint64_t)255 << shift;
+    const int in_bin = sel[2];
+    __syncthreads();  // sel and hist are rewritten by the next pass
+    if (in_bin == need) break;  // every key of the boundary bin is kept
+  }
+  *out_prefix = prefix;
+  *out_shift = shift;
+}
+
+__global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
+  __shared__ uint64_t skey[NSORT];
+  __shared__ uint16_t ssrc[NSORT];
   __shared__ uint8_t flag[BANK + PEND];
   __shared__ int16_t evict_list[BANK];
-  __shared__ int32_t move_src[PEND], move_dst[PEND];
-  __shared__ int warp_sums[32];
+  __shared__ int16_t move_src[PEND], move_dst[PEND];
+  __shared__ int warp_sums[CW];
   __shared__ int blk_seq[SPB], blk_c[SPB], blk_p[SPB];
+  __shared__ int hist[256];
+  __shared__ int sel[4];
 
   const int l = P.layer0 + blockIdx.y / NG;
   const int g = blockIdx.y % NG;
@@ -95,92 +235,133 @@ __global__ void __launch_bounds__(CT) k_commit(CommitParams P) {
   }
   __syncthreads();
   for (int bi = 0; bi < nb; ++bi) {
-  const int b = b0 + bi;
-  const int seq = blk_seq[bi];
-  if (seq < 0 || seq >= P.s_max) {
-    if (tid == 0 && blockIdx.y == 0) set_dev_error(P.err, ER_EINVAL);
-    continue;
-  }
-  const int c = blk_c[bi];
-  const int p = blk_p[bi];
-  if (P.only_if_full && p != PEND) continue;
-  if (c < 0 || c > BANK || p < 0 || p > PEND) {
-    if (tid == 0) set_dev_error(P.err, ER_ECAPACITY);
-    continue;
-  }
-  const size_t gi = grp(seq, l, g, P.L);
+    const int b = b0 + bi;
+    const int seq = blk_seq[bi];
+    if (seq < 0 || seq >= P.s_max) {
+      if (tid == 0 && blockIdx.y == 0) set_dev_error(P.err, ER_EINVAL);
+      continue;
+    }
+    const int c = blk_c[bi];
+    const int p = blk_p[bi];
+    if (P.only_if_full && p != PEND) continue;
+    if (c < 0 || c > BANK || p < 0 || p > PEND) {
+      if (tid == 0) set_dev_error(P.err, ER_ECAPACITY);
+      continue;
+    }
+    const size_t gi = grp(seq, l, g, P.L);
 
-  for (int i = tid; i < NSORT; i += CT) {
-    uint64_t k = 0;
-    if (i < c) k = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
-    else if (i >= BANK && i < BANK + p)
-      k = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
-    key[i] = k;
-    src[i] = (uint16_t)i;
-  }
-  for (int i = tid; i < BANK + PEND; i += CT) flag[i] = 0;
-  __syncthreads();
-
-  // bitonic sort, descending
-  for (int k = 2; k <= NSORT; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      const int i = ((tid & ~(j - 1)) << 1) | (tid & (j - 1));
-      const int m = i | j;
-      const uint64_t a = key[i], bb = key[m];
-      const bool desc = (i & k) == 0;
-      if (desc ? (a < bb) : (a > bb)) {
-        key[i] = bb;
-        key[m] = a;
-        const uint16_t t = src[i];
-        src[i] = src[m];
-        src[m] = t;
+    const int K = min(BANK, c + p);
+    for (int i = tid; i < BANK + PEND; i += CT) flag[i] = 0;
+    if (P.kept == nullptr) {
+      // only the kept set is needed: radix-select the K-th largest key
+      uint64_t key5[5];  // records tid + 256*q (bank 0..1023, then pending)
+#pragma unroll
+      for (int q = 0; q < 5; ++q) {
+        const int i = tid + CT * q;
+        uint64_t kv = 0;
+        if (i < BANK) {
+          if (i < c) kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
+        } else if (i - BANK < p) {
+          kv = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
+        }
+        key5[q] = kv;
       }
-      __syncthreads();
+      uint64_t prefix = 0;
+      int shift = 64;
+      if (c + p > BANK) radix_select(key5, K, hist, warp_sums, sel, &prefix, &shift);
+      __syncthreads();  // flags cleared before they are set
+#pragma unroll
+      for (int q = 0; q < 5; ++q)
+        if (key5[q] != 0 && (shift >= 64 || (key5[q] >> shift) >= (prefix >> shift)))
+          flag[tid + CT * q] = 1;
+    } else {
+      // the ranked list is wanted: full bitonic sort, elements 8*tid .. 8*tid+7
+      uint64_t key[EPT];
+      uint32_t src[EPT];
+#pragma unroll
+      for (int e = 0; e < EPT; ++e) {
+        const int i = tid * EPT + e;
+        uint64_t kv = 0;
+        if (i < c) kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
+        else if (i >= BANK && i < BANK + p)
+          kv = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
+        key[e] = kv;
+        src[e] = (uint32_t)i;
+      }
+      sort2048(key, src, skey, ssrc);
+      __syncthreads();  // flags cleared before they are set
+      // rank r = 8*tid + e
+#pragma unroll
+      for (int e = 0; e < EPT; ++e)
+        if (tid * EPT + e < K) flag[src[e]] = 1;
+      if (tid * EPT < BANK) {
+        int32_t* kp = P.kept + (((size_t)b * P.nlayers + (l - P.layer0)) * NG + g) * BANK;
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+          const int r = tid * EPT + e;
+          kp[r] = r < K ? (int32_t)src[e] : -1;
+        }
+      }
     }
-  }
+    __syncthreads();
 
-  const int K = min(BANK, c + p);
-  if (tid < K) flag[src[tid]] = 1;
-  if (P.kept) {
-    int32_t* kp = P.kept + (((size_t)b * P.nlayers + (l - P.layer0)) * NG + g) * BANK;
-    kp[tid] = tid < K ? (int32_t)src[tid] : -1;
-  }
-  __syncthreads();
-
-  // evicted bank slots, ascending
-  int total_evict = 0;
-  const int ev = (tid < c && !flag[tid]) ? 1 : 0;
-  const int ev_rank = block_scan_excl(ev, warp_sums, &total_evict);
-  if (ev) evict_list[ev_rank] = (int16_t)tid;
-  // pending winners, ascending pending index
-  int total_win = 0;
-  const int wn = (tid < p && flag[BANK + tid]) ? 1 : 0;
-  const int w_rank = block_scan_excl(wn, warp_sums, &total_win);
-  __syncthreads();
-  if (wn) {
-    const int dst = w_rank < total_evict ? (int)evict_list[w_rank] : c + (w_rank - total_evict);
-    move_src[w_rank] = tid;
-    move_dst[w_rank] = dst;
-  }
-  __syncthreads();
-
-  // move rows: one warp per winner, 16 bytes per lane per row
-  const int warp = tid >> 5, lane = tid & 31;
-  for (int w = warp; w < total_win; w += CT / 32) {
-    const int j = move_src[w], d = move_dst[w];
-    const uint4* sk = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + j) * D);
-    const uint4* sv = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + j) * D);
-    uint4* dk = reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + d) * D);
-    uint4* dv = reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + d) * D);
-    const uint4 a = sk[lane], a2 = sv[lane];
-    dk[lane] = a;
-    dv[lane] = a2;
-    if (lane == 0) {
-      P.bank_score[gi * BANK + d] = P.pend_score[gi * PEND + j];
-      P.bank_pos[gi * BANK + d] = P.pend_pos[gi * PEND + j];
+    // evicted bank slots, ascending (4 slots per thread)
+    int ev[4], nev = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int slot = tid * 4 + q;
+      ev[q] = (slot < c && !flag[slot]) ? 1 : 0;
+      nev += ev[q];
     }
-  }
-  __syncthreads();  // shared arrays are reused by the next sequence
+    int total_evict = 0;
+    int er = block_scan_excl(nev, warp_sums, &total_evict);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (ev[q]) evict_list[er++] = (int16_t)(tid * 4 + q);
+    // pending winners, ascending pending index (one per thread)
+    int total_win = 0;
+    const int wn = (tid < p && flag[BANK + tid]) ? 1 : 0;
+    const int w_rank = block_scan_excl(wn, warp_sums, &total_win);
+    __syncthreads();
+    if (wn) {
+      const int dst =
+          w_rank < total_evict ? (int)evict_list[w_rank] : c + (w_rank - total_evict);
+      move_src[w_rank] = (int16_t)tid;
+      move_dst[w_rank] = (int16_t)dst;
+    }
+    __syncthreads();
+
+    // move rows: one warp per winner, 16 bytes per lane per row, two winners in flight
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int w = warp; w < total_win; w += 2 * CW) {
+      const int w2 = w + CW;
+      const int j = move_src[w], d = move_dst[w];
+      const uint4 a = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + j) * D)[lane];
+      const uint4 a2 = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + j) * D)[lane];
+      uint4 bq = make_uint4(0, 0, 0, 0), bq2 = bq;
+      int j2 = 0, d2 = 0;
+      if (w2 < total_win) {
+        j2 = move_src[w2];
+        d2 = move_dst[w2];
+        bq = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + j2) * D)[lane];
+        bq2 = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + j2) * D)[lane];
+      }
+      reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + d) * D)[lane] = a;
+      reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + d) * D)[lane] = a2;
+      if (lane == 0) {
+        P.bank_score[gi * BANK + d] = P.pend_score[gi * PEND + j];
+        P.bank_pos[gi * BANK + d] = P.pend_pos[gi * PEND + j];
+      }
+      if (w2 < total_win) {
+        reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + d2) * D)[lane] = bq;
+        reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + d2) * D)[lane] = bq2;
+        if (lane == 0) {
+          P.bank_score[gi * BANK + d2] = P.pend_score[gi * PEND + j2];
+          P.bank_pos[gi * BANK + d2] = P.pend_pos[gi * PEND + j2];
+        }
+      }
+    }
+    __syncthreads();  // shared arrays are reused by the next sequence
   }
 }
 

@@ -132,16 +132,19 @@ def _tweak_ties(ost):
         ps[g, 3] = 100.0
 
 
+@pytest.mark.parametrize("want_kept", [True, False])
 @pytest.mark.parametrize("c,p,tweak", [(1024, 256, None), (1024, 256, _tweak_ties),
                                        (700, 256, None), (0, 256, None), (1024, 37, None),
-                                       (1000, 100, None), (1024, 0, None)])
-def test_commit_bit_exact(sab, c, p, tweak):
+                                       (1000, 100, None), (1024, 0, None), (900, 200, None)])
+def test_commit_bit_exact(sab, c, p, tweak, want_kept):
+    # with the ranked list requested the kernel sorts; without it, it radix-selects
     ost = _commit_state(50 + c + p, c, p, tweak=tweak)
     st = sab.State(1, 1)
     H.upload_state(st, ost)
     ref_kept = ost.commit(-1, 0, want_kept=True)
-    kept = sab.rma_commit(st, -1, [0], want_kept=True).cpu()
-    assert torch.equal(kept[0], ref_kept)
+    kept = sab.rma_commit(st, -1, [0], want_kept=want_kept)
+    if want_kept:
+        assert torch.equal(kept.cpu()[0], ref_kept)
     for n in oracle.OracleState.ARRAYS:
         assert torch.equal(getattr(st, n).cpu(), getattr(ost, n)), n
     assert sab.last_device_error(st) == 0
