@@ -167,9 +167,10 @@ int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* 
  * a host program whose device memory is all owned by another framework's
  * caching allocator, or a plugin interface that only receives tensor pointers
  * and may not call cudaMalloc itself.  Same result as er_rma_score.
- *  - The split-K partial sums live in one fixed device array inside the
- *    library (ER_SCORE_NOALLOC_MAX_TOKENS x 16 x 256 floats = 4 MiB), which
- *    every GPU that loads the library holds until the process exits.
+ *  - Its scratch (W1 split into three BF16 terms, 3.75 MiB, plus 8 partial
+ *    scores per token and group, 32 KiB at 256 tokens) lives in one fixed
+ *    4 MiB device array inside the library, which every GPU that loads the
+ *    library holds until the process exits.
  *  - n above ER_SCORE_NOALLOC_MAX_TOKENS returns ER_ECAPACITY; nothing runs.
  *  - The first call on a device (with that device current) looks the array's
  *    device address up with cudaGetSymbolAddress and caches it; make that

@@ -43,6 +43,7 @@
 
 #include "common.cuh"
 #include "params.cuh"
+#include "tc.cuh"
 
 namespace er {
 
@@ -600,32 +601,9 @@ size_t attend_ml_floats(int nq) { return (size_t)nq * NG * 2 * attend_splits(nq)
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // 2-D map of `rows` contiguous 512-byte BF16 rows; 64x64 boxes, 128-byte swizzle.
 bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows) {
-  auto fn = encode_fn();
-  if (!fn || rows == 0 || ((uintptr_t)base & 15u)) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)ROW_BYTES};
-  const cuuint32_t box[2] = {64, 64};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
+  return encode_bf16_2d(m, base, D, rows, ROW_BYTES, 64, 64);
 }
 
 }  // namespace

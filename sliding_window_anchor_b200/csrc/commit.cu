@@ -8,14 +8,16 @@
 // reading fixed for this library), -0 ranks as +0 and NaN below every number.
 //
 // One 256-thread block per (sequence, layer, group), up to 4 blocks per SM:
-//  1. 64-bit keys (ordered score << 32 | ~position) for the ≤1280 records,
-//     padded to 2048 with key 0, which ranks below every real record; each
-//     thread holds 8 consecutive keys (and their source indices) in registers;
-//  2. bitonic sort, descending: partner strides below 8 inside a thread, 8..128
-//     between the lanes of a warp (shuffles), 256 and up through shared memory
-//     (12 block barriers in all);
-//  3. flags for the top min(1024, c+p); two block scans give the evicted
-//     bank slots (ascending) and the pending winners (ascending);
+//  1. 64-bit keys (ordered score << 32 | ~position) for the ≤1280 records;
+//     key 0 (padding, empty slots) ranks below every real record;
+//  2. the kept set: when no ranked list is requested, a radix select on 8-bit
+//     digits finds the K-th largest key (K = min(1024, c+p)), usually in two
+//     or three histogram passes; when the ranked list is requested, a bitonic
+//     sort (descending) of 2048 keys, 8 per thread in registers: partner
+//     strides below 8 inside a thread, 8..128 across lanes (shuffles), 256 and
+//     up through shared memory;
+//  3. flags for the kept records; two block scans give the evicted bank slots
+//     (ascending) and the pending winners (ascending);
 //  4. each warp moves winners' K and V rows (512 B each, 16 B per lane) into
 //     their target slots, with the score and position.
 // Surviving anchors are not touched, so the write traffic is only the moved

@@ -15,8 +15,8 @@ namespace er {
 int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
                   cudaStream_t st);
 int launch_score(const float* w1, const float* w2, const uint16_t* x, int n, float* s,
-                 float* part, cudaStream_t st);
-size_t score_part_floats(int n);
+                 void* scratch, int32_t* err, cudaStream_t st);
+size_t score_scratch_bytes(int n);
 int launch_post_proj(const PostParams& P, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
                   cudaStream_t st);
@@ -32,7 +32,7 @@ namespace {
 struct LayerWs {
   uint16_t* proj;
   float* s;
-  float* score_part;
+  unsigned char* score_scratch;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
   float *part_o, *part_ml;
@@ -45,7 +45,7 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   LayerWs w;
   w.proj = c.take<uint16_t>((size_t)nq * QKV);
   w.s = c.take<float>((size_t)nq * NG);
-  w.score_part = c.take<float>(score_part_floats(nq));
+  w.score_scratch = c.take<unsigned char>(score_scratch_bytes(nq));
   w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
   w.chunk_k = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
@@ -89,7 +89,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   // a1: all six projections in one GEMM
   if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
   // a3: FP32 scores
-  if ((rc = launch_score(w->w1, w->w2, x, nq, W.s, W.score_part, s)) != ER_OK) return rc;
+  if ((rc = launch_score(w->w1, w->w2, x, nq, W.s, W.score_scratch, st->dev_error, s)) != ER_OK)
+    return rc;
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
   pp.proj = W.proj; pp.s = W.s; pp.nq = nq;
@@ -141,12 +142,12 @@ using namespace er;
 extern "C" {
 
 size_t er_decode_workspace_bytes(int32_t B) {
-  if (B < 0) return 0;
+  if (B < 1) return 0;
   return carve_ws(nullptr, B, false).bytes;
 }
 
 size_t er_prefill_workspace_bytes(int32_t T) {
-  if (T < 0 || T > PEND) return 0;
+  if (T < 1 || T > PEND) return 0;
   return carve_ws(nullptr, T, true).bytes;
 }
 
