@@ -42,9 +42,14 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-commit-bench", action="store_true")
-    ap.add_argument("--kernel", default="step", choices=["step", "attend", "commit"],
+    ap.add_argument("--no-prefill-bench", action="store_true")
+    ap.add_argument("--prefill-chunks", type=int, default=512,
+                    help="256-token chunks of the prefill stream (512 = 131072 tokens)")
+    ap.add_argument("--kernel", default="step",
+                    choices=["step", "attend", "commit", "prefill"],
                     help="step: the benchmark; attend/commit: one kernel alone at --batch "
-                         "sequences (profiling driver)")
+                         "sequences; prefill: --prefill-chunks chunks of one layer "
+                         "(profiling drivers)")
     ap.add_argument("--batch", type=int, default=256)
     return ap.parse_args()
 
@@ -249,8 +254,11 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_commit_bench and rank == 0:
         # the commit microbench reuses the decode state's memory (B=512 x 8 layers)
         cm = commit_microbench(st, dev)
+    pf = None
+    if not args.no_prefill_bench and rank == 0:
+        pf = prefill_bench(dev, args.prefill_chunks)
     return dict(ms=ms, launches=launches, clocks=clk, attend_ms=attend_ms, attend_n=attend_n,
-                fills=fills, commits=commits, e2e=e2e, commit_microbench=cm)
+                fills=fills, commits=commits, e2e=e2e, commit_microbench=cm, prefill=pf)
 
 
 # ------------------------------------------------------- commit microbench
@@ -312,6 +320,75 @@ def commit_microbench(st, dev, reps=3):
             "frac": alg / (ms / 1e3) / 1e9 / hbm, "peak_gbs": hbm, "peak_kind": kind}
 
 
+def prefill_attention_flops(t0: int, T: int, c: int, p0: int) -> int:
+    """Algorithmic FLOPs of one chunk's two reads (QKᵀ and PV, 2 FLOP per
+    multiply-add, 16 heads, head dim 256): query i at position t0+i reads
+    min(t0+i, 1023)+1 window keys and c + p0 + i + 1 anchors."""
+    keys = 0
+    for i in range(T):
+        keys += min(t0 + i, 1023) + 1 + c + p0 + i + 1
+    return keys * 16 * 256 * 2 * 2
+
+
+def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2):
+    """Chunked prefill of one stream from position 0 in 256-token chunks through
+    `layers` layers (every 4096th token scaled by 4), inputs resident before
+    timing.  Returns tokens/s over the whole stream and the attention share."""
+    import torch
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+    seed = wl.seed_of(4)
+    T = 256
+    weights = [sab.LayerWeights.from_dict(wl.make_weights(seed, l, device=dev))
+               for l in range(layers)]
+    st = sab.State(1, layers, device=dev)
+    ws = torch.empty(sab.prefill_workspace_bytes(T), dtype=torch.uint8, device=dev)
+    outs = [torch.empty(T, 2560, dtype=torch.bfloat16, device=dev) for _ in range(layers)]
+    xs = [[wl.make_x(seed, l, c, range(T), device=dev, big_every=4096, first_pos=c * T)
+           for l in range(layers)] for c in range(chunks)]
+    stream = torch.cuda.current_stream(dev)
+
+    def run(c0, c1):
+        for c in range(c0, c1):
+            for l in range(layers):
+                sab.swa_rma_prefill_chunk(st, weights[l], l, 0, xs[c][l], out=outs[l], ws=ws)
+            sab.advance(st, [0], T)
+
+    # warm-up on a scratch copy of the stream start, then restart from position 0
+    run(0, min(warm_chunks, chunks))
+    torch.cuda.synchronize(dev)
+    sab.state_init(st, [0])
+    torch.cuda.synchronize(dev)
+    sab.profile_read(reset=True)
+    sab.profile_enable(True)
+    n0 = sab.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(0, chunks)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    sab.profile_enable(False)
+    attn_ms, attn_n = sab.profile_read(reset=True)
+    launches = sab.launch_count() - n0
+    if sab.last_device_error(st) != 0:
+        raise RuntimeError("device error in the prefill bench")
+    ms = e0.elapsed_time(e1)
+    # attention FLOPs: bank and pending counts follow from the commit rule (every
+    # 256 tokens the block commits into a bank capped at 1024)
+    flops = 0
+    for c in range(chunks):
+        t0 = c * T
+        bank = min(1024, t0)
+        flops += prefill_attention_flops(t0, T, bank, 0)
+    flops *= layers
+    return {"workload": f"prefill_l{layers}_{chunks * T}tok_c256", "tokens": chunks * T,
+            "layers": layers, "ms": ms, "tok_per_s": chunks * T / (ms / 1e3),
+            "ms_per_chunk_layer": ms / (chunks * layers), "gpu_launches": launches,
+            "attention_ms": attn_ms, "attention_launches": attn_n,
+            "attention_tflops": flops / (attn_ms / 1e3) / 1e12 if attn_ms > 0 else None,
+            "attention_flops": flops}
+
+
 def single_kernel(args):
     """Profiling driver: one kernel alone on a --batch workload, three launches."""
     import torch
@@ -344,6 +421,9 @@ def single_kernel(args):
             raise RuntimeError("device error")
         out = {"kernel": "k_attend", "batch": B, "layers": 1, "ms": ms[-1], "alg_bytes": alg,
                "gbs": alg / (ms[-1] / 1e3) / 1e9}
+    elif args.kernel == "prefill":
+        out = {"kernel": "prefill", **prefill_bench(dev, args.prefill_chunks, layers=1,
+                                                    warm_chunks=1)}
     else:
         st = sab.State(B, LAYERS)
         r = commit_microbench(st, dev, reps=2)
@@ -481,6 +561,7 @@ def main():
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
         "commit_microbench": r["commit_microbench"],
+        "prefill": r["prefill"],
     }
     print(json.dumps(line), flush=True)
 

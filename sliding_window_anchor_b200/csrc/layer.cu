@@ -23,6 +23,11 @@ int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o
 int launch_commit(const CommitParams& P, cudaStream_t st);
 size_t attend_part_floats(int nq);
 size_t attend_ml_floats(int nq);
+size_t prefill_out_floats(int T);
+int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const uint16_t* q_swa,
+                          const uint16_t* q_rma, const uint16_t* chunk_k,
+                          const uint16_t* chunk_v, float* out, uint16_t* o_sum,
+                          cudaStream_t stream);
 
 }  // namespace er
 
@@ -35,7 +40,8 @@ struct LayerWs {
   unsigned char* score_scratch;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
-  float *part_o, *part_ml;
+  float *part_o, *part_ml;  // decode: split partials of the reads
+  float* pf_out;             // prefill: FP32 branch outputs [2][T][4096]
   uint16_t* o_sum;
   size_t bytes;
 };
@@ -50,8 +56,9 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
   w.chunk_k = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
   w.chunk_v = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
-  w.part_o = c.take<float>(attend_part_floats(nq));
-  w.part_ml = c.take<float>(attend_ml_floats(nq));
+  w.part_o = prefill ? nullptr : c.take<float>(attend_part_floats(nq));
+  w.part_ml = prefill ? nullptr : c.take<float>(attend_ml_floats(nq));
+  w.pf_out = prefill ? c.take<float>(prefill_out_floats(nq)) : nullptr;
   w.o_sum = c.take<uint16_t>((size_t)nq * OIN);
   w.bytes = c.used();
   return w;
@@ -103,16 +110,21 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   pp.layer = layer; pp.prefill = prefill ? 1 : 0; pp.seq_fixed = seq_fixed;
   pp.chunk_k = W.chunk_k; pp.chunk_v = W.chunk_v; pp.err = st->dev_error;
   if ((rc = launch_post_proj(pp, s)) != ER_OK) return rc;
-  // a5: both reads, merged into bf16(o_swa + o_rma)
-  AttendParams ap{};
-  ap.win_k = st->win_k; ap.win_v = st->win_v; ap.bank_k = st->bank_k; ap.bank_v = st->bank_v;
-  ap.pend_k = st->pend_k; ap.pend_v = st->pend_v; ap.meta = st->meta; ap.seq_ids = seq_ids;
-  ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
-  ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
-  ap.prefill = prefill ? 1 : 0; ap.seq_fixed = seq_fixed;
-  ap.chunk_k = W.chunk_k; ap.chunk_v = W.chunk_v;
-  ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.err = st->dev_error;
-  if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, s)) != ER_OK) return rc;
+  // a5 / a8: both reads, merged into bf16(o_swa + o_rma)
+  if (prefill) {
+    if ((rc = launch_prefill_attend(st, layer, seq_fixed, nq, W.q_swa, W.q_rma, W.chunk_k,
+                                    W.chunk_v, W.pf_out, W.o_sum, s)) != ER_OK)
+      return rc;
+  } else {
+    AttendParams ap{};
+    ap.win_k = st->win_k; ap.win_v = st->win_v; ap.bank_k = st->bank_k; ap.bank_v = st->bank_v;
+    ap.pend_k = st->pend_k; ap.pend_v = st->pend_v; ap.meta = st->meta; ap.seq_ids = seq_ids;
+    ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
+    ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
+    ap.prefill = 0; ap.seq_fixed = -1;
+    ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.err = st->dev_error;
+    if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, s)) != ER_OK) return rc;
+  }
   // a6: shared o_proj
   if ((rc = gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s)) != ER_OK) return rc;
   if (prefill) {

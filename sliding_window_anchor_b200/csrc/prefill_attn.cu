@@ -1,0 +1,440 @@
+// prefill_attn.cu — a8's two reads on the 5th-generation tensor cores.
+//
+// EdgeRock-4B 开源：72 MiB 固定 KV, §架构：递归、局部窗口与记忆锚点三件套 (16 query
+// heads over 4 KV groups, head dim 256, a 1024-position window beside the
+// anchor bank) with the reading fixed for this library: the RMA read is its
+// own softmax over committed + pending records, summed with the SWA read
+// before o_proj.  In a prefill chunk of T tokens starting at stream position
+// t0, query token i (position t = t0 + i) reads
+//   SWA: positions max(0, t-1023) .. t — older ones from the window ring (slot
+//        pos mod 1024, not yet overwritten by this chunk), the chunk's own
+//        rows j <= i;
+//   RMA: the c committed anchors and pending records 0 .. p0+i (the chunk's
+//        candidates were appended at p0 .. p0+T-1 before the reads).
+//
+// One CTA per (query tile, KV group, branch); a query tile is 32 tokens x the
+// group's 4 heads = 128 rows, the M of a tcgen05 MMA.  Keys stream in tiles of
+// 64 rows aligned to 64-slot boundaries of the ring, the chunk, the bank or the
+// pending block (so a TMA box never wraps); rows a query may not see are
+// masked in the softmax.
+//   warp 4    : TMA — Q once (four 64-dim slices, 4-D map picking the group's
+//               heads out of [T][16][256]), then K tiles (2 stages);
+//   warp 6    : TMA — V tiles (2 stages);
+//   warp 5    : TMEM owner (512 columns: O 0..255, two S buffers of 64) and
+//               MMA issuer: S_j = Q·K_jᵀ (M=128, N=64, K=256), then
+//               O += P_{j-1}·V_{j-1} (M=128, N=256, K=64, V read MN-major),
+//               so the tensor cores compute S_{j+1} while warps 0-3 work on
+//               the softmax of S_j;
+//   warps 0-3 : one thread per query row: S row from TMEM, mask, online
+//               softmax in base 2, P = exp2(s - m) rounded to BF16 into a
+//               swizzled shared-memory buffer (the A operand of the PV MMA).
+//               The running maximum is raised only when a tile's maximum
+//               exceeds it by more than 2^8; then the row of O is rescaled in
+//               TMEM (after the previous PV has completed).  At the end O / l
+//               goes out in FP32.
+// A second kernel adds the two branches and rounds to BF16 for o_proj.
+// Every wait is bounded (≈2 s) and records ER_ETIMEOUT instead of hanging.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace er {
+namespace {
+
+constexpr int PQ_TOK = 32;               // tokens per query tile
+constexpr int PM = 128;                  // query rows per tile (MMA M)
+constexpr int PKT = 64;                  // keys per key tile
+constexpr int SLICE = PM * 128;          // 128 rows x 64 BF16 (one Q slice, one P buffer)
+constexpr int KBOX = PKT * 128;          // one 64-row x 64-dim box, 8 KB
+constexpr int KTILE = 4 * KBOX;          // 64 keys x 256 dims, 32 KB
+constexpr int MAX_TILES = WIN / PKT + PEND / PKT;  // 20
+constexpr int PF_THREADS = 224;
+constexpr uint32_t TMEM_COLS = 512, TM_O = 0, TM_S = 256;
+constexpr float SCALE_LOG2 = 1.4426950408889634f / 16.0f;  // log2(e) / sqrt(256)
+constexpr float RESCALE_AT = 8.0f;
+
+enum : int { KIND_RING = 0, KIND_CHUNK = 1, KIND_BANK = 2, KIND_PEND = 3 };
+
+struct PTile {
+  int kind, row0, base, pad;
+};
+
+struct __align__(1024) PrefillSmem {
+  unsigned char q[4][SLICE];   // Q: 4 slices of 64 dims (64 KB)
+  unsigned char k[2][KTILE];   // K stages (64 KB)
+  unsigned char v[2][KTILE];   // V stages (64 KB)
+  unsigned char p[2][SLICE];   // P buffers (32 KB)
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2], v_full[2];
+  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int ntiles;
+  PTile tiles[MAX_TILES];
+};
+
+constexpr size_t PF_SMEM = sizeof(PrefillSmem) + 1024;
+static_assert(PF_SMEM <= 232448, "shared memory above the per-block limit");
+
+struct PrefillParams {
+  CUtensorMap tmap_q[2];  // q_swa, q_rma: {256, 4 heads, 4 groups, T}, box {64, 4, 1, 32}
+  CUtensorMap tmap_k[4];  // ring, chunk, bank, pending K rows; box 64 x 64
+  CUtensorMap tmap_v[4];
+  const int32_t* meta;
+  int seq, s_max, L, layer, T;
+  float* out;  // FP32 [2][T][16][256]: branch outputs
+  int32_t* err;
+};
+
+__device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
+
+// The key tiles one work item reads, in the order they are streamed.
+__device__ int build_tiles(PTile* tl, int br, int g, int i0, int T, int t0, int p0, int c,
+                           int gi) {
+  const int i_last = min(T, i0 + PQ_TOK) - 1;
+  int n = 0;
+  if (br == 0) {
+    // ring tiles holding at least one position the tile's first query still sees
+    const int lo_min = max(0, t0 + i0 - (WIN - 1));
+    for (int rt = 0; rt < WIN / PKT && t0 > 0; ++rt) {
+      int newest = INT_MIN;
+      for (int k = 0; k < PKT; ++k)
+        newest = max(newest, t0 - WIN + ((rt * PKT + k - t0) & (WIN - 1)));
+      if (newest >= lo_min) tl[n++] = {KIND_RING, gi * WIN + rt * PKT, rt * PKT, 0};
+    }
+    for (int ct = 0; ct * PKT <= i_last; ++ct)
+      tl[n++] = {KIND_CHUNK, g * T + ct * PKT, ct * PKT, 0};
+  } else {
+    for (int bt = 0; bt * PKT < c; ++bt) tl[n++] = {KIND_BANK, gi * BANK + bt * PKT, bt * PKT, 0};
+    for (int pt = 0; pt * PKT <= p0 + i_last; ++pt)
+      tl[n++] = {KIND_PEND, gi * PEND + pt * PKT, pt * PKT, 0};
+  }
+  return n;
+}
+
+__global__ void __launch_bounds__(PF_THREADS, 1)
+    k_prefill_attn(const __grid_constant__ PrefillParams P) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i0 = blockIdx.x * PQ_TOK, g = blockIdx.y, br = blockIdx.z;
+  const int T = P.T;
+  const int t0 = P.meta[P.seq * 4 + 0];
+  const int p0 = P.meta[P.seq * 4 + 1];
+  const int c = P.meta[P.seq * 4 + 2];
+  const int gi = (int)grp(P.seq, P.layer, g, P.L);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&S.q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.k_full[b], 1);
+      mbar_init(&S.k_empty[b], 1);
+      mbar_init(&S.v_full[b], 1);
+      mbar_init(&S.s_full[b], 1);
+      mbar_init(&S.s_empty[b], 128);
+      mbar_init(&S.p_full[b], 128);
+      mbar_init(&S.pv_done[b], 1);
+    }
+    mbar_init(&S.mma_done, 1);
+    fence_mbar_init();
+    const bool meta_ok = t0 >= 0 && p0 >= 0 && c >= 0 && c <= BANK && p0 + T <= PEND;
+    S.ntiles = meta_ok ? build_tiles(S.tiles, br, g, i0, T, t0, p0, c, gi) : 0;
+    if (!meta_ok) set_dev_error(P.err, ER_ECAPACITY);
+  }
+  if (warp == 5) tc::tmem_alloc(&S.tmem_base, TMEM_COLS);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = S.tmem_base;
+  const int n = S.ntiles;
+
+  if (warp == 4) {
+    // ------------------------------------------------------ Q + K producer
+    if (lane == 0 && n > 0) {
+      mbar_arrive_expect_tx(&S.q_full, 4 * SLICE);
+      for (int d = 0; d < 4; ++d)
+        tc::tma_load_4d(S.q[d], &P.tmap_q[br], 64 * d, 0, g, i0, &S.q_full);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int b = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&S.k_empty[b], ph ^ 1, P.err)) break;
+        const PTile tl = S.tiles[j];
+        mbar_arrive_expect_tx(&S.k_full[b], KTILE);
+        for (int d = 0; d < 4; ++d)
+          tc::tma_load_2d(S.k[b] + d * KBOX, &P.tmap_k[tl.kind], 64 * d, tl.row0, &S.k_full[b]);
+        ++issued;
+      }
+      // no copy may still be landing when the block exits
+      mbar_wait(&S.q_full, 0, P.err);
+      for (int j = max(0, issued - 2); j < issued; ++j)
+        mbar_wait(&S.k_full[j & 1], (j >> 1) & 1, P.err);
+    }
+  } else if (warp == 6) {
+    // ---------------------------------------------------------- V producer
+    if (lane == 0 && n > 0) {
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int b = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (!mbar_wait(&S.pv_done[b], ph ^ 1, P.err)) break;
+        const PTile tl = S.tiles[j];
+        mbar_arrive_expect_tx(&S.v_full[b], KTILE);
+        for (int d = 0; d < 4; ++d)
+          tc::tma_load_2d(S.v[b] + d * KBOX, &P.tmap_v[tl.kind], 64 * d, tl.row0, &S.v_full[b]);
+        ++issued;
+      }
+      for (int j = max(0, issued - 2); j < issued; ++j)
+        mbar_wait(&S.v_full[j & 1], (j >> 1) & 1, P.err);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0 && n > 0) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16(PM, PKT, false, false);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16(PM, 256, false, true);
+      bool ok = mbar_wait(&S.q_full, 0, P.err);
+      for (int j = 0; ok && j <= n; ++j) {
+        if (j < n) {
+          const int b = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          ok = mbar_wait(&S.k_full[b], ph, P.err) && mbar_wait(&S.s_empty[b], ph ^ 1, P.err);
+          if (!ok) break;
+          tc::fence_after_sync();
+          const uint32_t d_s = tmem + TM_S + PKT * b;
+#pragma unroll
+          for (int kk = 0; kk < 16; ++kk) {
+            const uint64_t a =
+                tc::desc_sw128(smem_u32(S.q[kk >> 2]) + 32 * (kk & 3), 16, 1024);
+            const uint64_t bd =
+                tc::desc_sw128(smem_u32(S.k[b]) + (kk >> 2) * KBOX + 32 * (kk & 3), 16, 1024);
+            tc::mma_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
+          }
+          tc::commit(&S.s_full[b]);
+          tc::commit(&S.k_empty[b]);
+        }
+        if (j >= 1) {
+          const int jj = j - 1, b = jj & 1;
+          const uint32_t ph = (jj >> 1) & 1;
+          ok = mbar_wait(&S.v_full[b], ph, P.err) && mbar_wait(&S.p_full[b], ph, P.err);
+          if (!ok) break;
+          tc::fence_after_sync();
+#pragma unroll
+          for (int kk = 0; kk < PKT / 16; ++kk) {
+            const uint64_t a = tc::desc_sw128(smem_u32(S.p[b]) + 32 * kk, 16, 1024);
+            // V tile as the MN-major B operand: 64-dim blocks KBOX apart, 8-key groups 1 KB apart
+            const uint64_t bd = tc::desc_sw128(smem_u32(S.v[b]) + 2048 * kk, KBOX, 1024);
+            tc::mma_bf16_ss(tmem + TM_O, a, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::commit(&S.pv_done[b]);
+        }
+      }
+      // nothing of this block's may still run on the tensor cores at exit
+      tc::commit(&S.mma_done);
+      mbar_wait(&S.mma_done, 0, P.err);
+    }
+  } else {
+    // ------------------------------------------------------ softmax, rows
+    const int r = threadIdx.x;  // 0..127 = TMEM lane
+    const int i = i0 + (r >> 2), hh = r & 3;
+    const int t = t0 + i;
+    const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = n > 0;
+    for (int j = 0; ok && j < n; ++j) {
+      const int b = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      ok = warp_all(mbar_wait(&S.s_full[b], ph, P.err));
+      if (!ok) break;
+      tc::fence_after_sync();
+      float s[PKT];
+      {
+        uint32_t raw[32];
+        tc::tmem_ld32(tmem + lane_addr + TM_S + PKT * b, raw);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(raw[k]);
+        tc::tmem_ld32(tmem + lane_addr + TM_S + PKT * b + 32, raw);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(raw[k]);
+      }
+      tc::fence_before_sync();
+      mbar_arrive(&S.s_empty[b]);
+
+      // which keys of this tile the row may see
+      const PTile tl = S.tiles[j];
+      int lo = 0, hi = -1;
+      if (tl.kind == KIND_RING) {
+        lo = max(0, t - (WIN - 1));
+        hi = t;
+      } else if (tl.kind == KIND_CHUNK) {
+        hi = i;
+      } else if (tl.kind == KIND_BANK) {
+        hi = c - 1;
+      } else {
+        hi = p0 + i;
+      }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < PKT; ++k) {
+        const int v = tl.kind == KIND_RING ? t0 - WIN + ((tl.base + k - t0) & (WIN - 1))
+                                           : tl.base + k;
+        s[k] = (v >= lo && v <= hi) ? s[k] * SCALE_LOG2 : -INFINITY;
+        mt = fmaxf(mt, s[k]);
+      }
+      const float m_new = fmaxf(m, mt);
+      const bool need = (m != -INFINITY) && (m_new > m + RESCALE_AT);
+      if (__any_sync(0xffffffffu, need)) {
+        // O holds P_0..P_{j-1}·V: wait for the last of those products, then rescale
+        ok = warp_all(mbar_wait(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, P.err));
+        if (!ok) break;
+        tc::fence_after_sync();
+        const float f = need ? exp2f(m - m_new) : 1.f;
+#pragma unroll 1
+        for (int cb = 0; cb < 8; ++cb) {
+          uint32_t o[32];
+          tc::tmem_ld32(tmem + lane_addr + TM_O + 32 * cb, o);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+          tc::tmem_st32(tmem + lane_addr + TM_O + 32 * cb, o);
+        }
+        tc::tmem_wait_st();
+        if (need) l *= f;
+      }
+      if (need || m == -INFINITY) m = m_new;
+      const float msub = m == -INFINITY ? 0.f : m;
+      uint32_t pk[PKT / 2];
+      float lsum = 0.f;
+#pragma unroll
+      for (int k = 0; k < PKT; k += 2) {
+        const __nv_bfloat162 h2 =
+            __floats2bfloat162_rn(exp2f(s[k] - msub), exp2f(s[k + 1] - msub));
+        const float2 back = __bfloat1622float2(h2);
+        lsum += back.x + back.y;
+        pk[k >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      l += lsum;
+      // the P buffer is free once PV_{j-2} has completed
+      if (j >= 2) {
+        ok = warp_all(mbar_wait(&S.pv_done[b], ((j - 2) >> 1) & 1, P.err));
+        if (!ok) break;
+      }
+      unsigned char* prow = S.p[b] + r * 128;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      mbar_arrive(&S.p_full[b]);
+    }
+    if (ok) ok = warp_all(mbar_wait(&S.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, P.err));
+    if (ok) {
+      tc::fence_after_sync();
+      const float inv = 1.f / l;
+      float* dst = P.out + ((size_t)(br * T + i) * NH + 4 * g + hh) * D;
+#pragma unroll 1
+      for (int cb = 0; cb < 8; ++cb) {
+        uint32_t o[32];
+        tc::tmem_ld32(tmem + lane_addr + TM_O + 32 * cb, o);
+        tc::tmem_wait_ld();
+        if (i < T) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * cb + e) =
+                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// o_sum[t][h*256 + d] = bf16(o_swa + o_rma), 8 values per thread.
+__global__ void k_prefill_combine(const float* __restrict__ out, int T,
+                                  uint16_t* __restrict__ o_sum) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * (OIN / 8)) return;
+  const size_t e = (size_t)idx * 8;
+  const float4* a = reinterpret_cast<const float4*>(out + e);
+  const float4* b = reinterpret_cast<const float4*>(out + (size_t)T * OIN + e);
+  const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
+  const __nv_bfloat162 h0 = __floats2bfloat162_rn(a0.x + b0.x, a0.y + b0.y);
+  const __nv_bfloat162 h1 = __floats2bfloat162_rn(a0.z + b0.z, a0.w + b0.w);
+  const __nv_bfloat162 h2 = __floats2bfloat162_rn(a1.x + b1.x, a1.y + b1.y);
+  const __nv_bfloat162 h3 = __floats2bfloat162_rn(a1.z + b1.z, a1.w + b1.w);
+  uint4 v;
+  v.x = *reinterpret_cast<const uint32_t*>(&h0);
+  v.y = *reinterpret_cast<const uint32_t*>(&h1);
+  v.z = *reinterpret_cast<const uint32_t*>(&h2);
+  v.w = *reinterpret_cast<const uint32_t*>(&h3);
+  *reinterpret_cast<uint4*>(o_sum + e) = v;
+}
+
+bool g_pf_attr[64] = {false};
+std::mutex g_pf_mu;
+
+}  // namespace
+
+// Workspace FP32 floats for the branch outputs of a T-token chunk.
+size_t prefill_out_floats(int T) { return (size_t)2 * T * OIN; }
+
+int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const uint16_t* q_swa,
+                          const uint16_t* q_rma, const uint16_t* chunk_k,
+                          const uint16_t* chunk_v, float* out, uint16_t* o_sum,
+                          cudaStream_t stream) {
+  if (T < 1 || T > PEND) return ER_EINVAL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ER_ECUDA;
+  {
+    std::lock_guard<std::mutex> lock(g_pf_mu);
+    if (!g_pf_attr[dev]) {
+      if (cudaFuncSetAttribute(k_prefill_attn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)PF_SMEM) != cudaSuccess)
+        return ER_ECUDA;
+      g_pf_attr[dev] = true;
+    }
+  }
+  PrefillParams P;
+  const uint64_t rows_win = (uint64_t)st->s_max * st->n_layers * NG * WIN;
+  const uint64_t rows_pend = (uint64_t)st->s_max * st->n_layers * NG * PEND;
+  const uint64_t qd[4] = {D, 4, NG, (uint64_t)T};
+  const uint64_t qs[3] = {D * 2, 4 * D * 2, NH * D * 2};
+  const uint32_t qb[4] = {64, 4, 1, PQ_TOK};
+  bool ok = encode_bf16(&P.tmap_q[0], q_swa, 4, qd, qs, qb) &&
+            encode_bf16(&P.tmap_q[1], q_rma, 4, qd, qs, qb);
+  const uint16_t* kb[4] = {st->win_k, chunk_k, st->bank_k, st->pend_k};
+  const uint16_t* vb[4] = {st->win_v, chunk_v, st->bank_v, st->pend_v};
+  const uint64_t rows[4] = {rows_win, (uint64_t)NG * T, rows_win, rows_pend};
+  for (int m = 0; m < 4; ++m)
+    ok = ok && encode_bf16_2d(&P.tmap_k[m], kb[m], D, rows[m], ROW_BYTES, 64, 64) &&
+         encode_bf16_2d(&P.tmap_v[m], vb[m], D, rows[m], ROW_BYTES, 64, 64);
+  if (!ok) return ER_ECUDA;
+  P.meta = st->meta;
+  P.seq = seq;
+  P.s_max = st->s_max;
+  P.L = st->n_layers;
+  P.layer = layer;
+  P.T = T;
+  P.out = out;
+  P.err = st->dev_error;
+  const dim3 grid((T + PQ_TOK - 1) / PQ_TOK, NG, 2);
+  k_prefill_attn<<<grid, PF_THREADS, PF_SMEM, stream>>>(P);
+  const int nv = T * (OIN / 8);
+  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, T, o_sum);
+  count_launches(2);
+  return launch_status();
+}
+
+}  // namespace er

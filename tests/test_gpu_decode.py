@@ -130,22 +130,44 @@ def test_decode_batched_sampled_sequences(sab, cfg_index):
         _kept_sets_agree(grow, orow, L)
 
 
-def test_prefill_chunks_match_oracle_and_decode(sab):
-    """Seeded state at 4096 (the ring wraps for every query), one layer: a full chunk of
-    256 (fills the block, commits) then a ragged chunk of 37."""
+PREFILL_CASES = {
+    # seeded at 4096: the ring wraps for every query; a full chunk (commits) then a ragged one
+    "wrap_t4096": dict(t0=4096, pend=0, bank=None, chunks=(256, 37)),
+    # the last chunk of the 131072-token stream (its last token is one of the x4 ones)
+    "last_chunk_t130816": dict(t0=130816, pend=0, bank=None, chunks=(256,)),
+    # a partly filled bank, 100 records already pending, an unaligned stream position
+    "partial_bank_t5000": dict(t0=5000, pend=100, bank=700, chunks=(156, 40)),
+    # the stream start: empty state, the ring partly written, the bank growing
+    "stream_start": dict(t0=None, pend=0, bank=None, chunks=(256, 256, 77, 50)),
+}
+
+
+@pytest.mark.parametrize("case", list(PREFILL_CASES))
+def test_prefill_chunks_match_oracle_and_decode(sab, case):
+    """One layer: each chunk through er_swa_rma_prefill_chunk against the oracle's
+    prefill and against the same tokens replayed one by one through the decode path
+    (state row 1); states and kept anchor sets must agree afterwards."""
+    cfg = PREFILL_CASES[case]
     seed = wl.seed_of(4)
     L = 1
     ow, wdict = H.oracle_weights(seed, 0)
     gw, gdict = H.gpu_weights(seed, 0)
     ost = oracle.OracleState(1, L)
-    H.seed_oracle_state(ost, [0], L, 4096, "zero", seed, [wdict])
     st = sab.State(2, L)
-    H.seed_gpu_state(st, L, 4096, [0, 0], seed, [gdict])
-    # row 1 replays the same stream token by token through the decode path
+    if cfg["t0"] is None:
+        sab.state_init(st, [0, 1])
+        pos = 0
+    else:
+        H.seed_oracle_state(ost, [0], L, cfg["t0"], [cfg["pend"]], seed, [wdict])
+        H.seed_gpu_state(st, L, cfg["t0"], [cfg["pend"]] * 2, seed, [gdict])
+        if cfg["bank"] is not None:
+            ost.meta[0, 2] = cfg["bank"]
+            st.meta[:, 2] = cfg["bank"]
+        pos = cfg["t0"]
     for n in oracle.OracleState.ARRAYS:
         getattr(st, n)[1].copy_(getattr(st, n)[0])
-    for ci, T in enumerate((256, 37)):
-        x = wl.make_x(seed, 0, 1000 + ci, range(T), big_every=4096, first_pos=4096)
+    for ci, T in enumerate(cfg["chunks"]):
+        x = wl.make_x(seed, 0, 1000 + ci, range(T), big_every=4096, first_pos=pos)
         got = sab.swa_rma_prefill_chunk(st, gw, 0, 0, x.cuda())
         sab.advance(st, [0], T)
         dec = []
@@ -155,8 +177,9 @@ def test_prefill_chunks_match_oracle_and_decode(sab):
         dec = torch.cat(dec).cpu()
         ref = ost.prefill_chunk(ow, 0, 0, x)
         ost.advance(0, T)
-        assert H.tol_ok(got.cpu(), ref), (ci, H.max_err(got.cpu(), ref))
-        assert H.tol_ok(got.cpu(), dec), (ci, H.max_err(got.cpu(), dec))
+        assert H.tol_ok(got.cpu(), ref), (case, ci, H.max_err(got.cpu(), ref))
+        assert H.tol_ok(got.cpu(), dec), (case, ci, H.max_err(got.cpu(), dec))
+        pos += T
     assert sab.last_device_error(st) == 0
     g0, g1 = H.download_row(st, 0), H.download_row(st, 1)
     orow = {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
