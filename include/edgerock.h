@@ -107,13 +107,18 @@ typedef struct er_state {
  *   w_o   BF16 [2560][4096]  shared o_proj
  *   q_norm_swa, k_norm_swa, q_norm_rma, k_norm_rma: BF16 [256] RMS-norm gains
  *                             (one per head dim, shared by all heads of the branch)
- *   w1    FP32 [256][2560], w2 FP32 [4][256]: the scorer, bias-free. */
+ *   w1    FP32 [256][2560], w2 FP32 [4][256]: the scorer, bias-free.
+ *   w1_split (optional, may be NULL): BF16 [3][256][2560], w1 written as three
+ *                             BF16 terms by er_score_split_w1 (prepared once per
+ *                             weight set); NULL makes every scorer call split
+ *                             w1 again into its workspace. */
 typedef struct er_layer_weights {
   const er_bf16* w_qkv;
   const er_bf16* w_o;
   const er_bf16 *q_norm_swa, *k_norm_swa, *q_norm_rma, *k_norm_rma;
   const float* w1;
   const float* w2;
+  const er_bf16* w1_split;
 } er_layer_weights;
 
 /* ---------------------------------------------------------------- state */
@@ -152,12 +157,21 @@ int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream);
 int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, const er_bf16* gain,
                     const int32_t* pos, er_stream_t stream);
 
-/* a3 — retention scores [F-arch], [N-rma]: s = W2 · SiLU(W1 · x), FP32
- * products and sums (split over K, summed in a fixed order: deterministic).
+/* a3 — retention scores [F-arch], [N-rma]: s = W2 · SiLU(W1 · x) with FP32
+ * accuracy: W1 is taken as three BF16 terms hi + mid + lo (residual below
+ * 2^-24 |W1|), each product with the BF16 x is exact and accumulates in FP32;
+ * partial sums are added in a fixed order (deterministic).
  * x: BF16 [n][2560]; s: FP32 [n][4] (one per KV group); n may be 0.
- * ws: scratch of er_score_workspace_bytes(n) bytes (the K-split partial sums;
- * contents on return are unspecified). */
+ * ws: scratch of er_score_workspace_bytes(n) bytes (room for the W1 terms when
+ * w->w1_split is NULL, and the partial scores; contents on return are
+ * unspecified). */
 size_t er_score_workspace_bytes(int32_t n);
+
+/* Writes w1 (FP32 [256][2560]) as three BF16 terms hi, mid, lo into terms
+ * (BF16 [3][256][2560], caller-owned device memory, 16-byte aligned): hi =
+ * bf16(w1), mid = bf16(w1 - hi), lo = bf16(w1 - hi - mid).  The result is the
+ * optional er_layer_weights.w1_split. */
+int er_score_split_w1(const float* w1, er_bf16* terms, er_stream_t stream);
 int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
                  size_t ws_bytes, er_stream_t stream);
 
@@ -167,10 +181,10 @@ int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* 
  * a host program whose device memory is all owned by another framework's
  * caching allocator, or a plugin interface that only receives tensor pointers
  * and may not call cudaMalloc itself.  Same result as er_rma_score.
- *  - Its scratch (W1 split into three BF16 terms, 3.75 MiB, plus 8 partial
- *    scores per token and group, 32 KiB at 256 tokens) lives in one fixed
- *    4 MiB device array inside the library, which every GPU that loads the
- *    library holds until the process exits.
+ *  - Its scratch (W1 split into three BF16 terms, 3.75 MiB, when w->w1_split
+ *    is NULL, plus 4 partial scores per token and group, 16 KiB at 256
+ *    tokens) lives in one fixed 4 MiB device array inside the library, which
+ *    every GPU that loads the library holds until the process exits.
  *  - n above ER_SCORE_NOALLOC_MAX_TOKENS returns ER_ECAPACITY; nothing runs.
  *  - The first call on a device (with that device current) looks the array's
  *    device address up with cudaGetSymbolAddress and caches it; make that
@@ -256,8 +270,8 @@ const char* er_error_string(int code);
 /* Number of kernels this library has launched since load (all threads). */
 uint64_t er_launch_count(void);
 
-/* When enabled, the a5 read kernel launches are bracketed by CUDA events on
- * their own stream; er_profile_read returns the summed milliseconds and the
+/* When enabled, launches of the read kernels (the a5 decode read and the a8
+ * prefill read) are bracketed by CUDA events on their own stream; er_profile_read returns the summed milliseconds and the
  * number of timed launches since the last reset (it synchronises the events).
  * Host-side bookkeeping only; not thread-safe. */
 int er_profile_enable(int enable);

@@ -72,9 +72,14 @@ class State:
 
 
 class LayerWeights:
-    """One layer's device weights (BF16 projections and gains, FP32 scorer)."""
+    """One layer's device weights (BF16 projections and gains, FP32 scorer).
 
-    def __init__(self, w_qkv, w_o, q_norm_swa, k_norm_swa, q_norm_rma, k_norm_rma, w1, w2):
+    With prepare=True (the default) W1's three BF16 terms are made once here
+    (er_score_split_w1) and every scorer call reuses them; prepare=False leaves
+    w1_split NULL, so each call splits W1 again in its workspace."""
+
+    def __init__(self, w_qkv, w_o, q_norm_swa, k_norm_swa, q_norm_rma, k_norm_rma, w1, w2,
+                 prepare: bool = True):
         bf, f32 = torch.bfloat16, torch.float32
         self.t = dict(w_qkv=w_qkv, w_o=w_o, q_norm_swa=q_norm_swa, k_norm_swa=k_norm_swa,
                       q_norm_rma=q_norm_rma, k_norm_rma=k_norm_rma, w1=w1, w2=w2)
@@ -86,14 +91,21 @@ class LayerWeights:
             if tuple(t.shape) != shape or t.dtype != dt:
                 raise ValueError(f"{k}: expected {shape} {dt}, got {tuple(t.shape)} {t.dtype}")
             dev_ptr(t, dt, k)
+        self.w1_split = None
+        if prepare:
+            self.w1_split = torch.empty(3, 256, HIDDEN, dtype=bf, device=w1.device)
+            check("er_score_split_w1", lib().er_score_split_w1(
+                dev_ptr(w1, f32, "w1"), dev_ptr(self.w1_split, bf, "w1_split"),
+                stream_handle(None, w1.device)))
         self.c = _lib.CWeights(*[self.t[k].data_ptr() for k in
                                  ("w_qkv", "w_o", "q_norm_swa", "k_norm_swa", "q_norm_rma",
-                                  "k_norm_rma", "w1", "w2")])
+                                  "k_norm_rma", "w1", "w2")],
+                               self.w1_split.data_ptr() if self.w1_split is not None else None)
 
     @classmethod
-    def from_dict(cls, d):
+    def from_dict(cls, d, prepare: bool = True):
         return cls(d["w_qkv"], d["w_o"], d["q_norm_swa"], d["k_norm_swa"], d["q_norm_rma"],
-                   d["k_norm_rma"], d["w1"], d["w2"])
+                   d["k_norm_rma"], d["w1"], d["w2"], prepare=prepare)
 
     def ptr(self):
         return ctypes.byref(self.c)

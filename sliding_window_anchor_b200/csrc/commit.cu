@@ -19,7 +19,7 @@
 //  3. flags for the kept records; two block scans give the evicted bank slots
 //     (ascending) and the pending winners (ascending);
 //  4. each warp moves winners' K and V rows (512 B each, 16 B per lane) into
-//     their target slots, with the score and position.
+//     their target slots, with the score and position, four rows in flight.
 // Surviving anchors are not touched, so the write traffic is only the moved
 // records.
 #include "common.cuh"
@@ -333,33 +333,32 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
     }
     __syncthreads();
 
-    // move rows: one warp per winner, 16 bytes per lane per row, two winners in flight
+    // move rows: one warp per winner, 16 bytes per lane per row; MV winners per warp
+    // in flight (every load issued before the first store)
+    constexpr int MV = 4;
     const int warp = tid >> 5, lane = tid & 31;
-    for (int w = warp; w < total_win; w += 2 * CW) {
-      const int w2 = w + CW;
-      const int j = move_src[w], d = move_dst[w];
-      const uint4 a = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + j) * D)[lane];
-      const uint4 a2 = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + j) * D)[lane];
-      uint4 bq = make_uint4(0, 0, 0, 0), bq2 = bq;
-      int j2 = 0, d2 = 0;
-      if (w2 < total_win) {
-        j2 = move_src[w2];
-        d2 = move_dst[w2];
-        bq = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + j2) * D)[lane];
-        bq2 = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + j2) * D)[lane];
+    for (int w0 = warp; w0 < total_win; w0 += MV * CW) {
+      uint4 kr[MV], vr[MV];
+      int src[MV];
+#pragma unroll
+      for (int q = 0; q < MV; ++q) {
+        const int w = w0 + q * CW;
+        src[q] = w < total_win ? (int)move_src[w] : -1;
+        kr[q] = vr[q] = make_uint4(0, 0, 0, 0);
+        if (src[q] >= 0) {
+          kr[q] = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + src[q]) * D)[lane];
+          vr[q] = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + src[q]) * D)[lane];
+        }
       }
-      reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + d) * D)[lane] = a;
-      reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + d) * D)[lane] = a2;
-      if (lane == 0) {
-        P.bank_score[gi * BANK + d] = P.pend_score[gi * PEND + j];
-        P.bank_pos[gi * BANK + d] = P.pend_pos[gi * PEND + j];
-      }
-      if (w2 < total_win) {
-        reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + d2) * D)[lane] = bq;
-        reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + d2) * D)[lane] = bq2;
+#pragma unroll
+      for (int q = 0; q < MV; ++q) {
+        if (src[q] < 0) continue;
+        const int dst = move_dst[w0 + q * CW];
+        reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + dst) * D)[lane] = kr[q];
+        reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + dst) * D)[lane] = vr[q];
         if (lane == 0) {
-          P.bank_score[gi * BANK + d2] = P.pend_score[gi * PEND + j2];
-          P.bank_pos[gi * BANK + d2] = P.pend_pos[gi * PEND + j2];
+          P.bank_score[gi * BANK + dst] = P.pend_score[gi * PEND + src[q]];
+          P.bank_pos[gi * BANK + dst] = P.pend_pos[gi * PEND + src[q]];
         }
       }
     }

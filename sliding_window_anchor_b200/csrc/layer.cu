@@ -14,8 +14,8 @@ namespace er {
 
 int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
                   cudaStream_t st);
-int launch_score(const float* w1, const float* w2, const uint16_t* x, int n, float* s,
-                 void* scratch, int32_t* err, cudaStream_t st);
+int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
+                 int n, float* s, void* scratch, int32_t* err, cudaStream_t st);
 size_t score_scratch_bytes(int n);
 int launch_post_proj(const PostParams& P, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
@@ -68,7 +68,8 @@ bool weights_ok(const er_layer_weights* w) {
   return w && w->w_qkv && w->w_o && w->q_norm_swa && w->k_norm_swa && w->q_norm_rma &&
          w->k_norm_rma && w->w1 && w->w2 && aligned16(w->w_qkv) && aligned16(w->w_o) &&
          aligned16(w->q_norm_swa) && aligned16(w->k_norm_swa) && aligned16(w->q_norm_rma) &&
-         aligned16(w->k_norm_rma) && aligned16(w->w1) && aligned16(w->w2);
+         aligned16(w->k_norm_rma) && aligned16(w->w1) && aligned16(w->w2) &&
+         (!w->w1_split || aligned16(w->w1_split));
 }
 
 // The chunk's window rows enter the ring after all of its reads.
@@ -96,7 +97,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   // a1: all six projections in one GEMM
   if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
   // a3: FP32 scores
-  if ((rc = launch_score(w->w1, w->w2, x, nq, W.s, W.score_scratch, st->dev_error, s)) != ER_OK)
+  if ((rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, W.s, W.score_scratch, st->dev_error,
+                        s)) != ER_OK)
     return rc;
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};

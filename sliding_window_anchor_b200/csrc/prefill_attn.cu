@@ -12,36 +12,45 @@
 //   RMA: the c committed anchors and pending records 0 .. p0+i (the chunk's
 //        candidates were appended at p0 .. p0+T-1 before the reads).
 //
-// One CTA per (query tile, KV group, branch); a query tile is 32 tokens x the
+// One CTA per (query tile, KV group, branch, split); a query tile is 32 tokens x the
 // group's 4 heads = 128 rows, the M of a tcgen05 MMA.  Keys stream in tiles of
 // 64 rows aligned to 64-slot boundaries of the ring, the chunk, the bank or the
 // pending block (so a TMA box never wraps); rows a query may not see are
 // masked in the softmax.
 //   warp 4    : TMA — Q once (four 64-dim slices, 4-D map picking the group's
-//               heads out of [T][16][256]), then K tiles (2 stages);
+//               heads out of [T][16][256]), then K tiles (3 stages);
 //   warp 6    : TMA — V tiles (2 stages);
-//   warp 5    : TMEM owner (512 columns: O 0..255, two S buffers of 64) and
+//   warp 5    : TMEM owner (512 columns: O 0..255, two S buffers of 64 FP32
+//               columns, two P buffers of 32 columns of BF16 pairs) and
 //               MMA issuer: S_j = Q·K_jᵀ (M=128, N=64, K=256), then
-//               O += P_{j-1}·V_{j-1} (M=128, N=256, K=64, V read MN-major),
+//               O += P_{j-1}·V_{j-1} (M=128, N=256, K=64, P read from TMEM,
+//               V read MN-major),
 //               so the tensor cores compute S_{j+1} while warps 0-3 work on
 //               the softmax of S_j;
 //   warps 0-3 : one thread per query row: S row from TMEM, mask, online
-//               softmax in base 2, P = exp2(s - m) rounded to BF16 into a
-//               swizzled shared-memory buffer (the A operand of the PV MMA).
+//               softmax in base 2, P = exp2(s - m) rounded to BF16 and
+//               stored back to TMEM (the A operand of the PV MMA).
 //               The running maximum is raised only when a tile's maximum
 //               exceeds it by more than 2^8; then the row of O is rescaled in
 //               TMEM (after the previous PV has completed).  At the end O / l
-//               goes out in FP32.
-// A second kernel adds the two branches and rounds to BF16 for o_proj.
+//               and (m, l) go out in FP32.
+// An item's key tiles are split over NSPLIT CTAs (so a 256-token chunk fills
+// 128 SMs); a second kernel merges the splits of each branch by their (m, l),
+// adds the two branches and rounds to BF16 for o_proj.
 // Every wait is bounded (≈2 s) and records ER_ETIMEOUT instead of hanging.
 #include <math.h>
 
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "tc.cuh"
 
 namespace er {
+
+bool profile_begin(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t>* ev);
+void profile_end(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t> ev);
+
 namespace {
 
 constexpr int PQ_TOK = 32;               // tokens per query tile
@@ -52,27 +61,29 @@ constexpr int KBOX = PKT * 128;          // one 64-row x 64-dim box, 8 KB
 constexpr int KTILE = 4 * KBOX;          // 64 keys x 256 dims, 32 KB
 constexpr int MAX_TILES = WIN / PKT + PEND / PKT;  // 20
 constexpr int PF_THREADS = 224;
-constexpr uint32_t TMEM_COLS = 512, TM_O = 0, TM_S = 256;
+constexpr int KST = 3;                   // K stages
+constexpr uint32_t TMEM_COLS = 512, TM_O = 0, TM_S = 256, TM_P = 384;
 constexpr float SCALE_LOG2 = 1.4426950408889634f / 16.0f;  // log2(e) / sqrt(256)
 constexpr float RESCALE_AT = 8.0f;
+constexpr int NSPLIT = 2;                // key tiles of an item split over this many CTAs
 
 enum : int { KIND_RING = 0, KIND_CHUNK = 1, KIND_BANK = 2, KIND_PEND = 3 };
 
 struct PTile {
-  int kind, row0, base, pad;
+  int kind, row0, base;
+  int full;  // every key of the tile is visible to every query row of the item
 };
 
 struct __align__(1024) PrefillSmem {
   unsigned char q[4][SLICE];   // Q: 4 slices of 64 dims (64 KB)
-  unsigned char k[2][KTILE];   // K stages (64 KB)
-  unsigned char v[2][KTILE];   // V stages (64 KB)
-  unsigned char p[2][SLICE];   // P buffers (32 KB)
+  unsigned char k[KST][KTILE];  // K stages (96 KB)
+  unsigned char v[2][KTILE];    // V stages (64 KB)
   uint64_t q_full;
-  uint64_t k_full[2], k_empty[2], v_full[2];
+  uint64_t k_full[KST], k_empty[KST], v_full[2];
   uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
   uint64_t mma_done;
   uint32_t tmem_base;
-  int ntiles;
+  int ntiles, meta_ok;
   PTile tiles[MAX_TILES];
 };
 
@@ -85,7 +96,8 @@ struct PrefillParams {
   CUtensorMap tmap_v[4];
   const int32_t* meta;
   int seq, s_max, L, layer, T;
-  float* out;  // FP32 [2][T][16][256]: branch outputs
+  float* out;   // FP32 [2 branches][NSPLIT][T][16][256]: each split's O / l
+  float2* ml;   // [2][NSPLIT][T][16]: each split's (running maximum m in log2 units, l)
   int32_t* err;
 };
 
@@ -97,22 +109,36 @@ __device__ int build_tiles(PTile* tl, int br, int g, int i0, int T, int t0, int 
   const int i_last = min(T, i0 + PQ_TOK) - 1;
   int n = 0;
   if (br == 0) {
-    // ring tiles holding at least one position the tile's first query still sees
-    const int lo_min = max(0, t0 + i0 - (WIN - 1));
+    // ring tiles holding at least one position the item's first query still sees
+    const int lo_first = max(0, t0 + i0 - (WIN - 1));
+    const int lo_last = max(0, t0 + i_last - (WIN - 1));
+    // slot w = t0 mod 1024 holds the oldest position t0-1024, slot w-1 the newest t0-1;
+    // elsewhere positions rise by one per slot
+    const int w = t0 & (WIN - 1);
     for (int rt = 0; rt < WIN / PKT && t0 > 0; ++rt) {
-      int newest = INT_MIN;
-      for (int k = 0; k < PKT; ++k)
-        newest = max(newest, t0 - WIN + ((rt * PKT + k - t0) & (WIN - 1)));
-      if (newest >= lo_min) tl[n++] = {KIND_RING, gi * WIN + rt * PKT, rt * PKT, 0};
+      const int a = rt * PKT, z = a + PKT - 1;
+      const int pos_a = t0 - WIN + ((a - t0) & (WIN - 1));
+      const int pos_z = t0 - WIN + ((z - t0) & (WIN - 1));
+      const int oldest = (w >= a && w <= z) ? t0 - WIN : pos_a;
+      const int newest = (w > a && w <= z) ? t0 - 1 : pos_z;
+      if (newest >= lo_first)
+        tl[n++] = {KIND_RING, gi * WIN + a, a, oldest >= lo_last ? 1 : 0};
     }
     for (int ct = 0; ct * PKT <= i_last; ++ct)
-      tl[n++] = {KIND_CHUNK, g * T + ct * PKT, ct * PKT, 0};
+      tl[n++] = {KIND_CHUNK, g * T + ct * PKT, ct * PKT, ct * PKT + PKT - 1 <= i0 ? 1 : 0};
   } else {
-    for (int bt = 0; bt * PKT < c; ++bt) tl[n++] = {KIND_BANK, gi * BANK + bt * PKT, bt * PKT, 0};
+    for (int bt = 0; bt * PKT < c; ++bt)
+      tl[n++] = {KIND_BANK, gi * BANK + bt * PKT, bt * PKT, bt * PKT + PKT <= c ? 1 : 0};
     for (int pt = 0; pt * PKT <= p0 + i_last; ++pt)
-      tl[n++] = {KIND_PEND, gi * PEND + pt * PKT, pt * PKT, 0};
+      tl[n++] = {KIND_PEND, gi * PEND + pt * PKT, pt * PKT, pt * PKT + PKT - 1 <= p0 + i0 ? 1 : 0};
   }
   return n;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __global__ void __launch_bounds__(PF_THREADS, 1)
@@ -121,7 +147,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i0 = blockIdx.x * PQ_TOK, g = blockIdx.y, br = blockIdx.z;
+  const int i0 = blockIdx.x * PQ_TOK, g = blockIdx.y;
+  const int br = blockIdx.z / NSPLIT, split = blockIdx.z % NSPLIT;
   const int T = P.T;
   const int t0 = P.meta[P.seq * 4 + 0];
   const int p0 = P.meta[P.seq * 4 + 1];
@@ -130,9 +157,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&S.q_full, 1);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < KST; ++b) {
       mbar_init(&S.k_full[b], 1);
       mbar_init(&S.k_empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&S.v_full[b], 1);
       mbar_init(&S.s_full[b], 1);
       mbar_init(&S.s_empty[b], 128);
@@ -142,8 +171,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     mbar_init(&S.mma_done, 1);
     fence_mbar_init();
     const bool meta_ok = t0 >= 0 && p0 >= 0 && c >= 0 && c <= BANK && p0 + T <= PEND;
-    S.ntiles = meta_ok ? build_tiles(S.tiles, br, g, i0, T, t0, p0, c, gi) : 0;
-    if (!meta_ok) set_dev_error(P.err, ER_ECAPACITY);
+    int nt = 0;
+    if (meta_ok) {
+      // this CTA's contiguous share of the item's tiles
+      const int all = build_tiles(S.tiles, br, g, i0, T, t0, p0, c, gi);
+      const int tb = all * split / NSPLIT, te = all * (split + 1) / NSPLIT;
+      for (int j = tb; j < te; ++j) S.tiles[j - tb] = S.tiles[j];
+      nt = te - tb;
+    } else {
+      set_dev_error(P.err, ER_ECAPACITY);
+    }
+    S.ntiles = nt;
+    S.meta_ok = meta_ok ? 1 : 0;
   }
   if (warp == 5) tc::tmem_alloc(&S.tmem_base, TMEM_COLS);
   tc::fence_before_sync();
@@ -160,8 +199,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         tc::tma_load_4d(S.q[d], &P.tmap_q[br], 64 * d, 0, g, i0, &S.q_full);
       int issued = 0;
       for (int j = 0; j < n; ++j) {
-        const int b = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
+        const int b = j % KST;
+        const uint32_t ph = (j / KST) & 1;
         if (!mbar_wait(&S.k_empty[b], ph ^ 1, P.err)) break;
         const PTile tl = S.tiles[j];
         mbar_arrive_expect_tx(&S.k_full[b], KTILE);
@@ -171,8 +210,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       }
       // no copy may still be landing when the block exits
       mbar_wait(&S.q_full, 0, P.err);
-      for (int j = max(0, issued - 2); j < issued; ++j)
-        mbar_wait(&S.k_full[j & 1], (j >> 1) & 1, P.err);
+      for (int j = max(0, issued - KST); j < issued; ++j)
+        mbar_wait(&S.k_full[j % KST], (j / KST) & 1, P.err);
     }
   } else if (warp == 6) {
     // ---------------------------------------------------------- V producer
@@ -199,9 +238,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       bool ok = mbar_wait(&S.q_full, 0, P.err);
       for (int j = 0; ok && j <= n; ++j) {
         if (j < n) {
-          const int b = j & 1;
+          const int b = j & 1, kb = j % KST;
           const uint32_t ph = (j >> 1) & 1;
-          ok = mbar_wait(&S.k_full[b], ph, P.err) && mbar_wait(&S.s_empty[b], ph ^ 1, P.err);
+          ok = mbar_wait(&S.k_full[kb], (j / KST) & 1, P.err) &&
+               mbar_wait(&S.s_empty[b], ph ^ 1, P.err);
           if (!ok) break;
           tc::fence_after_sync();
           const uint32_t d_s = tmem + TM_S + PKT * b;
@@ -210,11 +250,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const uint64_t a =
                 tc::desc_sw128(smem_u32(S.q[kk >> 2]) + 32 * (kk & 3), 16, 1024);
             const uint64_t bd =
-                tc::desc_sw128(smem_u32(S.k[b]) + (kk >> 2) * KBOX + 32 * (kk & 3), 16, 1024);
+                tc::desc_sw128(smem_u32(S.k[kb]) + (kk >> 2) * KBOX + 32 * (kk & 3), 16, 1024);
             tc::mma_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
           }
           tc::commit(&S.s_full[b]);
-          tc::commit(&S.k_empty[b]);
+          tc::commit(&S.k_empty[kb]);
         }
         if (j >= 1) {
           const int jj = j - 1, b = jj & 1;
@@ -224,10 +264,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < PKT / 16; ++kk) {
-            const uint64_t a = tc::desc_sw128(smem_u32(S.p[b]) + 32 * kk, 16, 1024);
-            // V tile as the MN-major B operand: 64-dim blocks KBOX apart, 8-key groups 1 KB apart
+            // P from TMEM (16 keys = 8 columns per step); V tile as the MN-major B
+            // operand: 64-dim blocks KBOX apart, 8-key groups 1 KB apart
             const uint64_t bd = tc::desc_sw128(smem_u32(S.v[b]) + 2048 * kk, KBOX, 1024);
-            tc::mma_bf16_ss(tmem + TM_O, a, bd, idesc_pv, (jj > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + TM_O, tmem + TM_P + (PKT / 2) * b + 8 * kk, bd, idesc_pv,
+                            (jj > 0 || kk > 0) ? 1u : 0u);
           }
           tc::commit(&S.pv_done[b]);
         }
@@ -242,7 +283,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const int i = i0 + (r >> 2), hh = r & 3;
     const int t = t0 + i;
     const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
-    float m = -INFINITY, l = 0.f;
+    // ring slot u = (slot - t0) mod 1024 holds position t0 - 1024 + u: visible from
+    // u >= uth on; other kinds: key index base + k visible up to hi_*
+    const int uth = max(0, t - (WIN - 1)) - (t0 - WIN);
+    const int hi_chunk = i, hi_bank = c - 1, hi_pend = p0 + i;
+    float m = -INFINITY, l = 0.f;  // m in log2 units (scores x log2(e)/16)
     bool ok = n > 0;
     for (int j = 0; ok && j < n; ++j) {
       const int b = j & 1;
@@ -265,35 +310,33 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       tc::fence_before_sync();
       mbar_arrive(&S.s_empty[b]);
 
-      // which keys of this tile the row may see
       const PTile tl = S.tiles[j];
-      int lo = 0, hi = -1;
-      if (tl.kind == KIND_RING) {
-        lo = max(0, t - (WIN - 1));
-        hi = t;
-      } else if (tl.kind == KIND_CHUNK) {
-        hi = i;
-      } else if (tl.kind == KIND_BANK) {
-        hi = c - 1;
-      } else {
-        hi = p0 + i;
-      }
-      float mt = -INFINITY;
+      if (!tl.full) {
+        if (tl.kind == KIND_RING) {
+          const int ub = tl.base - t0;
 #pragma unroll
-      for (int k = 0; k < PKT; ++k) {
-        const int v = tl.kind == KIND_RING ? t0 - WIN + ((tl.base + k - t0) & (WIN - 1))
-                                           : tl.base + k;
-        s[k] = (v >= lo && v <= hi) ? s[k] * SCALE_LOG2 : -INFINITY;
-        mt = fmaxf(mt, s[k]);
+          for (int k = 0; k < PKT; ++k)
+            if (((ub + k) & (WIN - 1)) < uth) s[k] = -INFINITY;
+        } else {
+          const int khi =
+              (tl.kind == KIND_CHUNK ? hi_chunk : tl.kind == KIND_BANK ? hi_bank : hi_pend) -
+              tl.base;
+#pragma unroll
+          for (int k = 0; k < PKT; ++k)
+            if (k > khi) s[k] = -INFINITY;
+        }
       }
-      const float m_new = fmaxf(m, mt);
+      float mt = s[0];
+#pragma unroll
+      for (int k = 1; k < PKT; ++k) mt = fmaxf(mt, s[k]);
+      const float m_new = fmaxf(m, mt * SCALE_LOG2);
       const bool need = (m != -INFINITY) && (m_new > m + RESCALE_AT);
       if (__any_sync(0xffffffffu, need)) {
         // O holds P_0..P_{j-1}·V: wait for the last of those products, then rescale
         ok = warp_all(mbar_wait(&S.pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, P.err));
         if (!ok) break;
         tc::fence_after_sync();
-        const float f = need ? exp2f(m - m_new) : 1.f;
+        const float f = need ? ex2_approx(m - m_new) : 1.f;
 #pragma unroll 1
         for (int cb = 0; cb < 8; ++cb) {
           uint32_t o[32];
@@ -312,10 +355,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       float lsum = 0.f;
 #pragma unroll
       for (int k = 0; k < PKT; k += 2) {
-        const __nv_bfloat162 h2 =
-            __floats2bfloat162_rn(exp2f(s[k] - msub), exp2f(s[k + 1] - msub));
-        const float2 back = __bfloat1622float2(h2);
-        lsum += back.x + back.y;
+        const float pa = ex2_approx(fmaf(s[k], SCALE_LOG2, -msub));
+        const float pb = ex2_approx(fmaf(s[k + 1], SCALE_LOG2, -msub));
+        lsum += pa + pb;
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(pa, pb);
         pk[k >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       l += lsum;
@@ -324,33 +367,53 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         ok = warp_all(mbar_wait(&S.pv_done[b], ((j - 2) >> 1) & 1, P.err));
         if (!ok) break;
       }
-      unsigned char* prow = S.p[b] + r * 128;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4*>(prow + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      tc::fence_async_smem();
+      tc::tmem_st32(tmem + lane_addr + TM_P + (PKT / 2) * b, pk);
+      tc::tmem_wait_st();
       tc::fence_before_sync();
       mbar_arrive(&S.p_full[b]);
     }
     if (ok) ok = warp_all(mbar_wait(&S.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, P.err));
+    // this split's partial result: O / l and (m, l); a split without keys for the
+    // row (or without tiles) leaves O = 0, m = -inf, l = 0
+    const size_t row = ((size_t)(br * NSPLIT + split) * T + i) * NH + 4 * g + hh;
     if (ok) {
+      // every MMA and copy of the block is complete: the K stages serve as a 4 KB
+      // staging tile per warp, so each store instruction writes 4 whole 128-byte
+      // row segments (row r keeps its 16-byte chunk c at position c ^ (r & 7))
       tc::fence_after_sync();
-      const float inv = 1.f / l;
-      float* dst = P.out + ((size_t)(br * T + i) * NH + 4 * g + hh) * D;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* stage = reinterpret_cast<float*>(S.k[0]) + warp * (32 * 32);
+      const int q8 = lane & 7;
 #pragma unroll 1
       for (int cb = 0; cb < 8; ++cb) {
         uint32_t o[32];
         tc::tmem_ld32(tmem + lane_addr + TM_O + 32 * cb, o);
         tc::tmem_wait_ld();
-        if (i < T) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + 32 * cb + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(stage + lane * 32 + ((c ^ (lane & 7)) << 2)) =
+              make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
+                          __uint_as_float(o[4 * c + 2]) * inv,
+                          __uint_as_float(o[4 * c + 3]) * inv);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = 4 * k + (lane >> 3);      // row of this warp's 32
+          const int rg = 32 * warp + rr;           // row of the tile
+          const int ti = i0 + (rg >> 2);
+          if (ti < T) {
+            const size_t grow = ((size_t)(br * NSPLIT + split) * T + ti) * NH + 4 * g + (rg & 3);
+            *reinterpret_cast<float4*>(P.out + grow * D + 32 * cb + 4 * q8) =
+                *reinterpret_cast<const float4*>(stage + rr * 32 + ((q8 ^ (rr & 7)) << 2));
+          }
         }
+        __syncwarp();
       }
+      if (i < T) P.ml[row] = make_float2(m, l);
+    } else if (n == 0 && S.meta_ok && i < T) {
+      float4* dst = reinterpret_cast<float4*>(P.out + row * D);
+      for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      P.ml[row] = make_float2(-INFINITY, 0.f);
     }
   }
   tc::fence_before_sync();
@@ -361,25 +424,50 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   }
 }
 
-// o_sum[t][h*256 + d] = bf16(o_swa + o_rma), 8 values per thread.
-__global__ void k_prefill_combine(const float* __restrict__ out, int T,
-                                  uint16_t* __restrict__ o_sum) {
+// o_sum[t][h*256 + d] = bf16(o_swa + o_rma), each branch the merge of its
+// NSPLIT partial reads weighted by l·2^(m - M); 8 values per thread.
+__global__ void k_prefill_combine(const float* __restrict__ out, const float2* __restrict__ ml,
+                                  int T, uint16_t* __restrict__ o_sum) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * (OIN / 8)) return;
-  const size_t e = (size_t)idx * 8;
-  const float4* a = reinterpret_cast<const float4*>(out + e);
-  const float4* b = reinterpret_cast<const float4*>(out + (size_t)T * OIN + e);
-  const float4 a0 = a[0], a1 = a[1], b0 = b[0], b1 = b[1];
-  const __nv_bfloat162 h0 = __floats2bfloat162_rn(a0.x + b0.x, a0.y + b0.y);
-  const __nv_bfloat162 h1 = __floats2bfloat162_rn(a0.z + b0.z, a0.w + b0.w);
-  const __nv_bfloat162 h2 = __floats2bfloat162_rn(a1.x + b1.x, a1.y + b1.y);
-  const __nv_bfloat162 h3 = __floats2bfloat162_rn(a1.z + b1.z, a1.w + b1.w);
-  uint4 v;
-  v.x = *reinterpret_cast<const uint32_t*>(&h0);
-  v.y = *reinterpret_cast<const uint32_t*>(&h1);
-  v.z = *reinterpret_cast<const uint32_t*>(&h2);
-  v.w = *reinterpret_cast<const uint32_t*>(&h3);
-  *reinterpret_cast<uint4*>(o_sum + e) = v;
+  const int row = idx / (D / 8);  // token * 16 + head
+  const int d0 = (idx % (D / 8)) * 8;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    float2 v[NSPLIT];
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < NSPLIT; ++sp) {
+      v[sp] = ml[(size_t)(br * NSPLIT + sp) * T * NH + row];
+      if (v[sp].y > 0.f) M = fmaxf(M, v[sp].x);
+    }
+    float w[NSPLIT], wsum = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < NSPLIT; ++sp) {
+      w[sp] = v[sp].y > 0.f ? exp2f(v[sp].x - M) * v[sp].y : 0.f;
+      wsum += w[sp];
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+#pragma unroll
+    for (int sp = 0; sp < NSPLIT; ++sp) {
+      if (w[sp] == 0.f) continue;
+      const float ws = w[sp] * inv;
+      const float4* src = reinterpret_cast<const float4*>(
+          out + ((size_t)(br * NSPLIT + sp) * T * NH + row) * D + d0);
+      const float4 x0 = src[0], x1 = src[1];
+      acc[0] += ws * x0.x; acc[1] += ws * x0.y; acc[2] += ws * x0.z; acc[3] += ws * x0.w;
+      acc[4] += ws * x1.x; acc[5] += ws * x1.y; acc[6] += ws * x1.z; acc[7] += ws * x1.w;
+    }
+  }
+  uint4 pk;
+  uint32_t* pw = reinterpret_cast<uint32_t*>(&pk);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * q], acc[2 * q + 1]);
+    pw[q] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+  *reinterpret_cast<uint4*>(o_sum + (size_t)idx * 8) = pk;
 }
 
 bool g_pf_attr[64] = {false};
@@ -387,8 +475,11 @@ std::mutex g_pf_mu;
 
 }  // namespace
 
-// Workspace FP32 floats for the branch outputs of a T-token chunk.
-size_t prefill_out_floats(int T) { return (size_t)2 * T * OIN; }
+// Workspace FP32 floats for the partial reads of a T-token chunk: O / l per
+// (branch, split, token, head), then (m, l) pairs.
+size_t prefill_out_floats(int T) {
+  return (size_t)2 * NSPLIT * T * OIN + (size_t)2 * NSPLIT * T * NH * 2;
+}
 
 int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const uint16_t* q_swa,
                           const uint16_t* q_rma, const uint16_t* chunk_k,
@@ -428,11 +519,15 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   P.layer = layer;
   P.T = T;
   P.out = out;
+  P.ml = reinterpret_cast<float2*>(out + (size_t)2 * NSPLIT * T * OIN);
   P.err = st->dev_error;
-  const dim3 grid((T + PQ_TOK - 1) / PQ_TOK, NG, 2);
+  const dim3 grid((T + PQ_TOK - 1) / PQ_TOK, NG, 2 * NSPLIT);
+  std::pair<cudaEvent_t, cudaEvent_t> ev;
+  const bool timed = profile_begin(stream, &ev);
   k_prefill_attn<<<grid, PF_THREADS, PF_SMEM, stream>>>(P);
+  if (timed) profile_end(stream, ev);
   const int nv = T * (OIN / 8);
-  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, T, o_sum);
+  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, P.ml, T, o_sum);
   count_launches(2);
   return launch_status();
 }

@@ -54,6 +54,18 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a, uint64_
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
 
+// D[tmem] (+)= A·B with A read from TMEM (K-major: row i in lane i, two 16-bit
+// elements per 32-bit column, lower K index in the low half) and B from
+// shared memory; one thread issues.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+
 // The mbarrier receives one arrival once every MMA issued so far by this
 // thread has completed (its shared-memory operands may then be reused).
 __device__ __forceinline__ void commit(uint64_t* bar) {

@@ -56,11 +56,14 @@ def test_score_matches_oracle(sab, n):
     seed = 100 + n
     w = wl.make_weights(seed, 0)
     x = synth.normal((max(n, 1), 2560), seed, synth.MISC, torch.bfloat16)[:n]
-    gw, _ = H.gpu_weights(seed, 0)
+    gw, wdev = H.gpu_weights(seed, 0)
     got = sab.rma_score(gw, x.cuda()).cpu()
     if n == 0:
         assert got.shape == (0, 4)
         return
+    # W1 terms prepared with the weights or made by the call: the same terms, the same bits
+    unprepared = sab.LayerWeights.from_dict(wdev, prepare=False)
+    assert torch.equal(sab.rma_score(unprepared, x.cuda()).cpu(), got)
     ref = oracle.score(w["w1"], w["w2"], x)
     h = torch.nn.functional.silu(x.double() @ w["w1"].double().T).abs()
     cond = ref.double().abs() + h @ w["w2"].double().abs().T

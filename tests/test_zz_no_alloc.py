@@ -2,8 +2,9 @@
 
 Some callers of this library cannot give it scratch memory: their device
 memory belongs to another framework's allocator, or they only receive the
-input and output pointers.  For them the library keeps the scorer's split-K
-partial sums in a fixed array of its own (at most 256 tokens per call).  This
+input and output pointers.  For them the library keeps the scorer's scratch
+(W1 as three BF16 terms, the partial scores) in a fixed array of its own (at
+most 256 tokens per call).  This
 file checks, through the C ABI, that the allocation-free call returns what the
 workspace call returns, on two calls in a row (the second finds the array
 holding the first call's leftovers), and that a size above the maximum is
