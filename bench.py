@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-commit-bench", action="store_true")
     ap.add_argument("--no-prefill-bench", action="store_true")
+    ap.add_argument("--no-rma-off", action="store_true",
+                    help="skip the decode pass with the RMA switched off (the ablation)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph pass (one captured graph per decode step)")
     ap.add_argument("--prefill-chunks", type=int, default=512,
@@ -302,6 +304,40 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "steps": k_e2e}
 
 
+    rma_off = None
+    if not args.no_rma_off:
+        # the pages' ablation: the same decode with every RMA module off (window read only)
+        k_off = min(args.steps, 64)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        sab.profile_read(reset=True)
+        sab.profile_enable(True)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for s in range(k_off):
+            for l in range(LAYERS):
+                sab.swa_rma_decode(st, weights[l], l, ids, xs[s % n_x][l], out=outs[l], ws=ws,
+                                   rma_off=True)
+            sab.advance(st, ids, rma_off=True)
+        r1.record(stream)
+        torch.cuda.synchronize(dev)
+        sab.profile_enable(False)
+        off_attend_ms, off_attend_n = sab.profile_read(reset=True)
+        if sab.last_device_error(st) != 0:
+            raise RuntimeError("device error in the RMA-off pass")
+        off_ms = reduce_max(r0.elapsed_time(r1), dev)
+        # per (sequence, group): 1024 window rows (K + V), q_swa (4 x 512 B), o (4 x 1 KiB)
+        alg = B * 4 * (1024 * ROW + 4 * 512 + 4 * 1024)
+        hbm, kind = peaks()
+        per = off_attend_ms / max(off_attend_n, 1)
+        rma_off = {"value": whole_job_tokens_per_s(world, B, k_off, off_ms),
+                   "ms_per_step": off_ms / k_off, "steps": k_off,
+                   "attend_avg_launch_ms": per,
+                   "attend_frac": alg / (per / 1e3) / 1e9 / hbm if per > 0 else None,
+                   "attend_alg_bytes_per_launch": alg,
+                   "note": "ER_FLAG_RMA_OFF, eager: o_rma = 0, no score, append or commit"}
+
     ms = reduce_max(ms, dev)
     cm = None
     if not args.no_commit_bench and rank == 0:
@@ -312,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
         pf = prefill_bench(dev, args.prefill_chunks)
     return dict(ms=ms, launches=launches, clocks=clk, attend_ms=attend_ms, attend_n=attend_n,
                 fills=fills, commits=commits, e2e=e2e, commit_microbench=cm, prefill=pf,
-                graph=graph)
+                graph=graph, rma_off=rma_off)
 
 
 # ------------------------------------------------------- commit microbench
@@ -665,6 +701,7 @@ def main():
         "clocks": r["clocks"],
         "commit_microbench": r["commit_microbench"],
         "prefill": r["prefill"],
+        "rma_off": r["rma_off"],
         "eager": {"value": whole_job_tokens_per_s(world, B, args.steps, r["ms"]),
                   "ms_per_step": r["ms"] / args.steps, "gpu_launches": r["launches"],
                   "note": "the same steps launched call by call through the binding; "

@@ -144,6 +144,20 @@ int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stre
 int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
                er_stream_t stream);
 
+/* Flags of the *_ex calls.
+ *   ER_FLAG_RMA_OFF: the pages' ablation with every RMA module switched off
+ *   at inference time, recurrent layers and local attention kept (fluxbbs.com
+ *   "EdgeRock-4B 开源：72 MiB 固定 KV" §消融：关掉 RMA 会发生什么; neodrop.ai
+ *   §三段记忆，只记值得记的).  The layer calls then take o_rma = 0 and skip the score, the
+ *   pending append and the commit; er_advance_ex moves only the position, so
+ *   the anchor bank, the pending block and their counters stay as they were.
+ *   Use it for every layer of a step and for that step's advance. */
+#define ER_FLAG_RMA_OFF 1u
+
+/* er_advance with flags (0 or ER_FLAG_RMA_OFF; other bits: ER_EINVAL). */
+int er_advance_ex(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
+                  uint32_t flags, er_stream_t stream);
+
 /* Copies the device error word to *code (host) and clears it; synchronises
  * `stream`.  Returns ER_OK when the word was 0, else ER_EDEVICE. */
 int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream);
@@ -261,6 +275,19 @@ size_t er_prefill_workspace_bytes(int32_t T);
 int er_swa_rma_prefill_chunk(const er_state* st, const er_layer_weights* w, int32_t layer,
                              int32_t seq_id, const er_bf16* x, int32_t T, er_bf16* out,
                              void* ws, size_t ws_bytes, er_stream_t stream);
+
+/* The two layer calls with flags (0 or ER_FLAG_RMA_OFF; other bits:
+ * ER_EINVAL).  With ER_FLAG_RMA_OFF: out = W_o · bf16(o_swa), the window is
+ * written and read as usual, and the RMA memory (scores, pending block, bank,
+ * their counters) is neither read by the attention nor written; a prefill
+ * chunk still obeys pend_count + T <= 256.  Same workspace sizes.  The
+ * flag-less calls above are these with flags = 0. */
+int er_swa_rma_decode_ex(const er_state* st, const er_layer_weights* w, int32_t layer,
+                         const int32_t* seq_ids, int32_t B, const er_bf16* x, er_bf16* out,
+                         void* ws, size_t ws_bytes, uint32_t flags, er_stream_t stream);
+int er_swa_rma_prefill_chunk_ex(const er_state* st, const er_layer_weights* w, int32_t layer,
+                                int32_t seq_id, const er_bf16* x, int32_t T, er_bf16* out,
+                                void* ws, size_t ws_bytes, uint32_t flags, er_stream_t stream);
 
 /* ------------------------------------------------------ instrumentation */
 

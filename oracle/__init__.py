@@ -60,9 +60,9 @@ def lib():
         L.orc_score.argtypes = [vp, vp, vp, i32, vp]
         L.orc_attend_rows.argtypes = [vp, vp, vp, i32, vp]
         L.orc_commit.argtypes = [vp, i32, i32, vp]
-        L.orc_advance.argtypes = [vp, i32, i32]
-        L.orc_decode_layer.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp]
-        L.orc_prefill_chunk.argtypes = [vp, vp, i32, i32, vp, i32, vp]
+        L.orc_advance.argtypes = [vp, i32, i32, i32]
+        L.orc_decode_layer.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, i32]
+        L.orc_prefill_chunk.argtypes = [vp, vp, i32, i32, vp, i32, vp, i32]
         L.orc_prefill_chunk.restype = ctypes.c_int
         L.orc_append_pending.argtypes = [vp, i32, vp, i32, vp, vp, vp, vp]
         L.orc_f64_to_bf16.argtypes = [ctypes.c_double]
@@ -144,19 +144,20 @@ class OracleState:
 
     # ----------------------------------------------------------- the layer
     def decode_layer(self, w: OracleWeights, layer: int, seq: int, x: torch.Tensor,
-                     want_branches: bool = False):
+                     want_branches: bool = False, rma_off: bool = False):
         out = torch.empty(HIDDEN, dtype=torch.bfloat16)
         o_swa = torch.empty(NH, D, dtype=torch.float64) if want_branches else None
         o_rma = torch.empty(NH, D, dtype=torch.float64) if want_branches else None
         lib().orc_decode_layer(w.ptr(), self.ptr(), layer, seq, _p(x.contiguous()), _p(out),
-                               _p(o_swa), _p(o_rma))
+                               _p(o_swa), _p(o_rma), 1 if rma_off else 0)
         return (out, o_swa, o_rma) if want_branches else out
 
-    def prefill_chunk(self, w: OracleWeights, layer: int, seq: int, x: torch.Tensor):
+    def prefill_chunk(self, w: OracleWeights, layer: int, seq: int, x: torch.Tensor,
+                      rma_off: bool = False):
         T = x.shape[0]
         out = torch.empty(T, HIDDEN, dtype=torch.bfloat16)
         rc = lib().orc_prefill_chunk(w.ptr(), self.ptr(), layer, seq, _p(x.contiguous()), T,
-                                     _p(out))
+                                     _p(out), 1 if rma_off else 0)
         if rc != 0:
             raise ValueError("prefill chunk crosses the pending block boundary")
         return out
@@ -169,8 +170,8 @@ class OracleState:
         lib().orc_commit(self.ptr(), layer, seq, _p(kept))
         return kept
 
-    def advance(self, seq: int, T: int = 1):
-        lib().orc_advance(self.ptr(), seq, T)
+    def advance(self, seq: int, T: int = 1, rma_off: bool = False):
+        lib().orc_advance(self.ptr(), seq, T, 1 if rma_off else 0)
 
     def append_pending(self, layer, seqs, k, v, s, pos):
         seqs = torch.as_tensor(seqs, dtype=torch.int32).contiguous()

@@ -330,10 +330,12 @@ void orc_commit(orc_state* st, int layer, int seq, int32_t* kept) {
 }
 
 /* End of a step of T tokens (after every layer): position and pending count
- * advance; a full block has been committed by each layer, so it empties. */
-void orc_advance(orc_state* st, int seq, int T) {
+ * advance; a full block has been committed by each layer, so it empties.
+ * With the RMA switched off (the pages' ablation) only the position moves. */
+void orc_advance(orc_state* st, int seq, int T, int rma_off) {
   int32_t* meta = st->meta + (size_t)seq * 4;
   meta[0] += T;
+  if (rma_off) return;
   meta[1] += T;
   if (meta[1] >= OPEND) {
     meta[1] = 0;
@@ -383,9 +385,11 @@ static void output_token(const orc_weights* w, double o_swa[ONH][OD], double o_r
 /* ------------------------------------------------------- decode (a1–a7) */
 
 /* One decode step of one layer for one sequence.  Optional o_swa / o_rma
- * ([16][256] float64) receive the two branch outputs before o_proj. */
+ * ([16][256] float64) receive the two branch outputs before o_proj.  With
+ * rma_off (the pages' ablation of the RMA modules) the RMA output is 0, the
+ * token is not appended to pending and nothing commits. */
 void orc_decode_layer(const orc_weights* w, orc_state* st, int layer, int seq, const uint16_t* x,
-                      uint16_t* out, double* o_swa_out, double* o_rma_out) {
+                      uint16_t* out, double* o_swa_out, double* o_rma_out, int rma_off) {
   int32_t* meta = st->meta + (size_t)seq * 4;
   int32_t t = meta[0];
   int p = meta[1], c = meta[2];
@@ -397,6 +401,7 @@ void orc_decode_layer(const orc_weights* w, orc_state* st, int layer, int seq, c
   for (int g = 0; g < ONG; ++g) {
     memcpy(win_k_row(st, seq, layer, g, t % OWIN), tk->k_swa[g], OD * 2);
     memcpy(win_v_row(st, seq, layer, g, t % OWIN), tk->v_swa[g], OD * 2);
+    if (rma_off) continue;
     memcpy(pend_k_row(st, seq, layer, g, p), tk->k_rma[g], OD * 2);
     memcpy(pend_v_row(st, seq, layer, g, p), tk->v_rma[g], OD * 2);
     st->pend_score[(gi0 + g) * OPEND + p] = tk->s[g];
@@ -417,6 +422,10 @@ void orc_decode_layer(const orc_weights* w, orc_state* st, int layer, int seq, c
       ++n;
     }
     attend(tk->q_swa[h], kr, vr, n, o_swa[h]);
+    if (rma_off) {
+      for (int d = 0; d < OD; ++d) o_rma[h][d] = 0.0;
+      continue;
+    }
     n = 0;
     for (int i = 0; i < c; ++i) {
       kr[n] = bank_k_row(st, seq, layer, g, i);
@@ -436,7 +445,7 @@ void orc_decode_layer(const orc_weights* w, orc_state* st, int layer, int seq, c
 
   /* a7: the token that fills the block is read with all 1280 records, then
    * this layer commits; metadata moves on in orc_advance. */
-  if (p + 1 == OPEND) {
+  if (!rma_off && p + 1 == OPEND) {
     meta[1] = OPEND;
     orc_commit(st, layer, seq, NULL);
     meta[1] = p;
@@ -453,7 +462,7 @@ void orc_decode_layer(const orc_weights* w, orc_state* st, int layer, int seq, c
  * t0, the chunk's own tokens from t0) and the bank plus pending 0..p0+i.  The
  * chunk enters the ring after every token has been read. */
 int orc_prefill_chunk(const orc_weights* w, orc_state* st, int layer, int seq,
-                      const uint16_t* x, int T, uint16_t* out) {
+                      const uint16_t* x, int T, uint16_t* out, int rma_off) {
   int32_t* meta = st->meta + (size_t)seq * 4;
   int32_t t0 = meta[0];
   int p0 = meta[1], c = meta[2];
@@ -461,7 +470,7 @@ int orc_prefill_chunk(const orc_weights* w, orc_state* st, int layer, int seq,
   orc_tok* tk = (orc_tok*)malloc(sizeof(orc_tok) * (size_t)T);
   for (int i = 0; i < T; ++i) project_token(w, x + (size_t)i * OHID, t0 + i, &tk[i]);
   size_t gi0 = gidx(st, seq, layer, 0);
-  for (int i = 0; i < T; ++i)
+  for (int i = 0; i < T && !rma_off; ++i)
     for (int g = 0; g < ONG; ++g) {
       memcpy(pend_k_row(st, seq, layer, g, p0 + i), tk[i].k_rma[g], OD * 2);
       memcpy(pend_v_row(st, seq, layer, g, p0 + i), tk[i].v_rma[g], OD * 2);
@@ -488,6 +497,10 @@ int orc_prefill_chunk(const orc_weights* w, orc_state* st, int layer, int seq,
         ++n;
       }
       attend(tk[i].q_swa[h], kr, vr, n, o_swa[h]);
+      if (rma_off) {
+        for (int d = 0; d < OD; ++d) o_rma[h][d] = 0.0;
+        continue;
+      }
       n = 0;
       for (int b = 0; b < c; ++b) {
         kr[n] = bank_k_row(st, seq, layer, g, b);
@@ -508,7 +521,7 @@ int orc_prefill_chunk(const orc_weights* w, orc_state* st, int layer, int seq,
       memcpy(win_k_row(st, seq, layer, g, (t0 + i) % OWIN), tk[i].k_swa[g], OD * 2);
       memcpy(win_v_row(st, seq, layer, g, (t0 + i) % OWIN), tk[i].v_swa[g], OD * 2);
     }
-  if (p0 + T == OPEND) {
+  if (!rma_off && p0 + T == OPEND) {
     meta[1] = OPEND;
     orc_commit(st, layer, seq, NULL);
     meta[1] = p0;

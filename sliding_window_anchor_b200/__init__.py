@@ -123,10 +123,15 @@ def state_init(st: State, seq_ids, stream=None):
                                                stream_handle(stream, st.device)))
 
 
-def advance(st: State, seq_ids, T: int = 1, stream=None):
+def _flags(rma_off: bool) -> int:
+    return _lib.ER_FLAG_RMA_OFF if rma_off else 0
+
+
+def advance(st: State, seq_ids, T: int = 1, stream=None, rma_off: bool = False):
+    """End of a step of T tokens; with rma_off only the positions move."""
     ids = _ids(seq_ids, st.device)
-    check("er_advance", lib().er_advance(st.ptr(), dev_ptr(ids), ids.numel(), T,
-                                         stream_handle(stream, st.device)))
+    check("er_advance_ex", lib().er_advance_ex(st.ptr(), dev_ptr(ids), ids.numel(), T,
+                                               _flags(rma_off), stream_handle(stream, st.device)))
 
 
 def last_device_error(st: State, stream=None) -> int:
@@ -224,26 +229,26 @@ def swa_rma_attend(st: State, layer: int, seq_ids, q_swa, q_rma, ws=None, stream
 
 
 def swa_rma_decode(st: State, w: LayerWeights, layer: int, seq_ids, x, out=None, ws=None,
-                   stream=None):
+                   stream=None, rma_off: bool = False):
     ids = _ids(seq_ids, st.device)
     B = ids.numel()
     out = torch.empty(B, HIDDEN, dtype=torch.bfloat16, device=st.device) if out is None else out
     ws = _ws(decode_workspace_bytes(B), st.device, ws)
-    check("er_swa_rma_decode", lib().er_swa_rma_decode(
+    check("er_swa_rma_decode_ex", lib().er_swa_rma_decode_ex(
         st.ptr(), w.ptr(), layer, dev_ptr(ids), B, dev_ptr(x, torch.bfloat16, "x"),
-        dev_ptr(out, torch.bfloat16, "out"), dev_ptr(ws), ws.numel(),
+        dev_ptr(out, torch.bfloat16, "out"), dev_ptr(ws), ws.numel(), _flags(rma_off),
         stream_handle(stream, st.device)))
     return out
 
 
 def swa_rma_prefill_chunk(st: State, w: LayerWeights, layer: int, seq_id: int, x, out=None,
-                          ws=None, stream=None):
+                          ws=None, stream=None, rma_off: bool = False):
     T = x.shape[0]
     out = torch.empty(T, HIDDEN, dtype=torch.bfloat16, device=st.device) if out is None else out
     ws = _ws(prefill_workspace_bytes(T), st.device, ws)
-    check("er_swa_rma_prefill_chunk", lib().er_swa_rma_prefill_chunk(
+    check("er_swa_rma_prefill_chunk_ex", lib().er_swa_rma_prefill_chunk_ex(
         st.ptr(), w.ptr(), layer, int(seq_id), dev_ptr(x, torch.bfloat16, "x"), T,
-        dev_ptr(out, torch.bfloat16, "out"), dev_ptr(ws), ws.numel(),
+        dev_ptr(out, torch.bfloat16, "out"), dev_ptr(ws), ws.numel(), _flags(rma_off),
         stream_handle(stream, st.device)))
     return out
 

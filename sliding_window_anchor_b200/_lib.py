@@ -34,6 +34,9 @@ class CState(ctypes.Structure):
         ("s_max", ctypes.c_int32), ("n_layers", ctypes.c_int32)]
 
 
+ER_FLAG_RMA_OFF = 1  # the RMA switched off (the pages' ablation)
+
+
 class CWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_qkv", "w_o", "q_norm_swa", "k_norm_swa",
                                                "q_norm_rma", "k_norm_rma", "w1", "w2",
@@ -49,6 +52,8 @@ EXPORTS = {
                                      ctypes.c_void_p]),
     "er_advance": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_void_p, ctypes.c_int32,
                                   ctypes.c_int32, ctypes.c_void_p]),
+    "er_advance_ex": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_void_p, ctypes.c_int32,
+                                     ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p]),
     "er_last_device_error": (ctypes.c_int, [ctypes.POINTER(CState),
                                             ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
     "er_qk_norm_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
@@ -76,12 +81,22 @@ EXPORTS = {
                                          ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_size_t, ctypes.c_void_p]),
+    "er_swa_rma_decode_ex": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.POINTER(CWeights),
+                                            ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]),
     "er_prefill_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "er_swa_rma_prefill_chunk": (ctypes.c_int, [ctypes.POINTER(CState),
                                                 ctypes.POINTER(CWeights), ctypes.c_int32,
                                                 ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
                                                 ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_size_t, ctypes.c_void_p]),
+    "er_swa_rma_prefill_chunk_ex": (ctypes.c_int, [ctypes.POINTER(CState),
+                                                   ctypes.POINTER(CWeights), ctypes.c_int32,
+                                                   ctypes.c_int32, ctypes.c_void_p,
+                                                   ctypes.c_int32, ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_size_t,
+                                                   ctypes.c_uint32, ctypes.c_void_p]),
     "er_error_string": (ctypes.c_char_p, [ctypes.c_int]),
     "er_launch_count": (ctypes.c_uint64, []),
     "er_profile_enable": (ctypes.c_int, [ctypes.c_int]),

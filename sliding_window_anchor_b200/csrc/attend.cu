@@ -118,6 +118,7 @@ __device__ int item_ranges(const AttendParams& P, int qi, int g, int br, Range r
       r[n++] = Range{TM_CHUNK, g * P.nq, qi + 1};
     }
   } else {
+    if (P.rma_off) return 0;  // the RMA switched off: an empty read, o_rma = 0
     if (bank > 0) r[n++] = Range{TM_BANK, gi * BANK, bank};
     const int np = min(pend + (P.prefill ? qi : 0) + 1, PEND);
     if (np > 0) r[n++] = Range{TM_PEND, gi * PEND, np};

@@ -17,7 +17,7 @@ int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int 
 int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
                  int n, float* s, void* scratch, int32_t* err, cudaStream_t st);
 size_t score_scratch_bytes(int n);
-int launch_post_proj(const PostParams& P, cudaStream_t st);
+int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
                   cudaStream_t st);
 int launch_commit(const CommitParams& P, cudaStream_t st);
@@ -26,7 +26,7 @@ size_t attend_ml_floats(int nq);
 size_t prefill_out_floats(int T);
 int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const uint16_t* q_swa,
                           const uint16_t* q_rma, const uint16_t* chunk_k,
-                          const uint16_t* chunk_v, float* out, uint16_t* o_sum,
+                          const uint16_t* chunk_v, float* out, uint16_t* o_sum, bool rma_off,
                           cudaStream_t stream);
 
 }  // namespace er
@@ -89,16 +89,17 @@ __global__ void k_ring_write(const uint16_t* chunk_k, const uint16_t* chunk_v, u
 
 int run_layer(const er_state* st, const er_layer_weights* w, int layer, const int32_t* seq_ids,
               int seq_fixed, int nq, const uint16_t* x, uint16_t* out, void* ws, size_t ws_bytes,
-              cudaStream_t s) {
+              uint32_t flags, cudaStream_t s) {
   const bool prefill = seq_fixed >= 0;
+  const bool rma_off = (flags & ER_FLAG_RMA_OFF) != 0;
   LayerWs W = carve_ws(ws, nq, prefill);
   if (ws_bytes < W.bytes) return ER_ECAPACITY;
   int rc;
   // a1: all six projections in one GEMM
   if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
-  // a3: FP32 scores
-  if ((rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, W.s, W.score_scratch, st->dev_error,
-                        s)) != ER_OK)
+  // a3: FP32 scores (not with the RMA switched off)
+  if (!rma_off && (rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, W.s, W.score_scratch,
+                                     st->dev_error, s)) != ER_OK)
     return rc;
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
@@ -111,11 +112,11 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   pp.meta = st->meta; pp.seq_ids = seq_ids; pp.s_max = st->s_max; pp.L = st->n_layers;
   pp.layer = layer; pp.prefill = prefill ? 1 : 0; pp.seq_fixed = seq_fixed;
   pp.chunk_k = W.chunk_k; pp.chunk_v = W.chunk_v; pp.err = st->dev_error;
-  if ((rc = launch_post_proj(pp, s)) != ER_OK) return rc;
+  if ((rc = launch_post_proj(pp, rma_off, s)) != ER_OK) return rc;
   // a5 / a8: both reads, merged into bf16(o_swa + o_rma)
   if (prefill) {
     if ((rc = launch_prefill_attend(st, layer, seq_fixed, nq, W.q_swa, W.q_rma, W.chunk_k,
-                                    W.chunk_v, W.pf_out, W.o_sum, s)) != ER_OK)
+                                    W.chunk_v, W.pf_out, W.o_sum, rma_off, s)) != ER_OK)
       return rc;
   } else {
     AttendParams ap{};
@@ -123,7 +124,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     ap.pend_k = st->pend_k; ap.pend_v = st->pend_v; ap.meta = st->meta; ap.seq_ids = seq_ids;
     ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
     ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
-    ap.prefill = 0; ap.seq_fixed = -1;
+    ap.prefill = 0; ap.seq_fixed = -1; ap.rma_off = rma_off ? 1 : 0;
     ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.err = st->dev_error;
     if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, s)) != ER_OK) return rc;
   }
@@ -137,6 +138,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     if ((rc = launch_status()) != ER_OK) return rc;
   }
   // a7: commit this layer where the block is now full (decided on the device)
+  if (rma_off) return ER_OK;
   CommitParams cp{};
   cp.bank_k = st->bank_k; cp.bank_v = st->bank_v; cp.pend_k = st->pend_k; cp.pend_v = st->pend_v;
   cp.bank_score = st->bank_score; cp.pend_score = st->pend_score;
@@ -165,26 +167,41 @@ size_t er_prefill_workspace_bytes(int32_t T) {
   return carve_ws(nullptr, T, true).bytes;
 }
 
-int er_swa_rma_decode(const er_state* st, const er_layer_weights* w, int32_t layer,
-                      const int32_t* seq_ids, int32_t B, const er_bf16* x, er_bf16* out,
-                      void* ws, size_t ws_bytes, er_stream_t stream) {
+int er_swa_rma_decode_ex(const er_state* st, const er_layer_weights* w, int32_t layer,
+                         const int32_t* seq_ids, int32_t B, const er_bf16* x, er_bf16* out,
+                         void* ws, size_t ws_bytes, uint32_t flags, er_stream_t stream) {
   if (!st || B < 0 || layer < 0 || layer >= st->n_layers) return ER_EINVAL;
+  if (flags & ~ER_FLAG_RMA_OFF) return ER_EINVAL;
   if (B == 0) return ER_OK;
   if (B > st->s_max) return ER_ECAPACITY;
   if (!weights_ok(w) || !seq_ids || !x || !out || !ws) return ER_EINVAL;
   if (!aligned16(x) || !aligned16(out) || !aligned16(ws)) return ER_EINVAL;
-  return run_layer(st, w, layer, seq_ids, -1, B, x, out, ws, ws_bytes, (cudaStream_t)stream);
+  return run_layer(st, w, layer, seq_ids, -1, B, x, out, ws, ws_bytes, flags,
+                   (cudaStream_t)stream);
+}
+
+int er_swa_rma_decode(const er_state* st, const er_layer_weights* w, int32_t layer,
+                      const int32_t* seq_ids, int32_t B, const er_bf16* x, er_bf16* out,
+                      void* ws, size_t ws_bytes, er_stream_t stream) {
+  return er_swa_rma_decode_ex(st, w, layer, seq_ids, B, x, out, ws, ws_bytes, 0u, stream);
+}
+
+int er_swa_rma_prefill_chunk_ex(const er_state* st, const er_layer_weights* w, int32_t layer,
+                                int32_t seq_id, const er_bf16* x, int32_t T, er_bf16* out,
+                                void* ws, size_t ws_bytes, uint32_t flags, er_stream_t stream) {
+  if (!st || layer < 0 || layer >= st->n_layers || T < 1 || T > PEND) return ER_EINVAL;
+  if (flags & ~ER_FLAG_RMA_OFF) return ER_EINVAL;
+  if (seq_id < 0 || seq_id >= st->s_max) return ER_EINVAL;
+  if (!weights_ok(w) || !x || !out || !ws) return ER_EINVAL;
+  if (!aligned16(x) || !aligned16(out) || !aligned16(ws)) return ER_EINVAL;
+  return run_layer(st, w, layer, nullptr, seq_id, T, x, out, ws, ws_bytes, flags,
+                   (cudaStream_t)stream);
 }
 
 int er_swa_rma_prefill_chunk(const er_state* st, const er_layer_weights* w, int32_t layer,
                              int32_t seq_id, const er_bf16* x, int32_t T, er_bf16* out,
                              void* ws, size_t ws_bytes, er_stream_t stream) {
-  if (!st || layer < 0 || layer >= st->n_layers || T < 1 || T > PEND) return ER_EINVAL;
-  if (seq_id < 0 || seq_id >= st->s_max) return ER_EINVAL;
-  if (!weights_ok(w) || !x || !out || !ws) return ER_EINVAL;
-  if (!aligned16(x) || !aligned16(out) || !aligned16(ws)) return ER_EINVAL;
-  return run_layer(st, w, layer, nullptr, seq_id, T, x, out, ws, ws_bytes,
-                   (cudaStream_t)stream);
+  return er_swa_rma_prefill_chunk_ex(st, w, layer, seq_id, x, T, out, ws, ws_bytes, 0u, stream);
 }
 
 }  // extern "C"

@@ -138,9 +138,12 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   store8(dst + lane * 8, v);
 }
 
-int launch_post_proj(const PostParams& P, cudaStream_t st) {
+// Grid rows 0-2 hold the SWA head slots (q, k, v), rows 3-5 the RMA ones
+// (q, k and v with the pending append); with the RMA switched off only the
+// first three run.
+int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st) {
   if (P.nq <= 0) return ER_OK;
-  k_post_proj<<<dim3(P.nq, 6), 256, 0, st>>>(P);
+  k_post_proj<<<dim3(P.nq, rma_off ? 3 : 6), 256, 0, st>>>(P);
   count_launches(1);
   return launch_status();
 }

@@ -51,6 +51,7 @@ struct AttendParams {
   int direct;
   float *o_swa, *o_rma;  // FP32 [nq][16][256] (standalone read), or
   uint16_t* o_sum;       // BF16 [nq][4096] = bf16(o_swa + o_rma) (layer path)
+  int rma_off;           // the RMA read sees no records (o_rma = 0)
   int32_t* err;
 };
 

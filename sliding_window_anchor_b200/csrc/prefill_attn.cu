@@ -427,14 +427,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
 // o_sum[t][h*256 + d] = bf16(o_swa + o_rma), each branch the merge of its
 // NSPLIT partial reads weighted by l·2^(m - M); 8 values per thread.
 __global__ void k_prefill_combine(const float* __restrict__ out, const float2* __restrict__ ml,
-                                  int T, uint16_t* __restrict__ o_sum) {
+                                  int T, int nbr, uint16_t* __restrict__ o_sum) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * (OIN / 8)) return;
   const int row = idx / (D / 8);  // token * 16 + head
   const int d0 = (idx % (D / 8)) * 8;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int br = 0; br < 2; ++br) {
+  for (int br = 0; br < nbr; ++br) {
     float2 v[NSPLIT];
     float M = -INFINITY;
 #pragma unroll
@@ -483,7 +482,7 @@ size_t prefill_out_floats(int T) {
 
 int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const uint16_t* q_swa,
                           const uint16_t* q_rma, const uint16_t* chunk_k,
-                          const uint16_t* chunk_v, float* out, uint16_t* o_sum,
+                          const uint16_t* chunk_v, float* out, uint16_t* o_sum, bool rma_off,
                           cudaStream_t stream) {
   if (T < 1 || T > PEND) return ER_EINVAL;
   int dev = 0;
@@ -521,13 +520,15 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   P.out = out;
   P.ml = reinterpret_cast<float2*>(out + (size_t)2 * NSPLIT * T * OIN);
   P.err = st->dev_error;
-  const dim3 grid((T + PQ_TOK - 1) / PQ_TOK, NG, 2 * NSPLIT);
+  // branch 0 (SWA) and, unless the RMA is switched off, branch 1
+  const int nbr = rma_off ? 1 : 2;
+  const dim3 grid((T + PQ_TOK - 1) / PQ_TOK, NG, nbr * NSPLIT);
   std::pair<cudaEvent_t, cudaEvent_t> ev;
   const bool timed = profile_begin(stream, &ev);
   k_prefill_attn<<<grid, PF_THREADS, PF_SMEM, stream>>>(P);
   if (timed) profile_end(stream, ev);
   const int nv = T * (OIN / 8);
-  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, P.ml, T, o_sum);
+  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, P.ml, T, nbr, o_sum);
   count_launches(2);
   return launch_status();
 }

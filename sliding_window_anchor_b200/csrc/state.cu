@@ -79,9 +79,10 @@ __global__ void k_state_init(int32_t* meta, const int32_t* seq_ids, int n, int s
 }
 
 // End of a step of T tokens: the position moves on; a block that reached 256
-// was committed by every layer during the step and empties.
+// was committed by every layer during the step and empties.  With the RMA
+// switched off only the position moves.
 __global__ void k_advance(int32_t* meta, const int32_t* seq_ids, int n, int T, int s_max,
-                          int32_t* err) {
+                          int rma_off, int32_t* err) {
   int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b >= n) return;
   int s = seq_ids[b];
@@ -90,6 +91,10 @@ __global__ void k_advance(int32_t* meta, const int32_t* seq_ids, int n, int T, i
     return;
   }
   int32_t* m = meta + (size_t)s * 4;
+  if (rma_off) {
+    m[0] += T;
+    return;
+  }
   int pend = m[1] + T;
   if (pend > PEND) {
     set_dev_error(err, ER_ECAPACITY);
@@ -189,14 +194,20 @@ int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stre
   return launch_status();
 }
 
-int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
-               er_stream_t stream) {
+int er_advance_ex(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
+                  uint32_t flags, er_stream_t stream) {
   if (!st || !st->meta || (n > 0 && !seq_ids) || n < 0 || T < 1 || T > PEND) return ER_EINVAL;
+  if (flags & ~ER_FLAG_RMA_OFF) return ER_EINVAL;
   if (n == 0) return ER_OK;
-  k_advance<<<(n + 127) / 128, 128, 0, (cudaStream_t)stream>>>(st->meta, seq_ids, n, T,
-                                                               st->s_max, st->dev_error);
+  k_advance<<<(n + 127) / 128, 128, 0, (cudaStream_t)stream>>>(
+      st->meta, seq_ids, n, T, st->s_max, (flags & ER_FLAG_RMA_OFF) ? 1 : 0, st->dev_error);
   count_launches(1);
   return launch_status();
+}
+
+int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
+               er_stream_t stream) {
+  return er_advance_ex(st, seq_ids, n, T, 0u, stream);
 }
 
 int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream) {

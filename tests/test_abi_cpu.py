@@ -119,3 +119,14 @@ def test_host_validation_rejects_before_enqueue(L):
     assert L.er_qk_norm_rope(nul, nul, 0, nul, nul, nul) == 0
     assert L.er_launch_count() == before
     assert L.er_error_string(-2) == b"capacity exceeded"
+    # flags: the RMA switch is the only defined bit; others are refused before anything else
+    before = L.er_launch_count()
+    assert L.er_swa_rma_decode_ex(ctypes.byref(st), ctypes.byref(w), 0, nul, 0, nul, nul, nul,
+                                  0, 1, nul) == 0
+    assert L.er_swa_rma_decode_ex(ctypes.byref(st), ctypes.byref(w), 0, nul, 0, nul, nul, nul,
+                                  0, 2, nul) == -1
+    assert L.er_advance_ex(ctypes.byref(st), nul, 0, 1, 1, nul) == 0
+    assert L.er_advance_ex(ctypes.byref(st), nul, 0, 1, 4, nul) == -1
+    assert L.er_swa_rma_prefill_chunk_ex(ctypes.byref(st), ctypes.byref(w), 0, 0, nul, 16, nul,
+                                         nul, 0, 8, nul) == -1
+    assert L.er_launch_count() == before

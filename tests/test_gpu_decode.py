@@ -220,3 +220,70 @@ def test_out_of_range_sequence_is_recorded_not_faulted(sab):
     st.meta[1, 1] = 256
     sab.swa_rma_decode(st, gw, 0, [0, 1], x)
     assert sab.last_device_error(st) == -2
+
+
+RMA_ARRAYS = ("bank_k", "bank_v", "pend_k", "pend_v", "bank_score", "pend_score", "bank_pos",
+              "pend_pos")
+
+
+def test_rma_off_decode_matches_oracle_and_freezes_the_memory(sab):
+    """The pages' ablation (ER_FLAG_RMA_OFF): o_rma = 0, no score, append or commit; the
+    anchor memory and its counters stay bit-identical while the window moves on."""
+    seed, L, B, t0 = 61, 1, 8, 32768
+    gw, gdict = H.gpu_weights(seed, 0)
+    ow, wdict = H.oracle_weights(seed, 0)
+    fills = [250, 255, 0, 17, 128, 254, 3, 200]  # several would commit within 8 steps
+    st = sab.State(B, L)
+    H.seed_gpu_state(st, L, t0, fills, seed, [gdict])
+    before = {n: getattr(st, n).clone() for n in RMA_ARRAYS}
+    meta0 = st.meta.clone()
+    ids = torch.arange(B, dtype=torch.int32, device="cuda")
+    steps = 8
+    gouts = []
+    for step in range(steps):
+        x = wl.make_x(seed, 0, step, range(B), device="cuda")
+        gouts.append(sab.swa_rma_decode(st, gw, 0, ids, x, rma_off=True).cpu())
+        sab.advance(st, ids, rma_off=True)
+    assert sab.last_device_error(st) == 0
+    for n in RMA_ARRAYS:
+        assert torch.equal(getattr(st, n), before[n]), n
+    meta = st.meta.cpu()
+    assert torch.equal(meta[:, 0], meta0[:, 0].cpu() + steps)
+    assert torch.equal(meta[:, 1:], meta0[:, 1:].cpu())
+    for gseq in (1, 3):  # one whose block is full, one that would not commit
+        ost = oracle.OracleState(1, L)
+        H.seed_oracle_state(ost, [gseq], L, t0, [fills[gseq]], seed, [wdict])
+        for step in range(steps):
+            ref = ost.decode_layer(ow, 0, 0, wl.make_x(seed, 0, step, [gseq])[0], rma_off=True)
+            ost.advance(0, rma_off=True)
+            got = gouts[step][gseq]
+            assert H.tol_ok(got, ref), (gseq, step, H.max_err(got, ref))
+
+
+def test_rma_off_prefill_matches_oracle_and_decode(sab):
+    seed, L, t0 = 62, 1, 4096
+    gw, gdict = H.gpu_weights(seed, 0)
+    ow, wdict = H.oracle_weights(seed, 0)
+    st = sab.State(2, L)
+    H.seed_gpu_state(st, L, t0, [60, 60], seed, [gdict])
+    ost = oracle.OracleState(1, L)
+    H.seed_oracle_state(ost, [0], L, t0, [60], seed, [wdict])
+    for n in oracle.OracleState.ARRAYS:
+        getattr(st, n)[1].copy_(getattr(st, n)[0])
+    before = {n: getattr(st, n).clone() for n in RMA_ARRAYS}
+    T = 100
+    x = wl.make_x(seed, 0, 0, range(T), big_every=4096, first_pos=t0)
+    got = sab.swa_rma_prefill_chunk(st, gw, 0, 0, x.cuda(), rma_off=True).cpu()
+    sab.advance(st, [0], T, rma_off=True)
+    dec = []
+    for i in range(T):
+        dec.append(sab.swa_rma_decode(st, gw, 0, [1], x[i:i + 1].cuda(), rma_off=True))
+        sab.advance(st, [1], rma_off=True)
+    dec = torch.cat(dec).cpu()
+    ref = ost.prefill_chunk(ow, 0, 0, x, rma_off=True)
+    assert sab.last_device_error(st) == 0
+    assert H.tol_ok(got, ref), H.max_err(got, ref)
+    assert H.tol_ok(got, dec), H.max_err(got, dec)
+    for n in RMA_ARRAYS:
+        assert torch.equal(getattr(st, n), before[n]), n
+    assert st.meta[0].tolist() == [t0 + T, 60, 1024, 0]

@@ -451,6 +451,78 @@ def test_prefill_equals_token_by_token_decode():
         assert torch.equal(getattr(st_a, n), getattr(st_b, n)), n
 
 
+# ------------------------------------------------- RMA off (the pages' ablation)
+
+RMA_ARRAYS = ("bank_k", "bank_v", "pend_k", "pend_v", "bank_score", "pend_score", "bank_pos",
+              "pend_pos")
+
+
+def test_rma_off_equals_rma_on_when_every_anchor_value_is_zero():
+    # a special case that needs no flag: with zero v_rma weights and zero bank / pending
+    # V rows, every RMA read averages zeros, so o_rma = 0 exactly and both settings agree
+    _, w, st_on = _seeded(51, 3000, [100])
+    wz = dict(w)
+    wz["w_qkv"] = w["w_qkv"].clone()
+    wz["w_qkv"][11264:12288] = 0
+    ow = oracle.OracleWeights(wz["w_qkv"], wz["w_o"], wz["q_norm_swa"], wz["k_norm_swa"],
+                              wz["q_norm_rma"], wz["k_norm_rma"], wz["w1"], wz["w2"])
+    st_on.bank_v.zero_()
+    st_on.pend_v.zero_()
+    st_off = st_on.clone()
+    for step in range(3):
+        x = wl.make_x(51, 0, step, [0])[0]
+        out_on, _, o_rma = st_on.decode_layer(ow, 0, 0, x, want_branches=True)
+        out_off = st_off.decode_layer(ow, 0, 0, x, rma_off=True)
+        st_on.advance(0)
+        st_off.advance(0, rma_off=True)
+        assert bool((o_rma == 0).all())
+        assert torch.equal(out_on, out_off), step
+
+
+def test_rma_off_output_is_the_swa_branch_alone_and_memory_stays():
+    ow, w, st = _seeded(52, 5000, [200])
+    other = st.clone()
+    # different anchor memory in the second copy: K, V and scores
+    other.bank_k.copy_(torch.flip(other.bank_k, dims=[3]))
+    other.pend_v.mul_(-1)
+    other.bank_score.add_(1.5)
+    before = {n: getattr(st, n).clone() for n in RMA_ARRAYS}
+    ref = st.clone()
+    for step in range(3):
+        x = wl.make_x(52, 0, step, [0])[0]
+        out, o_swa, o_rma = st.decode_layer(ow, 0, 0, x, want_branches=True, rma_off=True)
+        out_other = other.decode_layer(ow, 0, 0, x, rma_off=True)
+        _, o_swa_on, _ = ref.decode_layer(ow, 0, 0, x, want_branches=True)
+        for s_ in (st, other):
+            s_.advance(0, rma_off=True)
+        ref.advance(0)
+        assert bool((o_rma == 0).all())
+        assert torch.equal(o_swa, o_swa_on)  # the SWA branch does not see the RMA switch
+        o = bf16_exact(o_swa.reshape(-1).numpy())
+        assert torch.equal(out, oracle.linear_bf16(w["w_o"], o))
+        assert torch.equal(out, out_other)  # the anchor memory is not read
+    for n in RMA_ARRAYS:
+        assert torch.equal(getattr(st, n), before[n]), n  # ... nor written
+    assert st.meta[0].tolist() == [5003, 200, 1024, 0]  # only the position moves
+    assert torch.equal(st.win_k, other.win_k) and torch.equal(st.win_v, other.win_v)
+
+
+def test_rma_off_prefill_equals_token_by_token_decode():
+    ow, w, st_a = _seeded(53, 4096, [40])
+    st_b = st_a.clone()
+    T = 17
+    xs = wl.make_x(53, 0, 0, range(T))
+    out_chunk = st_a.prefill_chunk(ow, 0, 0, xs, rma_off=True)
+    st_a.advance(0, T, rma_off=True)
+    outs = []
+    for i in range(T):
+        outs.append(st_b.decode_layer(ow, 0, 0, xs[i], rma_off=True))
+        st_b.advance(0, rma_off=True)
+    assert torch.equal(out_chunk, torch.stack(outs))
+    for n in oracle.OracleState.ARRAYS:
+        assert torch.equal(getattr(st_a, n), getattr(st_b, n)), n
+
+
 def test_full_bank_ignores_low_scoring_tail():
     # after the bank is full, extending the stream with tokens that score below every anchor
     # leaves the bank bit-identical whatever the stream length
