@@ -55,6 +55,8 @@ def parse():
                          "sequences; score: the scorer on --batch tokens; prefill: "
                          "--prefill-chunks chunks of one layer (profiling drivers)")
     ap.add_argument("--batch", type=int, default=256)
+    ap.add_argument("--sweep", action="store_true",
+                    help="layer-level batch sweep B = 1..512 (one JSON line per batch size)")
     return ap.parse_args()
 
 
@@ -508,6 +510,104 @@ def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2,
                 "note": "same chunks replayed from one captured CUDA graph per chunk"}}
 
 
+SWEEP_BATCHES = (1, 2, 4, 8, 16, 32, 64, 96, 128, 160, 192, 224, 256, 288, 320, 352, 384, 448,
+                 512)
+
+
+def batch_sweep(dev, batches=SWEEP_BATCHES, steps: int = 32, warmup: int = 4):
+    """One SWA∥RMA layer's decode step (a1–a7 + advance) at each batch size, on
+    the decode workload (t0 = 32768, window and bank full, pending fill
+    U{0..255}).  Throughput from the steps replayed out of CUDA graphs (one per
+    input buffer); the read kernel's GB/s from an eager pass with its launches
+    timed by CUDA events, over the algorithmic bytes of the rows it must read."""
+    import torch
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+    seed = wl.seed_of(3)
+    bmax = max(batches)
+    w = sab.LayerWeights.from_dict(wl.make_weights(seed, 0, device=dev))
+    st = sab.State(bmax, 1, device=dev)
+
+    def normrope(x, g, pos):
+        return sab.qk_norm_rope(x.contiguous(), g, pos.to(torch.int32).contiguous())
+
+    fills = wl.seed_state(st.arrays(), range(bmax), 1, T0, "uniform", seed, [w.t], normrope,
+                          device=dev).cpu().tolist()
+    done = [0] * bmax  # steps each sequence has taken
+    hbm, kind = peaks()
+    stream = torch.cuda.current_stream(dev)
+    n_x = 8
+    rows = []
+    for B in batches:
+        ids = torch.arange(B, dtype=torch.int32, device=dev)
+        ws = torch.empty(sab.decode_workspace_bytes(B), dtype=torch.uint8, device=dev)
+        xs = [wl.make_x(seed, 0, s, range(B), device=dev) for s in range(n_x)]
+        out = torch.empty(B, 2560, dtype=torch.bfloat16, device=dev)
+
+        def step(s):
+            sab.swa_rma_decode(st, w, 0, ids, xs[s % n_x], out=out, ws=ws)
+            sab.advance(st, ids)
+
+        def took(k):
+            for b in range(B):
+                done[b] += k
+
+        for s in range(warmup):
+            step(s)
+        took(warmup)
+        # eager pass: the read kernel's launches timed
+        alg = 0
+        for s in range(steps):
+            for b in range(B):
+                p = (fills[b] + done[b] + s) % 256
+                alg += 4 * ((1024 + 1024 + p + 1) * ROW + 2 * 4 * 512 + 2 * 4 * 1024)
+        torch.cuda.synchronize(dev)
+        sab.profile_read(reset=True)
+        sab.profile_enable(True)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(steps):
+            step(s)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        sab.profile_enable(False)
+        a_ms, a_n = sab.profile_read(reset=True)
+        eager_ms = e0.elapsed_time(e1)
+        took(steps)
+        # graph pass
+        stream_g = torch.cuda.Stream(dev)
+        graphs = []
+        for s in range(n_x):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream_g):
+                step(s)
+            graphs.append(g)
+        for s in range(warmup):
+            graphs[s % n_x].replay()
+        took(warmup)
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for s in range(steps):
+            graphs[s % n_x].replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        took(steps)
+        del graphs
+        if sab.last_device_error(st) != 0:
+            raise RuntimeError(f"device error in the sweep at B={B}")
+        g_ms = g0.elapsed_time(g1)
+        attend_gbs = (alg / steps) / (a_ms / a_n / 1e3) / 1e9 if a_n else None
+        row = {"workload": "decode_layer_t32768", "B": B, "layers": 1, "steps": steps,
+               "tok_per_s": B * steps / (g_ms / 1e3), "ms_per_step": g_ms / steps,
+               "eager_ms_per_step": eager_ms / steps,
+               "attend_ms": a_ms / a_n if a_n else None, "attend_gbs": attend_gbs,
+               "attend_frac": attend_gbs / hbm if attend_gbs else None, "peak_kind": kind}
+        print(json.dumps(row), flush=True)
+        rows.append(row)
+    return rows
+
+
 def single_kernel(args):
     """Profiling driver: one kernel alone on a --batch workload, three launches."""
     import torch
@@ -636,6 +736,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         reference_arm(args, rank, world)
+        return
+    if args.sweep:
+        import torch
+        batch_sweep(torch.device("cuda", 0))
         return
     if args.kernel != "step":
         single_kernel(args)
