@@ -20,6 +20,9 @@
 //     (ascending) and the pending winners (ascending);
 //  4. each warp moves winners' K and V rows (512 B each, 16 B per lane) into
 //     their target slots, with the score and position, four rows in flight.
+// Launches with few merges run as clusters of 8 CTAs that repeat steps 1-3
+// and split step 4 (a cluster barrier keeps every key read ahead of the first
+// bank write).
 // Surviving anchors are not touched, so the write traffic is only the moved
 // records.
 #include "common.cuh"
@@ -33,6 +36,7 @@ constexpr int CT = 256;   // threads per commit block
 constexpr int EPT = NSORT / CT;  // 8 keys per thread
 constexpr int CW = CT / 32;      // warps per block
 constexpr int SPB = 32;   // most sequences one block looks after (decode path)
+constexpr int REPL = 8;   // CTAs per cluster sharing the moves of a few merges
 
 __device__ __forceinline__ uint32_t ordered_score(float s) {
   uint32_t u = __float_as_uint(s);
@@ -208,6 +212,23 @@ __device__ void radix_select(const uint64_t (&key)[5], int K, int* hist, int* wa
   *out_shift = shift;
 }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+
+// Every thread of every CTA of the cluster (a cluster of one is the block).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
   __shared__ uint64_t skey[NSORT];
   __shared__ uint16_t ssrc[NSORT];
@@ -222,10 +243,14 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
   const int l = P.layer0 + blockIdx.y / NG;
   const int g = blockIdx.y % NG;
   const int tid = threadIdx.x;
-  // each block owns a run of `per_block` listed sequences; their metadata is read
+  // the CTAs of a cluster work on the same merges: each computes the same kept set
+  // and move list, and moves its share of the winners (rank r takes winners
+  // r*8+warp, r*8+warp + 8*ranks, ...)
+  const int rank = (int)cluster_ctarank(), nranks = (int)cluster_nctarank();
+  // each cluster owns a run of `per_block` listed sequences; their metadata is read
   // in one parallel load, so the (many) sequences with nothing to commit cost
   // no serial global-memory latency
-  const int b0 = blockIdx.x * P.per_block;
+  const int b0 = (blockIdx.x / nranks) * P.per_block;
   const int nb = min(P.per_block, P.n - b0);
   if (tid < nb) {
     const int seq = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b0 + tid];
@@ -296,7 +321,7 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
 #pragma unroll
       for (int e = 0; e < EPT; ++e)
         if (tid * EPT + e < K) flag[src[e]] = 1;
-      if (tid * EPT < BANK) {
+      if (rank == 0 && tid * EPT < BANK) {
         int32_t* kp = P.kept + (((size_t)b * P.nlayers + (l - P.layer0)) * NG + g) * BANK;
 #pragma unroll
         for (int e = 0; e < EPT; ++e) {
@@ -333,16 +358,19 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
     }
     __syncthreads();
 
+    // no CTA of the cluster writes the bank before every CTA has read this merge's keys
+    cluster_sync_all();
     // move rows: one warp per winner, 16 bytes per lane per row; MV winners per warp
     // in flight (every load issued before the first store)
     constexpr int MV = 4;
     const int warp = tid >> 5, lane = tid & 31;
-    for (int w0 = warp; w0 < total_win; w0 += MV * CW) {
+    const int movers = CW * nranks;
+    for (int w0 = rank * CW + warp; w0 < total_win; w0 += MV * movers) {
       uint4 kr[MV], vr[MV];
       int src[MV];
 #pragma unroll
       for (int q = 0; q < MV; ++q) {
-        const int w = w0 + q * CW;
+        const int w = w0 + q * movers;
         src[q] = w < total_win ? (int)move_src[w] : -1;
         kr[q] = vr[q] = make_uint4(0, 0, 0, 0);
         if (src[q] >= 0) {
@@ -353,7 +381,7 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
 #pragma unroll
       for (int q = 0; q < MV; ++q) {
         if (src[q] < 0) continue;
-        const int dst = move_dst[w0 + q * CW];
+        const int dst = move_dst[w0 + q * movers];
         reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + dst) * D)[lane] = kr[q];
         reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + dst) * D)[lane] = vr[q];
         if (lane == 0) {
@@ -376,12 +404,28 @@ __global__ void k_commit_finish(int32_t* meta, const int32_t* seq_ids, int n, in
   m[1] = 0;
 }
 
+// Device-gated commits (a layer call: few merges per launch) and small explicit
+// ones run as clusters of REPL CTAs that split each merge's row moves; large
+// explicit batches (every block busy) run one CTA per merge.
 int launch_commit(const CommitParams& P, cudaStream_t st) {
   if (P.n <= 0) return ER_OK;
   CommitParams Q = P;
   Q.per_block = P.only_if_full ? SPB : 1;
-  const int gx = (P.n + Q.per_block - 1) / Q.per_block;
-  k_commit<<<dim3(gx, P.nlayers * NG), CT, 0, st>>>(Q);
+  const int runs = (P.n + Q.per_block - 1) / Q.per_block;
+  const int repl = (P.only_if_full || P.n * P.nlayers <= 16) ? REPL : 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(runs * repl, P.nlayers * NG);
+  cfg.blockDim = dim3(CT);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = repl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_commit, Q) != cudaSuccess) return ER_ECUDA;
   count_launches(1);
   return launch_status();
 }
