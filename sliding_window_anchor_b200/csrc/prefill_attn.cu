@@ -12,32 +12,38 @@
 //   RMA: the c committed anchors and pending records 0 .. p0+i (the chunk's
 //        candidates were appended at p0 .. p0+T-1 before the reads).
 //
-// One CTA per (query tile, KV group, branch, split); a query tile is 32 tokens x the
-// group's 4 heads = 128 rows, the M of a tcgen05 MMA.  Keys stream in tiles of
-// 64 rows aligned to 64-slot boundaries of the ring, the chunk, the bank or the
-// pending block (so a TMA box never wraps); rows a query may not see are
-// masked in the softmax.
-//   warp 4    : TMA — Q once (four 64-dim slices, 4-D map picking the group's
-//               heads out of [T][16][256]), then K tiles (3 stages);
-//   warp 6    : TMA — V tiles (2 stages);
-//   warp 5    : TMEM owner (512 columns: O 0..255, two S buffers of 64 FP32
-//               columns, two P buffers of 32 columns of BF16 pairs) and
-//               MMA issuer: S_j = Q·K_jᵀ (M=128, N=64, K=256), then
-//               O += P_{j-1}·V_{j-1} (M=128, N=256, K=64, P read from TMEM,
-//               V read MN-major),
-//               so the tensor cores compute S_{j+1} while warps 0-3 work on
-//               the softmax of S_j;
-//   warps 0-3 : one thread per query row: S row from TMEM, mask, online
-//               softmax in base 2, P = exp2(s - m) rounded to BF16 and
-//               stored back to TMEM (the A operand of the PV MMA).
-//               The running maximum is raised only when a tile's maximum
-//               exceeds it by more than 2^8; then the row of O is rescaled in
-//               TMEM (after the previous PV has completed).  At the end O / l
-//               and (m, l) go out in FP32.
-// An item's key tiles are split over NSPLIT CTAs (so a 256-token chunk fills
-// 128 SMs); a second kernel merges the splits of each branch by their (m, l),
-// adds the two branches and rounds to BF16 for o_proj.
-// Every wait is bounded (≈2 s) and records ER_ETIMEOUT instead of hanging.
+// Work item = (64 tokens x the group's 4 heads = 256 query rows, KV group,
+// branch, split of the key tiles).  An item runs on a CTA pair (a 2-CTA
+// cluster) whose tensor-core MMAs span both SMs (tcgen05 cta_group::2): each
+// CTA keeps 128 query rows (its 32 tokens), their S, P and O in its own TMEM,
+// and fetches HALF of every key tile — 64 of its 128 keys, 128 of V's 256
+// dims — so the pair reads each K/V byte once for 256 query rows (one SM's
+// TMA engine delivers ~40 B per cycle; a whole tile per 128 rows left the
+// loop waiting on it).  Keys stream in tiles of 128 rows aligned to 128-slot
+// boundaries of the ring, the chunk, the bank or the pending block (so a TMA
+// box never wraps); rows a query may not see are masked in the softmax.
+//   warp 4    : TMA — Q once (a 4-D map picks the group's heads out of
+//               [T][16][256]), then this CTA's K halves (2 stages);
+//   warp 6    : TMA — this CTA's V halves (2 stages);
+//   warp 5    : TMEM (512 columns in both CTAs: O 0..255, two S buffers of 128
+//               FP32 columns; a tile's P, as BF16 pairs, overwrites the first
+//               half of its S buffer); in the even CTA one thread issues
+//               S = Q·Kᵀ (M=256, N=128, K=256) and, one tile behind,
+//               O += P·V (M=256, N=256, K=128, P read from TMEM, V MN-major),
+//               and commits each to both CTAs;
+//   warps 0-3 : one thread per query row: S from TMEM, mask, online softmax
+//               in base 2, P = exp2(s - m) rounded to BF16 and stored back to
+//               TMEM.  The running maximum is raised only when a tile's
+//               maximum exceeds it by more than 2^8; then the row of O is
+//               rescaled in TMEM (after the previous PV has completed).  At the
+//               end O / l and (m, l) go out in FP32 through a staging tile.
+// Both CTAs' loads count on the even CTA's barriers; each softmax warp of
+// both CTAs arrives (once per tile) on the even CTA's P-ready barrier.  No copy is
+// multicast.  An item's key tiles are split over NSPLIT pairs; a second
+// kernel merges the splits of each branch by their (m, l), adds the two
+// branches and rounds to BF16 for o_proj.
+// Every mbarrier wait is bounded (≈2 s) and records ER_ETIMEOUT instead of
+// hanging.
 #include <math.h>
 
 #include <mutex>
@@ -53,19 +59,27 @@ void profile_end(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t> ev);
 
 namespace {
 
-constexpr int PQ_TOK = 32;               // tokens per query tile
-constexpr int PM = 128;                  // query rows per tile (MMA M)
-constexpr int PKT = 64;                  // keys per key tile
-constexpr int SLICE = PM * 128;          // 128 rows x 64 BF16 (one Q slice, one P buffer)
-constexpr int KBOX = PKT * 128;          // one 64-row x 64-dim box, 8 KB
-constexpr int KTILE = 4 * KBOX;          // 64 keys x 256 dims, 32 KB
-constexpr int MAX_TILES = WIN / PKT + PEND / PKT;  // 20
+constexpr int PQ_TOK = 32;               // tokens per CTA
+constexpr int PAIR_TOK = 2 * PQ_TOK;     // tokens per CTA pair
+constexpr int PM = 128;                  // query rows per CTA (half the MMA's M)
+constexpr int PKT = 128;                 // keys per key tile
+constexpr int KH = PKT / 2;              // keys of a tile each CTA holds
+constexpr int SLICE = PM * 128;          // 128 rows x 64 BF16: one Q slice
+constexpr int KSL = KH * 128;            // 64 keys x 64 dims: one K slice, 8 KB
+constexpr int KHALF = 4 * KSL;           // this CTA's half of a K tile, 32 KB
+constexpr int VSL = PKT * 128;           // 128 keys x 64 dims: one V slice, 16 KB
+constexpr int VHALF = 2 * VSL;           // this CTA's half of a V tile (128 dims), 32 KB
+constexpr int KST = 2, VST = 2;          // stages
+constexpr int MAX_TILES = WIN / PKT + PEND / PKT;  // 10
 constexpr int PF_THREADS = 224;
-constexpr int KST = 3;                   // K stages
-constexpr uint32_t TMEM_COLS = 512, TM_O = 0, TM_S = 256, TM_P = 384;
+// TMEM: O in columns 0..255, two S buffers of 128 FP32 columns; a tile's P
+// (128 keys as 64 columns of BF16 pairs) overwrites the first half of its own S
+// buffer once the softmax has read it
+constexpr uint32_t TMEM_COLS = 512, TM_O = 0, TM_S = 256;
 constexpr float SCALE_LOG2 = 1.4426950408889634f / 16.0f;  // log2(e) / sqrt(256)
 constexpr float RESCALE_AT = 8.0f;
-constexpr int NSPLIT = 2;                // key tiles of an item split over this many CTAs
+constexpr int NSPLIT = 2;                // key tiles of an item split over this many pairs
+constexpr uint64_t kDrainNs = 200000;    // after a timeout: let copies in flight land
 
 enum : int { KIND_RING = 0, KIND_CHUNK = 1, KIND_BANK = 2, KIND_PEND = 3 };
 
@@ -75,25 +89,26 @@ struct PTile {
 };
 
 struct __align__(1024) PrefillSmem {
-  unsigned char q[4][SLICE];   // Q: 4 slices of 64 dims (64 KB)
-  unsigned char k[KST][KTILE];  // K stages (96 KB)
-  unsigned char v[2][KTILE];    // V stages (64 KB)
-  uint64_t q_full;
-  uint64_t k_full[KST], k_empty[KST], v_full[2];
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
-  uint64_t mma_done;
+  unsigned char q[4][SLICE];     // this CTA's 128 query rows, 4 slices of 64 dims (64 KB)
+  unsigned char k[KST][KHALF];   // K halves (64 KB)
+  unsigned char v[VST][VHALF];   // V halves (32 KB)
+  // used in the even CTA: both CTAs' copies and softmax warps arrive here
+  uint64_t q_full, k_full[KST], v_full[VST], p_full[2], mma_done;
+  // used in both CTAs: the even CTA's MMAs commit here
+  uint64_t k_empty[KST], s_full[2], pv_done[2];
   uint32_t tmem_base;
-  int ntiles, meta_ok;
+  int ntiles, meta_ok, failed;
   PTile tiles[MAX_TILES];
 };
 
 constexpr size_t PF_SMEM = sizeof(PrefillSmem) + 1024;
 static_assert(PF_SMEM <= 232448, "shared memory above the per-block limit");
+static_assert(4 * 32 * 32 * 4 <= KHALF, "epilogue staging must fit a K stage");
 
 struct PrefillParams {
   CUtensorMap tmap_q[2];  // q_swa, q_rma: {256, 4 heads, 4 groups, T}, box {64, 4, 1, 32}
-  CUtensorMap tmap_k[4];  // ring, chunk, bank, pending K rows; box 64 x 64
-  CUtensorMap tmap_v[4];
+  CUtensorMap tmap_k[4];  // ring, chunk, bank, pending K rows; box 64 dims x 64 rows
+  CUtensorMap tmap_v[4];  // the same V rows; box 64 dims x 128 rows
   const int32_t* meta;
   int seq, s_max, L, layer, T;
   float* out;   // FP32 [2 branches][NSPLIT][T][16][256]: each split's O / l
@@ -103,17 +118,17 @@ struct PrefillParams {
 
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
-// The key tiles one work item reads, in the order they are streamed.
+// The key tiles one work item (tokens i0 .. i0+63) reads, in streaming order.
 __device__ int build_tiles(PTile* tl, int br, int g, int i0, int T, int t0, int p0, int c,
                            int gi) {
-  const int i_last = min(T, i0 + PQ_TOK) - 1;
+  const int i_last = min(T, i0 + PAIR_TOK) - 1;
   int n = 0;
   if (br == 0) {
-    // ring tiles holding at least one position the item's first query still sees
+    // ring tiles holding at least one position the item's first query still sees;
+    // slot w = t0 mod 1024 holds the oldest position t0-1024, slot w-1 the newest
+    // t0-1; elsewhere positions rise by one per slot
     const int lo_first = max(0, t0 + i0 - (WIN - 1));
     const int lo_last = max(0, t0 + i_last - (WIN - 1));
-    // slot w = t0 mod 1024 holds the oldest position t0-1024, slot w-1 the newest t0-1;
-    // elsewhere positions rise by one per slot
     const int w = t0 & (WIN - 1);
     for (int rt = 0; rt < WIN / PKT && t0 > 0; ++rt) {
       const int a = rt * PKT, z = a + PKT - 1;
@@ -141,13 +156,16 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__global__ void __launch_bounds__(PF_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
     k_prefill_attn(const __grid_constant__ PrefillParams P) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   PrefillSmem& S = *reinterpret_cast<PrefillSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i0 = blockIdx.x * PQ_TOK, g = blockIdx.y;
+  const uint32_t rank = tc::cluster_rank();  // 0: issues the MMAs; 1: its peer
+  const uint32_t lead = rank & ~1u, peer = rank ^ 1u;
+  const int i0 = (blockIdx.x >> 1) * PAIR_TOK;  // the pair's first token
+  const int g = blockIdx.y;
   const int br = blockIdx.z / NSPLIT, split = blockIdx.z % NSPLIT;
   const int T = P.T;
   const int t0 = P.meta[P.seq * 4 + 0];
@@ -156,16 +174,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   const int gi = (int)grp(P.seq, P.layer, g, P.L);
 
   if (threadIdx.x == 0) {
-    mbar_init(&S.q_full, 1);
+    mbar_init(&S.q_full, 2);
     for (int b = 0; b < KST; ++b) {
-      mbar_init(&S.k_full[b], 1);
+      mbar_init(&S.k_full[b], 2);
       mbar_init(&S.k_empty[b], 1);
     }
+    for (int b = 0; b < VST; ++b) mbar_init(&S.v_full[b], 2);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&S.v_full[b], 1);
       mbar_init(&S.s_full[b], 1);
-      mbar_init(&S.s_empty[b], 128);
-      mbar_init(&S.p_full[b], 128);
+      mbar_init(&S.p_full[b], 2 * 4);  // one arrival per softmax warp of each CTA
       mbar_init(&S.pv_done[b], 1);
     }
     mbar_init(&S.mma_done, 1);
@@ -173,75 +190,76 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
     const bool meta_ok = t0 >= 0 && p0 >= 0 && c >= 0 && c <= BANK && p0 + T <= PEND;
     int nt = 0;
     if (meta_ok) {
-      // this CTA's contiguous share of the item's tiles
+      // this pair's contiguous share of the item's tiles (both CTAs build the same list)
       const int all = build_tiles(S.tiles, br, g, i0, T, t0, p0, c, gi);
       const int tb = all * split / NSPLIT, te = all * (split + 1) / NSPLIT;
       for (int j = tb; j < te; ++j) S.tiles[j - tb] = S.tiles[j];
       nt = te - tb;
-    } else {
+    } else if (rank == 0) {
       set_dev_error(P.err, ER_ECAPACITY);
     }
     S.ntiles = nt;
     S.meta_ok = meta_ok ? 1 : 0;
+    S.failed = 0;
   }
-  if (warp == 5) tc::tmem_alloc(&S.tmem_base, TMEM_COLS);
+  if (warp == 5) tc::tmem_alloc_pair(&S.tmem_base, TMEM_COLS);
   tc::fence_before_sync();
   __syncthreads();
+  tc::cluster_sync();  // both CTAs' barriers initialised, TMEM held by both
   tc::fence_after_sync();
   const uint32_t tmem = S.tmem_base;
   const int n = S.ntiles;
 
   if (warp == 4) {
-    // ------------------------------------------------------ Q + K producer
+    // ------------------------------------------------ Q + K halves (both CTAs)
     if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(&S.q_full, 4 * SLICE);
+      tc::mbar_arrive_expect_tx_cluster(tc::map_to_rank(&S.q_full, lead), 4 * SLICE);
       for (int d = 0; d < 4; ++d)
-        tc::tma_load_4d(S.q[d], &P.tmap_q[br], 64 * d, 0, g, i0, &S.q_full);
-      int issued = 0;
+        tc::tma_load_4d_pair(S.q[d], &P.tmap_q[br], 64 * d, 0, g, i0 + PQ_TOK * (int)rank,
+                             tc::map_to_rank(&S.q_full, lead));
       for (int j = 0; j < n; ++j) {
         const int b = j % KST;
-        const uint32_t ph = (j / KST) & 1;
-        if (!mbar_wait(&S.k_empty[b], ph ^ 1, P.err)) break;
+        if (!mbar_wait(&S.k_empty[b], ((j / KST) & 1) ^ 1, P.err)) {
+          S.failed = 1;
+          break;
+        }
         const PTile tl = S.tiles[j];
-        mbar_arrive_expect_tx(&S.k_full[b], KTILE);
+        const uint32_t full = tc::map_to_rank(&S.k_full[b], lead);
+        tc::mbar_arrive_expect_tx_cluster(full, KHALF);
         for (int d = 0; d < 4; ++d)
-          tc::tma_load_2d(S.k[b] + d * KBOX, &P.tmap_k[tl.kind], 64 * d, tl.row0, &S.k_full[b]);
-        ++issued;
+          tc::tma_load_2d_pair(S.k[b] + d * KSL, &P.tmap_k[tl.kind], 64 * d,
+                               tl.row0 + KH * (int)rank, full);
       }
-      // no copy may still be landing when the block exits
-      mbar_wait(&S.q_full, 0, P.err);
-      for (int j = max(0, issued - KST); j < issued; ++j)
-        mbar_wait(&S.k_full[j % KST], (j / KST) & 1, P.err);
     }
   } else if (warp == 6) {
-    // ---------------------------------------------------------- V producer
+    // ---------------------------------------------------- V halves (both CTAs)
     if (lane == 0 && n > 0) {
-      int issued = 0;
       for (int j = 0; j < n; ++j) {
-        const int b = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&S.pv_done[b], ph ^ 1, P.err)) break;
+        const int b = j % VST;
+        if (!mbar_wait(&S.pv_done[b], ((j / VST) & 1) ^ 1, P.err)) {
+          S.failed = 1;
+          break;
+        }
         const PTile tl = S.tiles[j];
-        mbar_arrive_expect_tx(&S.v_full[b], KTILE);
-        for (int d = 0; d < 4; ++d)
-          tc::tma_load_2d(S.v[b] + d * KBOX, &P.tmap_v[tl.kind], 64 * d, tl.row0, &S.v_full[b]);
-        ++issued;
+        const uint32_t full = tc::map_to_rank(&S.v_full[b], lead);
+        tc::mbar_arrive_expect_tx_cluster(full, VHALF);
+        for (int d = 0; d < 2; ++d)
+          tc::tma_load_2d_pair(S.v[b] + d * VSL, &P.tmap_v[tl.kind], 64 * (2 * (int)rank + d),
+                               tl.row0, full);
       }
-      for (int j = max(0, issued - 2); j < issued; ++j)
-        mbar_wait(&S.v_full[j & 1], (j >> 1) & 1, P.err);
     }
   } else if (warp == 5) {
-    // ------------------------------------------------------------------ MMA
-    if (lane == 0 && n > 0) {
-      constexpr uint32_t idesc_s = tc::idesc_bf16(PM, PKT, false, false);
-      constexpr uint32_t idesc_pv = tc::idesc_bf16(PM, 256, false, true);
+    // --------------------------------------------- MMA (even CTA, one thread)
+    if (lane == 0 && n > 0 && rank == lead) {
+      constexpr uint32_t idesc_s = tc::idesc_bf16(2 * PM, PKT, false, false);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16(2 * PM, 256, false, true);
       bool ok = mbar_wait(&S.q_full, 0, P.err);
       for (int j = 0; ok && j <= n; ++j) {
         if (j < n) {
+          // S buffer b last held P_{j-2}; P·V_{j-2} was issued before this MMA, and
+          // the MMAs of one thread run in issue order
           const int b = j & 1, kb = j % KST;
-          const uint32_t ph = (j >> 1) & 1;
-          ok = mbar_wait(&S.k_full[kb], (j / KST) & 1, P.err) &&
-               mbar_wait(&S.s_empty[b], ph ^ 1, P.err);
+          ok = mbar_wait(&S.k_full[kb], (j / KST) & 1, P.err);
           if (!ok) break;
           tc::fence_after_sync();
           const uint32_t d_s = tmem + TM_S + PKT * b;
@@ -250,37 +268,42 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
             const uint64_t a =
                 tc::desc_sw128(smem_u32(S.q[kk >> 2]) + 32 * (kk & 3), 16, 1024);
             const uint64_t bd =
-                tc::desc_sw128(smem_u32(S.k[kb]) + (kk >> 2) * KBOX + 32 * (kk & 3), 16, 1024);
-            tc::mma_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
+                tc::desc_sw128(smem_u32(S.k[kb]) + (kk >> 2) * KSL + 32 * (kk & 3), 16, 1024);
+            tc::mma_pair_bf16_ss(d_s, a, bd, idesc_s, kk > 0);
           }
-          tc::commit(&S.s_full[b]);
-          tc::commit(&S.k_empty[kb]);
+          tc::commit_pair(tc::map_to_rank(&S.s_full[b], rank));
+          tc::commit_pair(tc::map_to_rank(&S.s_full[b], peer));
+          tc::commit_pair(tc::map_to_rank(&S.k_empty[kb], rank));
+          tc::commit_pair(tc::map_to_rank(&S.k_empty[kb], peer));
         }
         if (j >= 1) {
-          const int jj = j - 1, b = jj & 1;
-          const uint32_t ph = (jj >> 1) & 1;
-          ok = mbar_wait(&S.v_full[b], ph, P.err) && mbar_wait(&S.p_full[b], ph, P.err);
+          const int jj = j - 1, b = jj & 1, vb = jj % VST;
+          ok = mbar_wait(&S.v_full[vb], (jj / VST) & 1, P.err) &&
+               mbar_wait(&S.p_full[b], (jj >> 1) & 1, P.err);
           if (!ok) break;
           tc::fence_after_sync();
 #pragma unroll
           for (int kk = 0; kk < PKT / 16; ++kk) {
-            // P from TMEM (16 keys = 8 columns per step); V tile as the MN-major B
-            // operand: 64-dim blocks KBOX apart, 8-key groups 1 KB apart
-            const uint64_t bd = tc::desc_sw128(smem_u32(S.v[b]) + 2048 * kk, KBOX, 1024);
-            tc::mma_bf16_ts(tmem + TM_O, tmem + TM_P + (PKT / 2) * b + 8 * kk, bd, idesc_pv,
-                            (jj > 0 || kk > 0) ? 1u : 0u);
+            // P from TMEM (the first half of S buffer b; 16 keys = 8 columns per
+            // step); this CTA's V half as the MN-major B operand: 64-dim blocks VSL
+            // apart, 8-key groups 1 KB apart
+            const uint64_t bd = tc::desc_sw128(smem_u32(S.v[vb]) + 2048 * kk, VSL, 1024);
+            tc::mma_pair_bf16_ts(tmem + TM_O, tmem + TM_S + PKT * b + 8 * kk, bd, idesc_pv,
+                                 (jj > 0 || kk > 0) ? 1u : 0u);
           }
-          tc::commit(&S.pv_done[b]);
+          tc::commit_pair(tc::map_to_rank(&S.pv_done[b], rank));
+          tc::commit_pair(tc::map_to_rank(&S.pv_done[b], peer));
         }
       }
-      // nothing of this block's may still run on the tensor cores at exit
-      tc::commit(&S.mma_done);
+      if (!ok) S.failed = 1;
+      // nothing of the pair's may still run on the tensor cores at exit
+      tc::commit_pair(tc::map_to_rank(&S.mma_done, rank));
       mbar_wait(&S.mma_done, 0, P.err);
     }
   } else {
     // ------------------------------------------------------ softmax, rows
     const int r = threadIdx.x;  // 0..127 = TMEM lane
-    const int i = i0 + (r >> 2), hh = r & 3;
+    const int i = i0 + PQ_TOK * (int)rank + (r >> 2), hh = r & 3;
     const int t = t0 + i;
     const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
     // ring slot u = (slot - t0) mod 1024 holds position t0 - 1024 + u: visible from
@@ -296,19 +319,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
       if (!ok) break;
       tc::fence_after_sync();
       float s[PKT];
-      {
+#pragma unroll
+      for (int cb = 0; cb < PKT / 32; ++cb) {
         uint32_t raw[32];
-        tc::tmem_ld32(tmem + lane_addr + TM_S + PKT * b, raw);
+        tc::tmem_ld32(tmem + lane_addr + TM_S + PKT * b + 32 * cb, raw);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(raw[k]);
-        tc::tmem_ld32(tmem + lane_addr + TM_S + PKT * b + 32, raw);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int k = 0; k < 32; ++k) s[32 + k] = __uint_as_float(raw[k]);
+        for (int k = 0; k < 32; ++k) s[32 * cb + k] = __uint_as_float(raw[k]);
       }
-      tc::fence_before_sync();
-      mbar_arrive(&S.s_empty[b]);
 
       const PTile tl = S.tiles[j];
       if (!tl.full) {
@@ -362,22 +380,28 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         pk[k >> 1] = *reinterpret_cast<const uint32_t*>(&h2);
       }
       l += lsum;
-      // the P buffer is free once PV_{j-2} has completed
-      if (j >= 2) {
-        ok = warp_all(mbar_wait(&S.pv_done[b], ((j - 2) >> 1) & 1, P.err));
-        if (!ok) break;
+      // P_j over the first half of S_j's buffer (this thread has read all of S_j)
+      {
+        uint32_t half[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) half[e] = pk[e];
+        tc::tmem_st32(tmem + lane_addr + TM_S + PKT * b, half);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) half[e] = pk[32 + e];
+        tc::tmem_st32(tmem + lane_addr + TM_S + PKT * b + 32, half);
       }
-      tc::tmem_st32(tmem + lane_addr + TM_P + (PKT / 2) * b, pk);
       tc::tmem_wait_st();
       tc::fence_before_sync();
-      mbar_arrive(&S.p_full[b]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive_cluster(tc::map_to_rank(&S.p_full[b], lead));
     }
     if (ok) ok = warp_all(mbar_wait(&S.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, P.err));
+    if (!ok && n > 0 && lane == 0) S.failed = 1;
     // this split's partial result: O / l and (m, l); a split without keys for the
     // row (or without tiles) leaves O = 0, m = -inf, l = 0
     const size_t row = ((size_t)(br * NSPLIT + split) * T + i) * NH + 4 * g + hh;
     if (ok) {
-      // every MMA and copy of the block is complete: the K stages serve as a 4 KB
+      // every MMA and copy of the pair is complete: the K stages serve as a 4 KB
       // staging tile per warp, so each store instruction writes 4 whole 128-byte
       // row segments (row r keeps its 16-byte chunk c at position c ^ (r & 7))
       tc::fence_after_sync();
@@ -390,17 +414,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
         tc::tmem_ld32(tmem + lane_addr + TM_O + 32 * cb, o);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<float4*>(stage + lane * 32 + ((c ^ (lane & 7)) << 2)) =
-              make_float4(__uint_as_float(o[4 * c]) * inv, __uint_as_float(o[4 * c + 1]) * inv,
-                          __uint_as_float(o[4 * c + 2]) * inv,
-                          __uint_as_float(o[4 * c + 3]) * inv);
+        for (int cc = 0; cc < 8; ++cc)
+          *reinterpret_cast<float4*>(stage + lane * 32 + ((cc ^ (lane & 7)) << 2)) =
+              make_float4(__uint_as_float(o[4 * cc]) * inv, __uint_as_float(o[4 * cc + 1]) * inv,
+                          __uint_as_float(o[4 * cc + 2]) * inv,
+                          __uint_as_float(o[4 * cc + 3]) * inv);
         __syncwarp();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const int rr = 4 * k + (lane >> 3);      // row of this warp's 32
-          const int rg = 32 * warp + rr;           // row of the tile
-          const int ti = i0 + (rg >> 2);
+          const int rg = 32 * warp + rr;           // row of this CTA's 128
+          const int ti = i0 + PQ_TOK * (int)rank + (rg >> 2);
           if (ti < T) {
             const size_t grow = ((size_t)(br * NSPLIT + split) * T + ti) * NH + 4 * g + (rg & 3);
             *reinterpret_cast<float4*>(P.out + grow * D + 32 * cb + 4 * q8) =
@@ -418,9 +442,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (S.failed) {
+    // a wait gave up: give copies that may still be in flight time to land
+    const uint64_t tw = globaltimer_ns();
+    while (globaltimer_ns() - tw < kDrainNs) {
+    }
+  }
+  tc::cluster_sync();  // the pair's MMAs are done with both CTAs' memory
   if (warp == 5) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tmem, TMEM_COLS);
+    tc::tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 
@@ -508,8 +539,8 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   const uint16_t* vb[4] = {st->win_v, chunk_v, st->bank_v, st->pend_v};
   const uint64_t rows[4] = {rows_win, (uint64_t)NG * T, rows_win, rows_pend};
   for (int m = 0; m < 4; ++m)
-    ok = ok && encode_bf16_2d(&P.tmap_k[m], kb[m], D, rows[m], ROW_BYTES, 64, 64) &&
-         encode_bf16_2d(&P.tmap_v[m], vb[m], D, rows[m], ROW_BYTES, 64, 64);
+    ok = ok && encode_bf16_2d(&P.tmap_k[m], kb[m], D, rows[m], ROW_BYTES, 64, KH) &&
+         encode_bf16_2d(&P.tmap_v[m], vb[m], D, rows[m], ROW_BYTES, 64, PKT);
   if (!ok) return ER_ECUDA;
   P.meta = st->meta;
   P.seq = seq;
@@ -522,7 +553,8 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   P.err = st->dev_error;
   // branch 0 (SWA) and, unless the RMA is switched off, branch 1
   const int nbr = rma_off ? 1 : 2;
-  const dim3 grid((T + PQ_TOK - 1) / PQ_TOK, NG, nbr * NSPLIT);
+  // x: CTA pairs (2-CTA clusters), one per 64 tokens
+  const dim3 grid(2 * ((T + PAIR_TOK - 1) / PAIR_TOK), NG, nbr * NSPLIT);
   std::pair<cudaEvent_t, cudaEvent_t> ev;
   const bool timed = profile_begin(stream, &ev);
   k_prefill_attn<<<grid, PF_THREADS, PF_SMEM, stream>>>(P);
