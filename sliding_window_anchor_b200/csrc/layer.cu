@@ -6,7 +6,7 @@
 // branches, o_proj, then commit this layer for sequences whose block the token
 // filled.  A prefill chunk writes its window rows only after every token read,
 // because the chunk's early tokens still see ring positions its late tokens
-// would overwrite.
+// would overwrite (the prefill read kernel's second launch moves them).
 #include "common.cuh"
 #include "params.cuh"
 
@@ -72,21 +72,6 @@ bool weights_ok(const er_layer_weights* w) {
          (!w->w1_split || aligned16(w->w1_split));
 }
 
-// The chunk's window rows enter the ring after all of its reads.
-__global__ void k_ring_write(const uint16_t* chunk_k, const uint16_t* chunk_v, uint16_t* win_k,
-                             uint16_t* win_v, const int32_t* meta, int seq, int s_max, int L,
-                             int layer, int T) {
-  const int i = blockIdx.x, g = blockIdx.y, lane = threadIdx.x & 31, is_v = threadIdx.x >> 5;
-  if (seq < 0 || seq >= s_max) return;
-  const int t = meta[seq * 4 + 0] + i;
-  if (t < 0) return;
-  const size_t row = grp(seq, layer, g, L) * WIN + (size_t)(t % WIN);
-  const uint4* src =
-      reinterpret_cast<const uint4*>((is_v ? chunk_v : chunk_k) + ((size_t)g * T + i) * D);
-  uint4* dst = reinterpret_cast<uint4*>((is_v ? win_v : win_k) + row * D);
-  dst[lane] = src[lane];
-}
-
 int run_layer(const er_state* st, const er_layer_weights* w, int layer, const int32_t* seq_ids,
               int seq_fixed, int nq, const uint16_t* x, uint16_t* out, void* ws, size_t ws_bytes,
               uint32_t flags, cudaStream_t s) {
@@ -130,13 +115,6 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   }
   // a6: shared o_proj
   if ((rc = gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s)) != ER_OK) return rc;
-  if (prefill) {
-    k_ring_write<<<dim3(nq, NG), 64, 0, s>>>(W.chunk_k, W.chunk_v, st->win_k, st->win_v,
-                                             st->meta, seq_fixed, st->s_max, st->n_layers,
-                                             layer, nq);
-    count_launches(1);
-    if ((rc = launch_status()) != ER_OK) return rc;
-  }
   // a7: commit this layer where the block is now full (decided on the device)
   if (rma_off) return ER_OK;
   CommitParams cp{};

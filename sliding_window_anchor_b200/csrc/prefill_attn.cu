@@ -41,7 +41,8 @@
 // both CTAs arrives (once per tile) on the even CTA's P-ready barrier.  No copy is
 // multicast.  An item's key tiles are split over NSPLIT pairs; a second
 // kernel merges the splits of each branch by their (m, l), adds the two
-// branches and rounds to BF16 for o_proj.
+// branches and rounds to BF16 for o_proj, and moves the chunk's window rows
+// into the ring (after every read of the chunk).
 // Every mbarrier wait is bounded (≈2 s) and records ER_ETIMEOUT instead of
 // hanging.
 #include <math.h>
@@ -456,11 +457,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
 }
 
 // o_sum[t][h*256 + d] = bf16(o_swa + o_rma), each branch the merge of its
-// NSPLIT partial reads weighted by l·2^(m - M); 8 values per thread.
+// NSPLIT partial reads weighted by l·2^(m - M); 8 values per thread.  Every
+// read of the chunk is done by now, so the same launch also moves the chunk's
+// window rows into the ring (slot (t0 + i) mod 1024): 256 16-byte pieces per
+// token (4 groups x K, V x 32).
+struct RingWrite {
+  const uint16_t *chunk_k, *chunk_v;  // [4][T][256]
+  uint16_t *win_k, *win_v;
+  const int32_t* meta;
+  int seq, s_max, L, layer;
+};
+
 __global__ void k_prefill_combine(const float* __restrict__ out, const float2* __restrict__ ml,
-                                  int T, int nbr, uint16_t* __restrict__ o_sum) {
+                                  int T, int nbr, uint16_t* __restrict__ o_sum, RingWrite rw) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * (OIN / 8)) return;
+  {
+    const int tok = idx / (OIN / 8), piece = idx % (OIN / 8);
+    if (piece < NG * 2 * 32 && rw.seq >= 0 && rw.seq < rw.s_max) {
+      const int g = piece >> 6, is_v = (piece >> 5) & 1, lane = piece & 31;
+      const int t = rw.meta[rw.seq * 4 + 0] + tok;
+      if (t >= 0) {
+        const size_t row = grp(rw.seq, rw.layer, g, rw.L) * WIN + (size_t)(t % WIN);
+        const uint4* src =
+            reinterpret_cast<const uint4*>((is_v ? rw.chunk_v : rw.chunk_k) + ((size_t)g * T + tok) * D);
+        reinterpret_cast<uint4*>((is_v ? rw.win_v : rw.win_k) + row * D)[lane] = src[lane];
+      }
+    }
+  }
   const int row = idx / (D / 8);  // token * 16 + head
   const int d0 = (idx % (D / 8)) * 8;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -560,7 +584,17 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   k_prefill_attn<<<grid, PF_THREADS, PF_SMEM, stream>>>(P);
   if (timed) profile_end(stream, ev);
   const int nv = T * (OIN / 8);
-  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, P.ml, T, nbr, o_sum);
+  RingWrite rw;
+  rw.chunk_k = chunk_k;
+  rw.chunk_v = chunk_v;
+  rw.win_k = st->win_k;
+  rw.win_v = st->win_v;
+  rw.meta = st->meta;
+  rw.seq = seq;
+  rw.s_max = st->s_max;
+  rw.L = st->n_layers;
+  rw.layer = layer;
+  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, P.ml, T, nbr, o_sum, rw);
   count_launches(2);
   return launch_status();
 }
