@@ -9,7 +9,8 @@
 // One warp owns one 256-wide head vector, 8 BF16 values per lane (one 16-byte
 // load); lanes 0..7 hold the rotated dims and exchange pairs with xor 4.  The
 // rotation angle pos * 1e7^(-2i/64) is formed and reduced in float64 so that
-// positions up to 2^18 keep full angle accuracy; the rotation itself is fp32.
+// positions up to 2^18 keep full angle accuracy (once per token in the layer
+// kernel, shared by its head vectors); the rotation itself is fp32.
 #include "common.cuh"
 #include "params.cuh"
 
@@ -65,6 +66,30 @@ __device__ __forceinline__ void norm_rope_lane(float v[8], const uint16_t* gain,
   }
 }
 
+// The same with the 32 (cos, sin) pairs of the position already in `cs`
+// (shared memory): the unfused layer kernel forms them once per token.
+__device__ __forceinline__ void norm_rope_lane_cs(float v[8], const uint16_t* gain,
+                                                  const float2* cs, int lane) {
+  float ss = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss * (1.0f / D) + 1e-6f);
+  float g[8];
+  load8(gain + lane * 8, g);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = (v[e] * inv) * g[e];
+  float partner[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    partner[e] = __shfl_xor_sync(0xffffffffu, v[e], 4);
+    const float2 f = cs[(lane & 3) * 8 + e];
+    if (lane < 4) v[e] = v[e] * f.x - partner[e] * f.y;        // dim i:    a cos - b sin
+    else if (lane < 8) v[e] = v[e] * f.x + partner[e] * f.y;   // dim i+32: b cos + a sin
+  }
+}
+
 __global__ void k_norm_rope(const uint16_t* x, uint16_t* y, int64_t n_rows, const uint16_t* gain,
                             const int32_t* pos) {
   const int lane = threadIdx.x & 31;
@@ -82,17 +107,20 @@ __global__ void k_norm_rope(const uint16_t* x, uint16_t* y, int64_t n_rows, cons
 // Grid (nq, 6) x 256 threads: warp slot hs = 0..47 covers, per token,
 // q_swa 0..15 | k_swa 16..19 | v_swa 20..23 | q_rma 24..39 | k_rma 40..43 | v_rma 44..47.
 __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
+  __shared__ float2 s_cs[32];  // the rotation of this token's position, formed once
   const int lane = threadIdx.x & 31;
   const int hs = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int qi = blockIdx.x;
   const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
-  if (seq < 0 || seq >= P.s_max) {
+  if (seq < 0 || seq >= P.s_max) {  // the same for the whole block
     if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);
     return;
   }
   const int32_t pos0 = P.meta[seq * 4 + 0];
   const int32_t pend0 = P.meta[seq * 4 + 1];
   const int32_t t = pos0 + (P.prefill ? qi : 0);
+  if (threadIdx.x < 32) s_cs[lane] = rope_cs_lane(t, lane);
+  __syncthreads();
   const int p_idx = pend0 + (P.prefill ? qi : 0);
   const bool state_ok = p_idx >= 0 && p_idx < PEND && t >= 0;
   if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
@@ -108,7 +136,7 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
 
   float v[8];
   load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
-  if (gain) norm_rope_lane(v, gain, t, lane);
+  if (gain) norm_rope_lane_cs(v, gain, s_cs, lane);
 
   uint16_t* dst = nullptr;
   if (hs < 16) {
