@@ -753,6 +753,14 @@ def oracle_tokens_per_s(budget_s=12.0, max_threads=8):
     return sum(counts) / dt, threads, sum(counts), dt
 
 
+def workload_config(world: int, launch: str) -> dict:
+    """The workload both arms report (the reference arm's launch is the host)."""
+    return {"workload": WORKLOAD, "B": B, "layers": LAYERS, "t0": T0,
+            "pending_fill": "U{0..255}", "state_gib_per_gpu": 36.0,
+            "l2": "inputs larger than L2 (36 GiB state per GPU), no flush",
+            "parallelism": f"replicas x{world}", "launch": launch}
+
+
 def reference_arm(args, rank, world):
     if rank != 0:
         return
@@ -762,8 +770,7 @@ def reference_arm(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": B, "layers": LAYERS, "t0": T0,
-                       "pending_fill": "U{0..255}"},
+            "config": workload_config(world, "the oracle on the host cores"),
             "cpu_baseline": {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle",
                              "sample": f"{toks} whole 8-layer decode steps of {cores} sequences "
                                        f"of the workload in {dt:.1f} s"},
@@ -833,11 +840,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": head_ms / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "B": B, "layers": LAYERS, "t0": T0,
-                   "pending_fill": "U{0..255}", "state_gib_per_gpu": 36.0,
-                   "l2": "inputs larger than L2 (36 GiB state per GPU), no flush",
-                   "parallelism": f"replicas x{world}",
-                   "launch": "one CUDA graph per step" if g else "eager"},
+        "config": workload_config(world, "one CUDA graph per step" if g else "eager"),
         "commits_per_s": world * r["commits"] / secs,
         "merges_per_s": world * r["commits"] * LAYERS * 4 / secs,
         "roofline": {"bound": "hbm", "kernel": "k_attend", "achieved": achieved, "peak": hbm,
