@@ -17,6 +17,7 @@ int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int 
 int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
                  int n, float* s, void* scratch, int32_t* err, cudaStream_t st);
 size_t score_scratch_bytes(int n);
+const float* score_partials(const void* scratch, int n);
 int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
                   cudaStream_t st);
@@ -36,7 +37,6 @@ namespace {
 
 struct LayerWs {
   uint16_t* proj;
-  float* s;
   unsigned char* score_scratch;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
@@ -50,7 +50,6 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   Carver c(base);
   LayerWs w;
   w.proj = c.take<uint16_t>((size_t)nq * QKV);
-  w.s = c.take<float>((size_t)nq * NG);
   w.score_scratch = c.take<unsigned char>(score_scratch_bytes(nq));
   w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
@@ -83,12 +82,13 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   // a1: all six projections in one GEMM
   if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
   // a3: FP32 scores (not with the RMA switched off)
-  if (!rma_off && (rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, W.s, W.score_scratch,
+  // (the partial scores stay in the scratch; k_post_proj adds them)
+  if (!rma_off && (rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr, W.score_scratch,
                                      st->dev_error, s)) != ER_OK)
     return rc;
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
-  pp.proj = W.proj; pp.s = W.s; pp.nq = nq;
+  pp.proj = W.proj; pp.s_part = score_partials(W.score_scratch, nq); pp.nq = nq;
   pp.gq_swa = w->q_norm_swa; pp.gk_swa = w->k_norm_swa;
   pp.gq_rma = w->q_norm_rma; pp.gk_rma = w->k_norm_rma;
   pp.q_swa = W.q_swa; pp.q_rma = W.q_rma;

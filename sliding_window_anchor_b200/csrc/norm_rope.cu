@@ -159,7 +159,11 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
     const size_t gi = grp(seq, P.layer, g, P.L);
     dst = ((hs < 44) ? P.pend_k : P.pend_v) + (gi * PEND + p_idx) * D;
     if (hs < 44 && lane == 0) {
-      P.pend_score[gi * PEND + p_idx] = P.s[qi * NG + g];
+      // the score: the 4 quarter partials added in order (as k_score_sum does)
+      float sc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sc += P.s_part[((size_t)q * P.nq + qi) * NG + g];
+      P.pend_score[gi * PEND + p_idx] = sc;
       P.pend_pos[gi * PEND + p_idx] = t;
     }
   }

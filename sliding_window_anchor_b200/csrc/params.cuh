@@ -10,7 +10,7 @@ namespace er {
 
 struct PostParams {
   const uint16_t* proj;  // [nq][12288]
-  const float* s;        // [nq][4]
+  const float* s_part;   // [4 hidden quarters][nq][4]: the scorer's partial scores
   int nq;
   const uint16_t *gq_swa, *gk_swa, *gq_rma, *gk_rma;
   uint16_t *q_swa, *q_rma;  // [nq][16][256] each

@@ -269,6 +269,13 @@ std::mutex g_attr_mu;
 
 }  // namespace
 
+// Where launch_score leaves the partial scores [4][n][4] in its scratch.
+const float* score_partials(const void* scratch, int n) {
+  Carver c(const_cast<void*>(scratch));
+  c.take<uint16_t>((size_t)NPART * SH * HID);
+  return c.take<float>((size_t)NQ * n * NG);
+}
+
 // Scratch layout: the W1 terms (3 x 256 x 2560 BF16; only used when the
 // weights carry no prepared terms), then the partial scores.
 size_t score_scratch_bytes(int n) {
@@ -278,6 +285,8 @@ size_t score_scratch_bytes(int n) {
   return c.used();
 }
 
+// s == nullptr: leave the 4 quarter partials in the scratch (score_partials)
+// for a consumer that adds them itself.
 int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
                  int n, float* s, void* scratch, int32_t* err, cudaStream_t st) {
   if (n <= 0) return ER_OK;
@@ -310,7 +319,11 @@ int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, con
   P.n = n;
   P.err = err;
   k_score_tc<<<dim3(KPARTS, (n + TM - 1) / TM, NQ), 192, SCORE_SMEM, st>>>(P);
-  k_score_sum<<<(n * NG + 255) / 256, 256, 0, st>>>(part, n, s);
+  if (s) {
+    k_score_sum<<<(n * NG + 255) / 256, 256, 0, st>>>(part, n, s);
+  } else {
+    --launches;
+  }
   count_launches(launches);
   return launch_status();
 }
