@@ -30,7 +30,11 @@
  *    outputs, workspace); the library never allocates or frees device memory
  *    and never synchronises the stream, except er_last_device_error, which
  *    reads one word back.
- *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).
+ *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  A
+ *    layer call may also run part of its work (the commit, beside o_proj) on
+ *    a side stream the library keeps per device, forked from and joined back
+ *    to `stream` inside the call, so everything still completes in `stream`
+ *    order and the call can be captured in a CUDA graph.
  *  - Return value: ER_OK, or a negative ER_E* code.  Host-side argument checks
  *    happen before anything is enqueued; a failed check enqueues nothing.
  *    Conditions only the device can see (a sequence id out of range, a full

@@ -7,6 +7,8 @@
 // filled.  A prefill chunk writes its window rows only after every token read,
 // because the chunk's early tokens still see ring positions its late tokens
 // would overwrite (the prefill read kernel's second launch moves them).
+#include <mutex>
+
 #include "common.cuh"
 #include "params.cuh"
 
@@ -63,6 +65,31 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   return w;
 }
 
+// The commit of a layer call runs beside its o_proj GEMM: they touch disjoint
+// data (anchor rows vs the read output).  A side stream per device takes the
+// commit between a fork and a join on the caller's stream, so the call's work
+// still completes in the caller's stream order (and stays capturable).
+struct Side {
+  std::mutex mu;
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+Side g_side[64];
+
+Side* side_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  Side& sd = g_side[dev];
+  std::lock_guard<std::mutex> lock(sd.mu);
+  if (!sd.stream) {
+    if (cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+  }
+  return &sd;
+}
+
 bool weights_ok(const er_layer_weights* w) {
   return w && w->w_qkv && w->w_o && w->q_norm_swa && w->k_norm_swa && w->q_norm_rma &&
          w->k_norm_rma && w->w1 && w->w2 && aligned16(w->w_qkv) && aligned16(w->w_o) &&
@@ -113,10 +140,9 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.err = st->dev_error;
     if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, s)) != ER_OK) return rc;
   }
-  // a6: shared o_proj
-  if ((rc = gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s)) != ER_OK) return rc;
-  // a7: commit this layer where the block is now full (decided on the device)
-  if (rma_off) return ER_OK;
+  // a7: commit this layer where the block is now full (decided on the device),
+  // beside a6, the shared o_proj (disjoint data)
+  if (rma_off) return gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
   CommitParams cp{};
   cp.bank_k = st->bank_k; cp.bank_v = st->bank_v; cp.pend_k = st->pend_k; cp.pend_v = st->pend_v;
   cp.bank_score = st->bank_score; cp.pend_score = st->pend_score;
@@ -125,7 +151,19 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   cp.n = prefill ? 1 : nq; cp.s_max = st->s_max; cp.L = st->n_layers;
   cp.layer0 = layer; cp.nlayers = 1; cp.p_add = prefill ? nq : 1; cp.only_if_full = 1;
   cp.kept = nullptr; cp.err = st->dev_error;
-  return launch_commit(cp, s);
+  Side* sd = side_for_current_device();
+  if (!sd) return ER_ECUDA;
+  std::lock_guard<std::mutex> lock(sd->mu);  // the events are re-recorded by every call
+  if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
+      cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
+    return ER_ECUDA;
+  const int rc_commit = launch_commit(cp, sd->stream);
+  const int rc_proj = gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
+  // join: the caller's stream waits for the commit whatever happened above
+  if (cudaEventRecord(sd->join, sd->stream) != cudaSuccess ||
+      cudaStreamWaitEvent(s, sd->join, 0) != cudaSuccess)
+    return ER_ECUDA;
+  return rc_commit != ER_OK ? rc_commit : rc_proj;
 }
 
 }  // namespace
