@@ -65,10 +65,11 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   return w;
 }
 
-// The commit of a layer call runs beside its o_proj GEMM: they touch disjoint
-// data (anchor rows vs the read output).  A side stream per device takes the
-// commit between a fork and a join on the caller's stream, so the call's work
-// still completes in the caller's stream order (and stays capturable).
+// Steps of a layer call that run beside library GEMMs on a side stream: the
+// commit beside o_proj (anchor rows vs the read output) and, in a prefill
+// chunk, the scorer beside the q/k/v projection (both only read x).  A side stream per device takes them
+// between a fork and a join on the caller's stream, so the call's work still
+// completes in the caller's stream order (and stays capturable).
 struct Side {
   std::mutex mu;
   cudaStream_t stream = nullptr;
@@ -106,13 +107,33 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   LayerWs W = carve_ws(ws, nq, prefill);
   if (ws_bytes < W.bytes) return ER_ECAPACITY;
   int rc;
-  // a1: all six projections in one GEMM
-  if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
-  // a3: FP32 scores (not with the RMA switched off)
-  // (the partial scores stay in the scratch; k_post_proj adds them)
-  if (!rma_off && (rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr, W.score_scratch,
-                                     st->dev_error, s)) != ER_OK)
-    return rc;
+  Side* sd = side_for_current_device();
+  if (!sd) return ER_ECUDA;
+  if (rma_off) {
+    // a1: all six projections in one GEMM
+    if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
+  } else if (!prefill) {
+    // a1, then a3 (FP32 scores; the partials stay in the scratch, k_post_proj
+    // adds them).  Measured: beside a batch's a1 GEMM, which fills the GPU, the
+    // scorer slowed the decode step, so here they run in turn.
+    if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
+    if ((rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr, W.score_scratch,
+                           st->dev_error, s)) != ER_OK)
+      return rc;
+  } else {
+    // a prefill chunk: a3 on the side stream beside a1 (both read only x)
+    std::lock_guard<std::mutex> lock(sd->mu);  // the events are re-recorded by every call
+    if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
+      return ER_ECUDA;
+    const int rc_score = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr,
+                                      W.score_scratch, st->dev_error, sd->stream);
+    const int rc_proj = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s);
+    if (cudaEventRecord(sd->join, sd->stream) != cudaSuccess ||
+        cudaStreamWaitEvent(s, sd->join, 0) != cudaSuccess)
+      return ER_ECUDA;
+    if ((rc = rc_score != ER_OK ? rc_score : rc_proj) != ER_OK) return rc;
+  }
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
   pp.proj = W.proj; pp.s_part = score_partials(W.score_scratch, nq); pp.nq = nq;
@@ -151,8 +172,6 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   cp.n = prefill ? 1 : nq; cp.s_max = st->s_max; cp.L = st->n_layers;
   cp.layer0 = layer; cp.nlayers = 1; cp.p_add = prefill ? nq : 1; cp.only_if_full = 1;
   cp.kept = nullptr; cp.err = st->dev_error;
-  Side* sd = side_for_current_device();
-  if (!sd) return ER_ECUDA;
   std::lock_guard<std::mutex> lock(sd->mu);  // the events are re-recorded by every call
   if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
       cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
