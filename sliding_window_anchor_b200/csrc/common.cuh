@@ -58,6 +58,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// -------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while its
+// predecessor on the stream is still running; it must pass grid_dep_wait()
+// before touching anything the predecessor writes.  grid_dep_trigger() lets a
+// kernel's dependents launch before it has finished (they still wait for all of
+// its memory operations in grid_dep_wait).  Both are no-ops for a plain launch.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------- mbarrier + bulk copies
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -108,6 +108,7 @@ __global__ void k_norm_rope(const uint16_t* x, uint16_t* y, int64_t n_rows, cons
 // q_swa 0..15 | k_swa 16..19 | v_swa 20..23 | q_rma 24..39 | k_rma 40..43 | v_rma 44..47.
 __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   __shared__ float2 s_cs[32];  // the rotation of this token's position, formed once
+  grid_dep_trigger();  // a prefill read may set itself up meanwhile (it waits for us)
   const int lane = threadIdx.x & 31;
   const int hs = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int qi = blockIdx.x;

@@ -208,6 +208,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
   __syncthreads();
   tc::cluster_sync();  // both CTAs' barriers initialised, TMEM held by both
   tc::fence_after_sync();
+  // launched behind the norm/RoPE kernel that writes q, the chunk rows and the
+  // pending records: everything above read only metadata written earlier
+  grid_dep_wait();
+  grid_dep_trigger();  // the combine kernel may launch (it waits for this grid)
   const uint32_t tmem = S.tmem_base;
   const int n = S.ntiles;
 
@@ -470,6 +474,7 @@ struct RingWrite {
 
 __global__ void k_prefill_combine(const float* __restrict__ out, const float2* __restrict__ ml,
                                   int T, int nbr, uint16_t* __restrict__ o_sum, RingWrite rw) {
+  grid_dep_wait();  // the partial reads of the kernel before
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * (OIN / 8)) return;
   {
@@ -581,7 +586,19 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   const dim3 grid(2 * ((T + PAIR_TOK - 1) / PAIR_TOK), NG, nbr * NSPLIT);
   std::pair<cudaEvent_t, cudaEvent_t> ev;
   const bool timed = profile_begin(stream, &ev);
-  k_prefill_attn<<<grid, PF_THREADS, PF_SMEM, stream>>>(P);
+  // both kernels launch programmatically: they may start while their
+  // predecessor runs, and wait for it (grid_dep_wait) before its outputs
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(PF_THREADS);
+  cfg.dynamicSmemBytes = PF_SMEM;
+  cfg.stream = stream;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  const bool launched = cudaLaunchKernelEx(&cfg, k_prefill_attn, P) == cudaSuccess;
   if (timed) profile_end(stream, ev);
   const int nv = T * (OIN / 8);
   RingWrite rw;
@@ -594,7 +611,17 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   rw.s_max = st->s_max;
   rw.L = st->n_layers;
   rw.layer = layer;
-  k_prefill_combine<<<(nv + 255) / 256, 256, 0, stream>>>(out, P.ml, T, nbr, o_sum, rw);
+  cudaLaunchConfig_t cfg2 = {};
+  cfg2.gridDim = dim3((nv + 255) / 256);
+  cfg2.blockDim = dim3(256);
+  cfg2.dynamicSmemBytes = 0;
+  cfg2.stream = stream;
+  cfg2.attrs = pdl;
+  cfg2.numAttrs = 1;
+  if (!launched ||
+      cudaLaunchKernelEx(&cfg2, k_prefill_combine, (const float*)out, (const float2*)P.ml, T,
+                         nbr, o_sum, rw) != cudaSuccess)
+    return ER_ECUDA;
   count_launches(2);
   return launch_status();
 }
