@@ -260,6 +260,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
     fence_mbar_init();
   }
   __syncthreads();
+  // launched behind the kernel that writes q, the window slot and the pending
+  // record (norm/RoPE): nothing above touched them
+  grid_dep_wait();
 
   // contiguous, even-length item ranges per CTA: a (query, group)'s two branch
   // items are read back to back by the same CTA
@@ -646,7 +649,22 @@ int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* 
   P.o_sum = o_sum;
   std::pair<cudaEvent_t, cudaEvent_t> ev;
   const bool timed = profile_begin(st, &ev);
-  k_attend<<<grid, NTHREADS, sizeof(AttnSmem) + 1024, st>>>(P);
+  // a programmatic launch: the CTAs may start while the kernel before still runs
+  // and wait for it (grid_dep_wait) before reading anything it writes
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = sizeof(AttnSmem) + 1024;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_attend, P) != cudaSuccess) {
+    if (timed) profile_end(st, ev);
+    return ER_ECUDA;
+  }
   if (timed) profile_end(st, ev);
   count_launches(1);
   int rc = launch_status();

@@ -122,6 +122,9 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   const int32_t t = pos0 + (P.prefill ? qi : 0);
   if (threadIdx.x < 32) s_cs[lane] = rope_cs_lane(t, lane);
   __syncthreads();
+  // launched behind the scorer / the projection GEMM: the angles above used only
+  // metadata; the projections and the partial scores come from them
+  grid_dep_wait();
   const int p_idx = pend0 + (P.prefill ? qi : 0);
   const bool state_ok = p_idx >= 0 && p_idx < PEND && t >= 0;
   if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
@@ -176,7 +179,18 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
 // first three run.
 int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st) {
   if (P.nq <= 0) return ER_OK;
-  k_post_proj<<<dim3(P.nq, rma_off ? 3 : 6), 256, 0, st>>>(P);
+  // a programmatic launch (see grid_dep_wait above)
+  cudaLaunchAttribute pdl[1];
+  pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.nq, rma_off ? 3 : 6);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cfg.attrs = pdl;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_post_proj, P) != cudaSuccess) return ER_ECUDA;
   count_launches(1);
   return launch_status();
 }

@@ -121,6 +121,7 @@ __global__ void __cluster_dims__(KPARTS, 1, 1) __launch_bounds__(192, 1)
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   ScoreSmem& S = *reinterpret_cast<ScoreSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  grid_dep_trigger();  // the norm/RoPE kernel may set itself up (it waits for us)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();  // the K part
   const int m0 = blockIdx.y * TM;
