@@ -69,6 +69,7 @@ typedef struct CUstream_st* er_stream_t; /* same type as cudaStream_t */
 #define ER_ROPE_DIMS 64
 #define ER_SCORE_HIDDEN 256
 #define ER_QKV_ROWS 12288 /* 4096 + 1024 + 1024 (SWA) + 4096 + 1024 + 1024 (RMA) */
+#define ER_QKV_SCORE_ROWS 13056 /* ER_QKV_ROWS + the three BF16 terms of W1 (3 x 256) */
 #define ER_O_IN 4096      /* 16 heads x 256 */
 
 enum {
@@ -115,7 +116,21 @@ typedef struct er_state {
  *   w1_split (optional, may be NULL): BF16 [3][256][2560], w1 written as three
  *                             BF16 terms by er_score_split_w1 (prepared once per
  *                             weight set); NULL makes every scorer call split
- *                             w1 again into its workspace. */
+ *                             w1 again into its workspace.
+ *   w_qkv_score (optional, may be NULL): BF16 [13056][2560], rows 0..12287 equal
+ *                             to w_qkv and rows 12288..13055 the three W1 terms in
+ *                             w1_split's layout (er_prepare_qkv_score writes it).
+ *                             When set, the layer calls take a1 and the W1·x
+ *                             product of a3 from ONE GEMM over it (FP32 output;
+ *                             the projections are then rounded to BF16, the same
+ *                             values a BF16-output GEMM gives) and apply SiLU and
+ *                             W2 in the norm/RoPE kernel, so no separate scorer
+ *                             launch runs (calls with ER_FLAG_RMA_OFF score
+ *                             nothing and project from w_qkv with BF16 output).
+ *                             w_qkv, w1 and w1_split must still be
+ *                             valid (the standalone er_rma_score reads them); a
+ *                             caller can point w_qkv and w1_split into this
+ *                             buffer so the layer holds one copy. */
 typedef struct er_layer_weights {
   const er_bf16* w_qkv;
   const er_bf16* w_o;
@@ -123,6 +138,7 @@ typedef struct er_layer_weights {
   const float* w1;
   const float* w2;
   const er_bf16* w1_split;
+  const er_bf16* w_qkv_score;
 } er_layer_weights;
 
 /* ---------------------------------------------------------------- state */
@@ -190,6 +206,14 @@ size_t er_score_workspace_bytes(int32_t n);
  * bf16(w1), mid = bf16(w1 - hi), lo = bf16(w1 - hi - mid).  The result is the
  * optional er_layer_weights.w1_split. */
 int er_score_split_w1(const float* w1, er_bf16* terms, er_stream_t stream);
+
+/* Builds er_layer_weights.w_qkv_score: copies w_qkv (BF16 [12288][2560]) into
+ * rows 0..12287 of out (BF16 [13056][2560], caller-owned device memory,
+ * 16-byte aligned, not overlapping w_qkv) and writes w1's three BF16 terms
+ * (as er_score_split_w1) into rows 12288..13055.  Stream-ordered; ER_EINVAL
+ * on NULL or unaligned pointers. */
+int er_prepare_qkv_score(const er_bf16* w_qkv, const float* w1, er_bf16* out,
+                         er_stream_t stream);
 int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
                  size_t ws_bytes, er_stream_t stream);
 

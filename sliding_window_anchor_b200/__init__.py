@@ -74,9 +74,12 @@ class State:
 class LayerWeights:
     """One layer's device weights (BF16 projections and gains, FP32 scorer).
 
-    With prepare=True (the default) W1's three BF16 terms are made once here
-    (er_score_split_w1) and every scorer call reuses them; prepare=False leaves
-    w1_split NULL, so each call splits W1 again in its workspace."""
+    With prepare=True (the default) one BF16 [13056][2560] buffer is built here
+    (er_prepare_qkv_score): W_qkv followed by W1's three BF16 terms.  The layer
+    calls then run the q/k/v projection and the scorer's W1 product as one GEMM,
+    and w_qkv and w1_split become views of that buffer (one copy on the device).
+    prepare=False leaves w1_split and w_qkv_score NULL: the layer calls project
+    and score separately, and each scorer call splits W1 again in its workspace."""
 
     def __init__(self, w_qkv, w_o, q_norm_swa, k_norm_swa, q_norm_rma, k_norm_rma, w1, w2,
                  prepare: bool = True):
@@ -92,15 +95,19 @@ class LayerWeights:
                 raise ValueError(f"{k}: expected {shape} {dt}, got {tuple(t.shape)} {t.dtype}")
             dev_ptr(t, dt, k)
         self.w1_split = None
+        self.w_qkv_score = None
         if prepare:
-            self.w1_split = torch.empty(3, 256, HIDDEN, dtype=bf, device=w1.device)
-            check("er_score_split_w1", lib().er_score_split_w1(
-                dev_ptr(w1, f32, "w1"), dev_ptr(self.w1_split, bf, "w1_split"),
-                stream_handle(None, w1.device)))
+            self.w_qkv_score = torch.empty(QKV + 3 * 256, HIDDEN, dtype=bf, device=w1.device)
+            check("er_prepare_qkv_score", lib().er_prepare_qkv_score(
+                dev_ptr(w_qkv, bf, "w_qkv"), dev_ptr(w1, f32, "w1"),
+                dev_ptr(self.w_qkv_score, bf, "w_qkv_score"), stream_handle(None, w1.device)))
+            self.t["w_qkv"] = self.w_qkv_score[:QKV]
+            self.w1_split = self.w_qkv_score[QKV:].view(3, 256, HIDDEN)
+        opt = lambda t: t.data_ptr() if t is not None else None
         self.c = _lib.CWeights(*[self.t[k].data_ptr() for k in
                                  ("w_qkv", "w_o", "q_norm_swa", "k_norm_swa", "q_norm_rma",
                                   "k_norm_rma", "w1", "w2")],
-                               self.w1_split.data_ptr() if self.w1_split is not None else None)
+                               opt(self.w1_split), opt(self.w_qkv_score))
 
     @classmethod
     def from_dict(cls, d, prepare: bool = True):

@@ -40,7 +40,7 @@ ER_FLAG_RMA_OFF = 1  # the RMA switched off (the pages' ablation)
 class CWeights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("w_qkv", "w_o", "q_norm_swa", "k_norm_swa",
                                                "q_norm_rma", "k_norm_rma", "w1", "w2",
-                                               "w1_split")]
+                                               "w1_split", "w_qkv_score")]
 
 
 EXPORTS = {
@@ -60,6 +60,8 @@ EXPORTS = {
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "er_score_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "er_score_split_w1": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "er_prepare_qkv_score": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p]),
     "er_rma_score": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p, ctypes.c_int32,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                     ctypes.c_void_p]),

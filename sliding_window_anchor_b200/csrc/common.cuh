@@ -22,6 +22,7 @@ constexpr int PEND = ER_PENDING;        // 256
 constexpr int ROPE = ER_ROPE_DIMS;      // 64
 constexpr int SH = ER_SCORE_HIDDEN;     // 256
 constexpr int QKV = ER_QKV_ROWS;        // 12288
+constexpr int QKVS = ER_QKV_SCORE_ROWS; // 13056: q/k/v rows + the 3 x 256 W1-term rows
 constexpr int OIN = ER_O_IN;            // 4096
 constexpr int ROW_BYTES = D * 2;        // one BF16 K or V row
 

@@ -16,6 +16,8 @@ namespace er {
 
 int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
                   cudaStream_t st);
+int gemm_bf16_xwt_f32(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
+                      int ldy, cudaStream_t st);
 int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
                  int n, float* s, void* scratch, int32_t* err, cudaStream_t st);
 size_t score_scratch_bytes(int n);
@@ -38,7 +40,7 @@ namespace er {
 namespace {
 
 struct LayerWs {
-  uint16_t* proj;
+  void* proj;  // BF16 [nq][12288], or FP32 [nq][13056] with the fused weights
   unsigned char* score_scratch;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
@@ -51,7 +53,7 @@ struct LayerWs {
 LayerWs carve_ws(void* base, int nq, bool prefill) {
   Carver c(base);
   LayerWs w;
-  w.proj = c.take<uint16_t>((size_t)nq * QKV);
+  w.proj = c.take<float>((size_t)nq * QKVS);
   w.score_scratch = c.take<unsigned char>(score_scratch_bytes(nq));
   w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
@@ -96,7 +98,8 @@ bool weights_ok(const er_layer_weights* w) {
          w->k_norm_rma && w->w1 && w->w2 && aligned16(w->w_qkv) && aligned16(w->w_o) &&
          aligned16(w->q_norm_swa) && aligned16(w->k_norm_swa) && aligned16(w->q_norm_rma) &&
          aligned16(w->k_norm_rma) && aligned16(w->w1) && aligned16(w->w2) &&
-         (!w->w1_split || aligned16(w->w1_split));
+         (!w->w1_split || aligned16(w->w1_split)) &&
+         (!w->w_qkv_score || aligned16(w->w_qkv_score));
 }
 
 int run_layer(const er_state* st, const er_layer_weights* w, int layer, const int32_t* seq_ids,
@@ -109,14 +112,22 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   int rc;
   Side* sd = side_for_current_device();
   if (!sd) return ER_ECUDA;
-  if (rma_off) {
+  // with the RMA off nothing is scored: the plain BF16 projection is cheaper
+  const bool fused = w->w_qkv_score != nullptr && !rma_off;
+  uint16_t* proj_bf = static_cast<uint16_t*>(W.proj);
+  float* proj_f = static_cast<float*>(W.proj);
+  if (fused) {
+    // a1 and a3's W1·x in one GEMM, FP32 out
+    if ((rc = gemm_bf16_xwt_f32(x, w->w_qkv_score, proj_f, nq, QKVS, HID, QKVS, s)) != ER_OK)
+      return rc;
+  } else if (rma_off) {
     // a1: all six projections in one GEMM
-    if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
+    if ((rc = gemm_bf16_xwt(x, w->w_qkv, proj_bf, nq, QKV, HID, s)) != ER_OK) return rc;
   } else if (!prefill) {
     // a1, then a3 (FP32 scores; the partials stay in the scratch, k_post_proj
     // adds them).  Measured: beside a batch's a1 GEMM, which fills the GPU, the
     // scorer slowed the decode step, so here they run in turn.
-    if ((rc = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s)) != ER_OK) return rc;
+    if ((rc = gemm_bf16_xwt(x, w->w_qkv, proj_bf, nq, QKV, HID, s)) != ER_OK) return rc;
     if ((rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr, W.score_scratch,
                            st->dev_error, s)) != ER_OK)
       return rc;
@@ -128,7 +139,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
       return ER_ECUDA;
     const int rc_score = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr,
                                       W.score_scratch, st->dev_error, sd->stream);
-    const int rc_proj = gemm_bf16_xwt(x, w->w_qkv, W.proj, nq, QKV, HID, s);
+    const int rc_proj = gemm_bf16_xwt(x, w->w_qkv, proj_bf, nq, QKV, HID, s);
     if (cudaEventRecord(sd->join, sd->stream) != cudaSuccess ||
         cudaStreamWaitEvent(s, sd->join, 0) != cudaSuccess)
       return ER_ECUDA;
@@ -136,7 +147,11 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   }
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
-  pp.proj = W.proj; pp.s_part = score_partials(W.score_scratch, nq); pp.nq = nq;
+  pp.proj = fused ? nullptr : proj_bf;
+  pp.proj_f32 = fused ? proj_f : nullptr;
+  pp.s_part = fused ? nullptr : score_partials(W.score_scratch, nq);
+  pp.w2 = w->w2;
+  pp.nq = nq;
   pp.gq_swa = w->q_norm_swa; pp.gk_swa = w->k_norm_swa;
   pp.gq_rma = w->q_norm_rma; pp.gk_rma = w->k_norm_rma;
   pp.q_swa = W.q_swa; pp.q_rma = W.q_rma;

@@ -139,7 +139,16 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   else { col = OFF_V_RMA + (hs - 44) * D; }
 
   float v[8];
-  load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
+  if (P.proj_f32) {
+    // FP32 sums of the fused GEMM, rounded to BF16 as a BF16-output GEMM would
+    const float4* src = reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + col) +
+                        lane * 2;
+    const float4 a = src[0], b = src[1];
+    v[0] = bf1(f2bf(a.x)); v[1] = bf1(f2bf(a.y)); v[2] = bf1(f2bf(a.z)); v[3] = bf1(f2bf(a.w));
+    v[4] = bf1(f2bf(b.x)); v[5] = bf1(f2bf(b.y)); v[6] = bf1(f2bf(b.z)); v[7] = bf1(f2bf(b.w));
+  } else {
+    load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
+  }
   if (gain) norm_rope_lane_cs(v, gain, s_cs, lane);
 
   uint16_t* dst = nullptr;
@@ -162,13 +171,34 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
     const int g = (hs < 44) ? hs - 40 : hs - 44;
     const size_t gi = grp(seq, P.layer, g, P.L);
     dst = ((hs < 44) ? P.pend_k : P.pend_v) + (gi * PEND + p_idx) * D;
-    if (hs < 44 && lane == 0) {
-      // the score: the 4 quarter partials added in order (as k_score_sum does)
+    if (hs < 44) {
       float sc = 0.f;
+      if (P.proj_f32) {
+        // the score of group g from the fused GEMM: h_j = hi_j + mid_j + lo_j (the
+        // three W1-term sums, smallest first), s_g = sum_j W2[g][j] SiLU(h_j);
+        // lane covers j = 8 lane .. 8 lane + 7, then a fixed-order warp sum
+        const float4* hrow =
+            reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + QKV) + lane * 2;
+        const float4* w2g = reinterpret_cast<const float4*>(P.w2 + g * 256) + lane * 2;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) sc += P.s_part[((size_t)q * P.nq + qi) * NG + g];
-      P.pend_score[gi * PEND + p_idx] = sc;
-      P.pend_pos[gi * PEND + p_idx] = t;
+        for (int e = 0; e < 2; ++e) {
+          const float4 hi = hrow[e], mid = hrow[64 + e], lo = hrow[128 + e], w2 = w2g[e];
+          const float h0 = (lo.x + mid.x) + hi.x, h1 = (lo.y + mid.y) + hi.y;
+          const float h2 = (lo.z + mid.z) + hi.z, h3 = (lo.w + mid.w) + hi.w;
+          sc += w2.x * (h0 / (1.0f + expf(-h0))) + w2.y * (h1 / (1.0f + expf(-h1))) +
+                w2.z * (h2 / (1.0f + expf(-h2))) + w2.w * (h3 / (1.0f + expf(-h3)));
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+      } else if (lane == 0) {
+        // the separate scorer: its 4 quarter partials added in order
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sc += P.s_part[((size_t)q * P.nq + qi) * NG + g];
+      }
+      if (lane == 0) {
+        P.pend_score[gi * PEND + p_idx] = sc;
+        P.pend_pos[gi * PEND + p_idx] = t;
+      }
     }
   }
   store8(dst + lane * 8, v);

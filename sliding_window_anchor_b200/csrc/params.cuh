@@ -9,8 +9,10 @@
 namespace er {
 
 struct PostParams {
-  const uint16_t* proj;  // [nq][12288]
-  const float* s_part;   // [4 hidden quarters][nq][4]: the scorer's partial scores
+  const uint16_t* proj;      // [nq][12288] BF16 (separate scorer), or
+  const float* proj_f32;     // [nq][13056] FP32: q/k/v sums, then hi/mid/lo W1-term sums
+  const float* s_part;       // separate scorer: [4 hidden quarters][nq][4] partial scores
+  const float* w2;           // fused: W2 [4][256] FP32
   int nq;
   const uint16_t *gq_swa, *gk_swa, *gq_rma, *gk_rma;
   uint16_t *q_swa, *q_rma;  // [nq][16][256] each

@@ -363,6 +363,21 @@ int er_score_split_w1(const float* w1, er_bf16* terms, er_stream_t stream) {
   return launch_status();
 }
 
+int er_prepare_qkv_score(const er_bf16* w_qkv, const float* w1, er_bf16* out,
+                         er_stream_t stream) {
+  if (!w_qkv || !w1 || !out || !aligned16(w_qkv) || !aligned16(w1) || !aligned16(out))
+    return ER_EINVAL;
+  const size_t qkv_bytes = (size_t)QKV * HID * sizeof(uint16_t);
+  const uintptr_t a = reinterpret_cast<uintptr_t>(w_qkv), b = reinterpret_cast<uintptr_t>(out);
+  if (a < b + (size_t)QKVS * HID * sizeof(uint16_t) && b < a + qkv_bytes) return ER_EINVAL;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(out, w_qkv, qkv_bytes, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return ER_ECUDA;
+  k_w1_split<<<148 * 4, 256, 0, st>>>(w1, out + (size_t)QKV * HID, SH * HID);
+  count_launches(1);
+  return launch_status();
+}
+
 int er_rma_score_noalloc(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s,
                          er_stream_t stream) {
   if (!w || n < 0 || (n > 0 && (!w->w1 || !w->w2 || !x || !s))) return ER_EINVAL;

@@ -20,10 +20,11 @@ def oracle_weights(seed, layer):
                                 w["q_norm_rma"], w["k_norm_rma"], w["w1"], w["w2"]), w
 
 
-def gpu_weights(seed, layer):
+def gpu_weights(seed, layer, prepare=True):
+    """Device weights; prepare=True gives the fused q/k/v + W1-term GEMM weights."""
     import sliding_window_anchor_b200 as sab
     w = wl.make_weights(seed, layer, device="cuda")
-    return sab.LayerWeights.from_dict(w), w
+    return sab.LayerWeights.from_dict(w, prepare=prepare), w
 
 
 def gpu_normrope(x, gain, pos):
@@ -69,3 +70,24 @@ def tol_ok(gpu, ref, atol=1e-2, rtol=1e-2):
 
 def max_err(gpu, ref):
     return float((gpu.double().cpu() - ref.double().cpu()).abs().max())
+
+
+def kept_sets_agree(gpu_row, ost_row, n_layers):
+    """Bank position sets per (layer, group) match, up to near-ties at the boundary."""
+    for l in range(n_layers):
+        for g in range(4):
+            c = int(ost_row["meta"][2])
+            gp = set(gpu_row["bank_pos"][l, g, :c].tolist())
+            op = set(ost_row["bank_pos"][l, g, :c].tolist())
+            if gp == op:
+                continue
+            # records only one side kept must sit at the boundary score within 1e-5 relative
+            ob = ost_row["bank_score"][l, g, :c].double()
+            smin = float(ob.min())
+            for side, pos_set, other, scores, poss in (
+                    ("gpu", gp, op, gpu_row["bank_score"][l, g, :c], gpu_row["bank_pos"][l, g, :c]),
+                    ("oracle", op, gp, ost_row["bank_score"][l, g, :c], ost_row["bank_pos"][l, g, :c])):
+                for pos in pos_set - other:
+                    s = float(scores[(poss == pos).nonzero()[0, 0]])
+                    assert abs(s - smin) <= 1e-5 * max(abs(smin), 1e-30) + 1e-12, (side, l, g, pos)
+    return True

@@ -130,3 +130,14 @@ def test_host_validation_rejects_before_enqueue(L):
     assert L.er_swa_rma_prefill_chunk_ex(ctypes.byref(st), ctypes.byref(w), 0, 0, nul, 16, nul,
                                          nul, 0, 8, nul) == -1
     assert L.er_launch_count() == before
+    # the fused q/k/v + W1-term weights: NULL, unaligned or overlapping buffers are refused
+    base = 1 << 40
+    qkv_bytes = 12288 * 2560 * 2
+    before = L.er_launch_count()
+    assert L.er_prepare_qkv_score(nul, ok, ok, nul) == -1
+    assert L.er_prepare_qkv_score(ok, ok, fake, nul) == -1
+    assert L.er_prepare_qkv_score(ctypes.c_void_p(base), ok,
+                                  ctypes.c_void_p(base + qkv_bytes - 4096), nul) == -1
+    assert L.er_prepare_qkv_score(ctypes.c_void_p(base + qkv_bytes), ok,
+                                  ctypes.c_void_p(base + 4096), nul) == -1
+    assert L.er_launch_count() == before

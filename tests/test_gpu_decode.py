@@ -26,27 +26,6 @@ def sab():
     return m
 
 
-def _kept_sets_agree(gpu_row, ost_row, n_layers):
-    """Bank position sets per (layer, group) match, up to near-ties at the boundary."""
-    for l in range(n_layers):
-        for g in range(4):
-            c = int(ost_row["meta"][2])
-            gp = set(gpu_row["bank_pos"][l, g, :c].tolist())
-            op = set(ost_row["bank_pos"][l, g, :c].tolist())
-            if gp == op:
-                continue
-            # records only one side kept must sit at the boundary score within 1e-5 relative
-            ob = ost_row["bank_score"][l, g, :c].double()
-            smin = float(ob.min())
-            for side, pos_set, other, scores, poss in (
-                    ("gpu", gp, op, gpu_row["bank_score"][l, g, :c], gpu_row["bank_pos"][l, g, :c]),
-                    ("oracle", op, gp, ost_row["bank_score"][l, g, :c], ost_row["bank_pos"][l, g, :c])):
-                for pos in pos_set - other:
-                    s = float(scores[(poss == pos).nonzero()[0, 0]])
-                    assert abs(s - smin) <= 1e-5 * max(abs(smin), 1e-30) + 1e-12, (side, l, g, pos)
-    return True
-
-
 def _run_oracle_seq(ow_list, ost, row, steps, layers, seed, gseq, x_of):
     outs = {}
     for step in range(steps):
@@ -84,7 +63,7 @@ def test_decode_single_layer_256_steps_with_commit(sab):
     grow, orow = H.download_row(st, 0), {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
     assert torch.equal(grow["meta"], orow["meta"])
     assert int(orow["meta"][1]) == 0 and int(orow["meta"][0]) == cfg["t0"] + 256
-    _kept_sets_agree(grow, orow, L)
+    H.kept_sets_agree(grow, orow, L)
 
 
 @pytest.mark.parametrize("cfg_index", [2, 3])
@@ -127,7 +106,7 @@ def test_decode_batched_sampled_sequences(sab, cfg_index):
         grow = H.download_row(st, gseq)
         orow = {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
         assert torch.equal(grow["meta"], orow["meta"])
-        _kept_sets_agree(grow, orow, L)
+        H.kept_sets_agree(grow, orow, L)
 
 
 PREFILL_CASES = {
@@ -139,6 +118,10 @@ PREFILL_CASES = {
     "partial_bank_t5000": dict(t0=5000, pend=100, bank=700, chunks=(156, 40)),
     # the stream start: empty state, the ring partly written, the bank growing
     "stream_start": dict(t0=None, pend=0, bank=None, chunks=(256, 256, 77, 50)),
+    # weights without preparation: the projection and the scorer as separate launches
+    # (prefill and, through the replay, decode)
+    "partial_bank_t5000_unprepared": dict(t0=5000, pend=100, bank=700, chunks=(156, 40),
+                                          prepare=False),
 }
 
 
@@ -151,7 +134,7 @@ def test_prefill_chunks_match_oracle_and_decode(sab, case):
     seed = wl.seed_of(4)
     L = 1
     ow, wdict = H.oracle_weights(seed, 0)
-    gw, gdict = H.gpu_weights(seed, 0)
+    gw, gdict = H.gpu_weights(seed, 0, prepare=cfg.get("prepare", True))
     ost = oracle.OracleState(1, L)
     st = sab.State(2, L)
     if cfg["t0"] is None:
@@ -184,8 +167,8 @@ def test_prefill_chunks_match_oracle_and_decode(sab, case):
     g0, g1 = H.download_row(st, 0), H.download_row(st, 1)
     orow = {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
     assert torch.equal(g0["meta"], orow["meta"]) and torch.equal(g1["meta"], orow["meta"])
-    _kept_sets_agree(g0, orow, L)
-    _kept_sets_agree(g1, orow, L)
+    H.kept_sets_agree(g0, orow, L)
+    H.kept_sets_agree(g1, orow, L)
 
 
 def test_snapshot_restore_is_bit_identical(sab):

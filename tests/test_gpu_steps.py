@@ -70,6 +70,26 @@ def test_score_matches_oracle(sab, n):
     assert bool(((got.double() - ref.double()).abs() <= 1e-4 * cond).all())
 
 
+def test_prepare_qkv_score_layout(sab):
+    """er_prepare_qkv_score: rows 0..12287 are W_qkv's bits, rows 12288.. the three
+    W1 terms exactly as er_score_split_w1 writes them."""
+    w = wl.make_weights(7, 0, device="cuda")
+    gw = sab.LayerWeights.from_dict(w)
+    assert gw.w_qkv_score.shape == (12288 + 768, 2560)
+    assert torch.equal(gw.w_qkv_score[:12288], w["w_qkv"])
+    plain = sab.LayerWeights.from_dict(w, prepare=False)
+    assert plain.w_qkv_score is None and plain.w1_split is None
+    terms = torch.empty(3, 256, 2560, dtype=torch.bfloat16, device="cuda")
+    from sliding_window_anchor_b200 import _lib
+    _lib.check("er_score_split_w1", _lib.lib().er_score_split_w1(
+        w["w1"].data_ptr(), terms.data_ptr(), None))
+    torch.cuda.synchronize()
+    assert torch.equal(gw.w_qkv_score[12288:].view(3, 256, 2560), terms)
+    # hi + mid + lo reproduces W1 to within 2^-24 relative (the three-term split)
+    s = terms.double().sum(0)
+    assert bool(((s - w["w1"].double()).abs() <= 2.0 ** -24 * w["w1"].double().abs()).all())
+
+
 # ----------------------------------------------------------------- a4
 
 def test_append_bit_exact(sab):
