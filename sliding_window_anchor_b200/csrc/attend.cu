@@ -59,11 +59,12 @@ constexpr int NTHREADS = (NCW + 1) * 32;
 constexpr int BOX = 64 * 128;           // one 64-row x 64-dim box (8 KB, 128 B per row)
 constexpr int TILE_BYTES = 4 * BOX;     // a 64-row K (or V) tile: four boxes
 constexpr float kLog2eOver16 = 1.4426950408889634f / 16.0f;
-constexpr int F_FIRST = 1, F_LAST = 2;
+constexpr int F_FIRST = 1, F_LAST = 2, F_END = 4;  // F_END: no more work for this CTA
 
 struct TileDesc {
   int rows;
   int flags;
+  int item;
 };
 
 struct __align__(1024) AttnSmem {
@@ -138,11 +139,11 @@ __device__ __forceinline__ void item_coords(const AttendParams& P, int item, int
 
 struct Tile {
   int map, row;
-  int rows, flags, qi, g, br;
+  int rows, flags, qi, g, br, item;
 };
 
-// The CTA's tile sequence: items item_begin..item_end-1, each the tiles of its
-// split (or one empty tile when the split has no rows).
+// The tiles of items begin..end-1, each the tiles of its split (or one empty
+// tile when the split has no rows).
 struct TileIter {
   const AttendParams* P;
   int item, item_end;
@@ -178,6 +179,7 @@ struct TileIter {
   }
   __device__ bool next(Tile* t) {
     if (item >= item_end) return false;
+    t->item = item;
     t->qi = qi;
     t->g = g;
     t->br = br;
@@ -264,20 +266,34 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
   // record (norm/RoPE): nothing above touched them
   grid_dep_wait();
 
-  // contiguous, even-length item ranges per CTA: a (query, group)'s two branch
-  // items are read back to back by the same CTA
-  int per = (n_items + gridDim.x - 1) / gridDim.x;
-  per += per & 1;
-  const int item_begin = min(n_items, (int)blockIdx.x * per);
-  const int item_end = min(n_items, item_begin + per);
+  // Work is handed out in units of two consecutive items (a (query, group)'s
+  // two branch items when unsplit, read back to back by one CTA): the producer
+  // takes the next unit from a counter in global memory (zeroed before the
+  // launch) when it has issued the last one, so CTAs that meet short items take
+  // more and all finish within about one unit of each other.  Nothing waits on
+  // another CTA.
+  const int n_units = n_items / 2;
 
   if (warp == NCW) {
     // ------------------------------------------------------------ producer
+    auto take_unit = [&]() {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(P.sched, 1);
+      u = __shfl_sync(0xffffffffu, u, 0);
+      return (u < 0 || u > n_units) ? n_units : u;  // past the end: no more work
+    };
     TileIter ld;
-    ld.init(&P, item_begin, item_end);
+    int unit = take_unit();
+    ld.init(&P, 2 * unit, 2 * min(unit + 1, n_units));
     Tile t;
     uint32_t tc = 0;
-    while (ld.next(&t)) {
+    while (true) {
+      if (!ld.next(&t)) {
+        if (unit >= n_units) break;
+        unit = take_unit();
+        ld.init(&P, 2 * unit, 2 * min(unit + 1, n_units));
+        continue;
+      }
       const int stage = tc % STAGES;
       const uint32_t phase = (tc / STAGES) & 1;
       if (lane == 0 && !mbar_wait(&S.empty[stage], phase ^ 1, P.err)) S.abort_flag = 1;
@@ -290,6 +306,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
         const uint32_t bytes = (t.rows > 0 ? 2u * TILE_BYTES : 0u) + qbytes;
         S.desc[stage].rows = t.rows;
         S.desc[stage].flags = t.flags;
+        S.desc[stage].item = t.item;
         if (bytes) mbar_arrive_expect_tx(&S.full[stage], bytes);
         else mbar_arrive(&S.full[stage]);
         if (qbytes)
@@ -304,6 +321,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
         }
       }
       ++tc;
+    }
+    if (!S.abort_flag) {
+      // the end marker: an empty tile the consumers stop at
+      const int stage = tc % STAGES;
+      const uint32_t phase = (tc / STAGES) & 1;
+      if (lane == 0 && !mbar_wait(&S.empty[stage], phase ^ 1, P.err)) S.abort_flag = 1;
+      __syncwarp();
+      if (!S.abort_flag) {
+        if (lane == 0) {
+          S.desc[stage].rows = 0;
+          S.desc[stage].flags = F_END;
+          S.desc[stage].item = -1;
+          mbar_arrive(&S.full[stage]);
+        }
+        ++tc;
+      }
     }
     // drain: the last tile of each stage must have landed before exit
     if (lane == 0)
@@ -334,9 +367,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
 #pragma unroll
   for (int i = 0; i < 8; ++i) keep[i] = 0.f;
 
-  for (int item = item_begin; item < item_end; ++item) {
-    int qi, g, br, split;
-    item_coords(P, item, &qi, &g, &br, &split);
+  int item = 0, qi = 0, g = 0, br = 0;
+  while (true) {
+    bool end = false;
     uint32_t qb[16][2];  // Qᵀ B fragments for the 16 k-steps (heads >= 4 are zero)
     float o[16][4];      // Oᵀ accumulators: dims 16mt + gq (+8) x heads 2cq (+1)
 #pragma unroll
@@ -355,8 +388,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
         S.abort_flag = 1;
       }
       const TileDesc d = S.desc[stage];
+      if (!aborted && (d.flags & F_END)) {
+        end = true;
+        break;
+      }
       const int nrows = aborted ? 0 : min(16, d.rows - row0);
-      if (d.flags & F_FIRST) {
+      if (!aborted && (d.flags & F_FIRST)) {
+        // a new item: its coordinates come with its first tile
+        int split;
+        item = d.item;
+        item_coords(P, item, &qi, &g, &br, &split);
         const uint16_t* q = S.q[stage];
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk) {
@@ -461,6 +502,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[stage]);
     }
+    if (end) break;
 
     // ---- merge the 4 warps' partials of this item
     // merge slot of (warp, head): 1 KB inside this warp's own rows of K box `head`
@@ -515,7 +557,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
           acc[4] += b.x * f; acc[5] += b.y * f; acc[6] += b.z * f; acc[7] += b.w * f;
         }
       }
-      if (P.direct) {
+      if (aborted) {
+        // a wait ran out (error recorded): the item index may be stale, write nothing
+      } else if (P.direct) {
         const float rcp = Ls > 0.f ? 1.0f / Ls : 0.f;
         const size_t oi = ((size_t)qi * NH + g * HPG + h) * D + d0;
         if (P.o_sum == nullptr) {
@@ -612,9 +656,13 @@ bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows) {
 
 }  // namespace
 
+// P0.sched must be 0 when the kernel starts: zero_sched makes this call clear it
+// first (a memset on st); the layer path has k_post_proj clear it instead.
 int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* o_sum,
-                  cudaStream_t st) {
+                  bool zero_sched, cudaStream_t st) {
   if (P0.nq <= 0) return ER_OK;
+  if (!P0.sched) return ER_EINVAL;
+  if (zero_sched && cudaMemsetAsync(P0.sched, 0, sizeof(int), st) != cudaSuccess) return ER_ECUDA;
   AttendParams P = P0;
   P.splits = attend_splits(P.nq);
   const uint64_t groups = (uint64_t)P.s_max * P.L * NG;
@@ -686,6 +734,7 @@ size_t er_attend_workspace_bytes(int32_t B) {
   Carver c(nullptr);
   c.take<float>(attend_part_floats(B));
   c.take<float>(attend_ml_floats(B));
+  c.take<int>(1);
   return c.used();
 }
 
@@ -709,8 +758,9 @@ int er_swa_rma_attend(const er_state* st, int32_t layer, const int32_t* seq_ids,
   P.q_swa = q_swa; P.q_rma = q_rma; P.nq = B; P.prefill = 0;
   P.part_o = c.take<float>(attend_part_floats(B));
   P.part_ml = c.take<float>(attend_ml_floats(B));
+  P.sched = c.take<int>(1);
   P.err = st->dev_error;
-  return launch_attend(P, o_swa, o_rma, nullptr, (cudaStream_t)stream);
+  return launch_attend(P, o_swa, o_rma, nullptr, true, (cudaStream_t)stream);
 }
 
 }  // extern "C"

@@ -24,7 +24,7 @@ size_t score_scratch_bytes(int n);
 const float* score_partials(const void* scratch, int n);
 int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
-                  cudaStream_t st);
+                  bool zero_sched, cudaStream_t st);
 int launch_commit(const CommitParams& P, cudaStream_t st);
 size_t attend_part_floats(int nq);
 size_t attend_ml_floats(int nq);
@@ -45,6 +45,7 @@ struct LayerWs {
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
   float *part_o, *part_ml;  // decode: split partials of the reads
+  int* sched;                // decode: the read's work counter
   float* pf_out;             // prefill: FP32 branch outputs [2][T][4096]
   uint16_t* o_sum;
   size_t bytes;
@@ -61,6 +62,7 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   w.chunk_v = prefill ? c.take<uint16_t>((size_t)NG * nq * D) : nullptr;
   w.part_o = prefill ? nullptr : c.take<float>(attend_part_floats(nq));
   w.part_ml = prefill ? nullptr : c.take<float>(attend_ml_floats(nq));
+  w.sched = prefill ? nullptr : c.take<int>(1);
   w.pf_out = prefill ? c.take<float>(prefill_out_floats(nq)) : nullptr;
   w.o_sum = c.take<uint16_t>((size_t)nq * OIN);
   w.bytes = c.used();
@@ -160,6 +162,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   pp.meta = st->meta; pp.seq_ids = seq_ids; pp.s_max = st->s_max; pp.L = st->n_layers;
   pp.layer = layer; pp.prefill = prefill ? 1 : 0; pp.seq_fixed = seq_fixed;
   pp.chunk_k = W.chunk_k; pp.chunk_v = W.chunk_v; pp.err = st->dev_error;
+  pp.sched_reset = W.sched;
   if ((rc = launch_post_proj(pp, rma_off, s)) != ER_OK) return rc;
   // a5 / a8: both reads, merged into bf16(o_swa + o_rma)
   if (prefill) {
@@ -173,8 +176,9 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
     ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
     ap.prefill = 0; ap.seq_fixed = -1; ap.rma_off = rma_off ? 1 : 0;
-    ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.err = st->dev_error;
-    if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, s)) != ER_OK) return rc;
+    ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.sched = W.sched; ap.err = st->dev_error;
+    // k_post_proj above zeroed the work counter
+    if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s)) != ER_OK) return rc;
   }
   // a7: commit this layer where the block is now full (decided on the device),
   // beside a6, the shared o_proj (disjoint data)

@@ -112,6 +112,9 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   const int lane = threadIdx.x & 31;
   const int hs = blockIdx.y * 8 + (threadIdx.x >> 5);
   const int qi = blockIdx.x;
+  // the read that follows takes its work units from this counter; it waits for
+  // this kernel to complete before the first one
+  if (P.sched_reset && qi == 0 && hs == 0 && lane == 0) *P.sched_reset = 0;
   const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
   if (seq < 0 || seq >= P.s_max) {  // the same for the whole block
     if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);

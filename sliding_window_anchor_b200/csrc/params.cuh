@@ -25,6 +25,7 @@ struct PostParams {
   int prefill;                 // 0: token b of sequence seq_ids[b]; 1: token i of seq_fixed
   int seq_fixed;
   uint16_t *chunk_k, *chunk_v; // prefill: [4][nq][256] window rows of the chunk
+  int* sched_reset;            // decode: the read's work counter, zeroed here (or NULL)
   int32_t* err;
 };
 
@@ -54,6 +55,7 @@ struct AttendParams {
   float *o_swa, *o_rma;  // FP32 [nq][16][256] (standalone read), or
   uint16_t* o_sum;       // BF16 [nq][4096] = bf16(o_swa + o_rma) (layer path)
   int rma_off;           // the RMA read sees no records (o_rma = 0)
+  int* sched;            // work counter, 0 at launch (the CTAs take units from it)
   int32_t* err;
 };
 
