@@ -50,10 +50,11 @@ def parse():
     ap.add_argument("--prefill-chunks", type=int, default=512,
                     help="256-token chunks of the prefill stream (512 = 131072 tokens)")
     ap.add_argument("--kernel", default="step",
-                    choices=["step", "attend", "commit", "prefill", "score"],
+                    choices=["step", "attend", "commit", "prefill", "score", "layer"],
                     help="step: the benchmark; attend/commit: one kernel alone at --batch "
                          "sequences; score: the scorer on --batch tokens; prefill: "
-                         "--prefill-chunks chunks of one layer (profiling drivers)")
+                         "--prefill-chunks chunks of one layer; layer: one decode layer "
+                         "call at --batch sequences (profiling drivers)")
     ap.add_argument("--batch", type=int, default=256)
     ap.add_argument("--sweep", action="store_true",
                     help="layer-level batch sweep B = 1..512 (one JSON line per batch size)")
@@ -707,6 +708,32 @@ def single_kernel(args):
     elif args.kernel == "prefill":
         out = {"kernel": "prefill", **prefill_bench(dev, args.prefill_chunks, layers=1,
                                                     warm_chunks=1)}
+    elif args.kernel == "layer":
+        # the decode workload's state for one layer (t0 = 32768, pending U{0..255})
+        seed = wl.seed_of(3)
+        w = sab.LayerWeights.from_dict(wl.make_weights(seed, 0, device=dev))
+        st = sab.State(B, 1, device=dev)
+        nr = lambda x, g, p: sab.qk_norm_rope(x.contiguous(), g, p.to(torch.int32).contiguous())
+        wl.seed_state(st.arrays(), range(B), 1, T0, "uniform", seed, [w.t], nr, device=dev)
+        ids = torch.arange(B, dtype=torch.int32, device=dev)
+        ws = torch.empty(sab.decode_workspace_bytes(B), dtype=torch.uint8, device=dev)
+        xs = [wl.make_x(seed, 0, s, range(B), device=dev) for s in range(2)]
+        y = torch.empty(B, 2560, dtype=torch.bfloat16, device=dev)
+        ms = []
+        for i in range(7):  # the first is a warm-up
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sab.swa_rma_decode(st, w, 0, ids, xs[i % 2], out=y, ws=ws)
+            e1.record()
+            sab.advance(st, ids)
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        if sab.last_device_error(st) != 0:
+            raise RuntimeError("device error")
+        med = sorted(ms[1:])[len(ms[1:]) // 2]
+        out = {"kernel": "layer", "batch": B, "layers": 1, "ms": med,
+               "ms_calls": [round(m, 4) for m in ms[1:]],
+               "note": "one decode layer call (a1-a7) per timed region, eager; median of 6"}
     else:
         st = sab.State(B, LAYERS)
         r = commit_microbench(st, dev, reps=2)

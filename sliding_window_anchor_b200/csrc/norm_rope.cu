@@ -8,9 +8,10 @@
 //
 // One warp owns one 256-wide head vector, 8 BF16 values per lane (one 16-byte
 // load); lanes 0..7 hold the rotated dims and exchange pairs with xor 4.  The
-// rotation angle pos * 1e7^(-2i/64) is formed and reduced in float64 so that
-// positions up to 2^18 keep full angle accuracy (once per token in the layer
-// kernel, shared by its head vectors); the rotation itself is fp32.
+// rotation angle pos * 1e7^(-2i/64) is formed and reduced (to [-1/2, 1/2] turn)
+// in float64 so that positions up to 2^18 keep full angle accuracy (once per
+// token in the layer kernel, shared by its head vectors); the rotation itself
+// is fp32.
 #include "common.cuh"
 #include "params.cuh"
 
@@ -30,13 +31,36 @@ __device__ __forceinline__ void store8(uint16_t* dst, const float v[8]) {
   *reinterpret_cast<uint4*>(dst) = w;
 }
 
-// cos/sin of pos * 1e7^(-2i/64) for i = lane (0..31): the angle is formed and
-// reduced in float64 (one evaluation per lane), then rounded to float.
+// Turns per position of rotary frequency i: 1e7^(-2i/64) / (2 pi), i = 0..31,
+// each the float64 nearest to the real value (printed to 17 digits).
+__device__ const double kTurnsPerPos[32] = {
+    0.15915494309189535, 0.09617675759898782,
+    0.058119267441876246, 0.03512126351841045,
+    0.02122365276477766, 0.012825376753422709,
+    0.0077503288755374055, 0.004683495762645621,
+    0.00283021958306234, 0.0017102914776258452,
+    0.0010335229661843405, 0.0006245541976934049,
+    0.00037741584717419774, 0.00022807103406603446,
+    0.00013782250260398286, 8.32856408171725e-05,
+    5.0329212104487035e-05, 3.0413761198270857e-05,
+    1.8378926105679668e-05, 1.1106318702115607e-05,
+    6.711508300522725e-06, 4.055740239059148e-06,
+    2.450869186206985e-06, 1.4810514021707515e-06,
+    8.949940160889103e-07, 5.408416532072578e-07,
+    3.2682865872357e-07, 1.9750137869302395e-07,
+    1.1934937021124886e-07, 7.212239359585222e-08,
+    4.358330210530733e-08, 2.6337232136895232e-08,
+};
+
+// cos/sin of pos * 1e7^(-2i/64) for i = lane (0..31).  The angle is formed in
+// turns in float64 and reduced there to [-1/2, 1/2] turn (for pos < 2^18 the
+// product is within ~1e-11 turn), so the float64 sincospi that evaluates it
+// never needs a large-argument reduction; the results are rounded to float.
 __device__ __forceinline__ float2 rope_cs_lane(int32_t pos, int lane) {
-  const double kLog2Theta = 23.253496664211536;  // log2(1e7)
-  const double inv_freq = exp2(-(double)lane * (kLog2Theta / 32.0));
+  const double turns = (double)pos * kTurnsPerPos[lane];
+  const double red = turns - rint(turns);
   double sn, cs;
-  sincos((double)pos * inv_freq, &sn, &cs);
+  sincospi(2.0 * red, &sn, &cs);
   return make_float2((float)cs, (float)sn);
 }
 
@@ -104,54 +128,22 @@ __global__ void k_norm_rope(const uint16_t* x, uint16_t* y, int64_t n_rows, cons
 }  // namespace
 
 
-// Grid (nq, 6) x 256 threads: warp slot hs = 0..47 covers, per token,
-// q_swa 0..15 | k_swa 16..19 | v_swa 20..23 | q_rma 24..39 | k_rma 40..43 | v_rma 44..47.
-__global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
-  __shared__ float2 s_cs[32];  // the rotation of this token's position, formed once
-  grid_dep_trigger();  // a prefill read may set itself up meanwhile (it waits for us)
-  const int lane = threadIdx.x & 31;
-  const int hs = blockIdx.y * 8 + (threadIdx.x >> 5);
-  const int qi = blockIdx.x;
-  // the read that follows takes its work units from this counter; it waits for
-  // this kernel to complete before the first one
-  if (P.sched_reset && qi == 0 && hs == 0 && lane == 0) *P.sched_reset = 0;
-  const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
-  if (seq < 0 || seq >= P.s_max) {  // the same for the whole block
-    if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);
-    return;
-  }
-  const int32_t pos0 = P.meta[seq * 4 + 0];
-  const int32_t pend0 = P.meta[seq * 4 + 1];
-  const int32_t t = pos0 + (P.prefill ? qi : 0);
-  if (threadIdx.x < 32) s_cs[lane] = rope_cs_lane(t, lane);
-  __syncthreads();
-  // launched behind the scorer / the projection GEMM: the angles above used only
-  // metadata; the projections and the partial scores come from them
-  grid_dep_wait();
-  const int p_idx = pend0 + (P.prefill ? qi : 0);
-  const bool state_ok = p_idx >= 0 && p_idx < PEND && t >= 0;
-  if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
+// Grid (nq, 6) x 256 threads: warp slot hs = 8 blockIdx.y + warp covers, per
+// token, q_swa 0..15 | k_swa 16..19 | v_swa 20..23 | q_rma 24..39 | k_rma 40..43
+// | v_rma 44..47 (blockIdx.y < 3 only with the RMA off).  A one-block-per-token
+// layout with six rows per warp was measured slower (its rows' norm/RoPE chains
+// run in series, at half the resident warps).
+namespace {
 
-  int col;
+// One head row: norm + RoPE where it has a gain, then its destination.
+__device__ __forceinline__ void post_row(const PostParams& P, int hs, int lane, int qi, int seq,
+                                         int32_t t, int p_idx, bool state_ok,
+                                         const float2* s_cs, float v[8]) {
   const uint16_t* gain = nullptr;
-  if (hs < 16) { col = OFF_Q_SWA + hs * D; gain = P.gq_swa; }
-  else if (hs < 20) { col = OFF_K_SWA + (hs - 16) * D; gain = P.gk_swa; }
-  else if (hs < 24) { col = OFF_V_SWA + (hs - 20) * D; }
-  else if (hs < 40) { col = OFF_Q_RMA + (hs - 24) * D; gain = P.gq_rma; }
-  else if (hs < 44) { col = OFF_K_RMA + (hs - 40) * D; gain = P.gk_rma; }
-  else { col = OFF_V_RMA + (hs - 44) * D; }
-
-  float v[8];
-  if (P.proj_f32) {
-    // FP32 sums of the fused GEMM, rounded to BF16 as a BF16-output GEMM would
-    const float4* src = reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + col) +
-                        lane * 2;
-    const float4 a = src[0], b = src[1];
-    v[0] = bf1(f2bf(a.x)); v[1] = bf1(f2bf(a.y)); v[2] = bf1(f2bf(a.z)); v[3] = bf1(f2bf(a.w));
-    v[4] = bf1(f2bf(b.x)); v[5] = bf1(f2bf(b.y)); v[6] = bf1(f2bf(b.z)); v[7] = bf1(f2bf(b.w));
-  } else {
-    load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
-  }
+  if (hs < 16) gain = P.gq_swa;
+  else if (hs < 20) gain = P.gk_swa;
+  else if (hs >= 24 && hs < 40) gain = P.gq_rma;
+  else if (hs >= 40 && hs < 44) gain = P.gk_rma;
   if (gain) norm_rope_lane_cs(v, gain, s_cs, lane);
 
   uint16_t* dst = nullptr;
@@ -207,9 +199,74 @@ __global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
   store8(dst + lane * 8, v);
 }
 
-// Grid rows 0-2 hold the SWA head slots (q, k, v), rows 3-5 the RMA ones
-// (q, k and v with the pending append); with the RMA switched off only the
-// first three run.
+// Column of head row hs inside a projection row.
+__device__ __forceinline__ int row_col(int hs) {
+  if (hs < 16) return OFF_Q_SWA + hs * D;
+  if (hs < 20) return OFF_K_SWA + (hs - 16) * D;
+  if (hs < 24) return OFF_V_SWA + (hs - 20) * D;
+  if (hs < 40) return OFF_Q_RMA + (hs - 24) * D;
+  if (hs < 44) return OFF_K_RMA + (hs - 40) * D;
+  return OFF_V_RMA + (hs - 44) * D;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
+  __shared__ float2 s_cs[32];  // the rotation of this token's position
+  __shared__ int s_tok[4];     // seq, t, p_idx, valid
+  grid_dep_trigger();  // a prefill read may set itself up meanwhile (it waits for us)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int hs = blockIdx.y * 8 + warp;
+  const int qi = blockIdx.x;
+  // the read that follows takes its work units from this counter; it waits for
+  // this kernel to complete before the first one
+  if (P.sched_reset && qi == 0 && hs == 0 && lane == 0) *P.sched_reset = 0;
+  if (warp == 0) {
+    // metadata only (written before the kernel this one is launched behind)
+    const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
+    const bool valid = seq >= 0 && seq < P.s_max;
+    int32_t t = 0, p_idx = 0;
+    if (valid) {
+      t = P.meta[seq * 4 + 0] + (P.prefill ? qi : 0);
+      p_idx = P.meta[seq * 4 + 1] + (P.prefill ? qi : 0);
+    }
+    s_cs[lane] = rope_cs_lane(t, lane);
+    if (lane == 0) {
+      s_tok[0] = seq;
+      s_tok[1] = t;
+      s_tok[2] = p_idx;
+      s_tok[3] = valid ? 1 : 0;
+    }
+  }
+  // launched behind the scorer / the projection GEMM: the projections and the
+  // partial scores come from them.  The row is loaded before the barrier so that
+  // its latency overlaps warp 0's metadata and rotations.
+  grid_dep_wait();
+  float v[8];
+  const int col = row_col(hs);
+  if (P.proj_f32) {
+    // FP32 sums of the fused GEMM, rounded to BF16 as a BF16-output GEMM would
+    const float4* src =
+        reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + col) + lane * 2;
+    const float4 a = src[0], b = src[1];
+    v[0] = bf1(f2bf(a.x)); v[1] = bf1(f2bf(a.y)); v[2] = bf1(f2bf(a.z)); v[3] = bf1(f2bf(a.w));
+    v[4] = bf1(f2bf(b.x)); v[5] = bf1(f2bf(b.y)); v[6] = bf1(f2bf(b.z)); v[7] = bf1(f2bf(b.w));
+  } else {
+    load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
+  }
+  __syncthreads();
+  if (!s_tok[3]) {  // the same for the whole block
+    if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);
+    return;
+  }
+  const int seq = s_tok[0];
+  const int32_t t = s_tok[1];
+  const int p_idx = s_tok[2];
+  const bool state_ok = p_idx >= 0 && p_idx < PEND && t >= 0;
+  if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
+  post_row(P, hs, lane, qi, seq, t, p_idx, state_ok, s_cs, v);
+}
+
 int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st) {
   if (P.nq <= 0) return ER_OK;
   // a programmatic launch (see grid_dep_wait above)
