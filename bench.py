@@ -784,6 +784,36 @@ def oracle_tokens_per_s(budget_s=12.0, max_threads=8):
     return sum(counts) / dt, threads, sum(counts), dt
 
 
+def oracle_merges_per_s(budget_s=4.0):
+    """The oracle's commit (a full sort of the 1280 records, then the moves) on the
+    commit workload, one thread: one sequence x 8 layers x 4 groups per call, the
+    pending block re-filled (scores with ~5% ties, fresh positions) before each."""
+    import torch
+    import oracle
+    import synth
+    from synth import workloads as wl
+    seed = wl.seed_of(1)
+    ost = oracle.OracleState(1, LAYERS)
+    arrays = {n: getattr(ost, n) for n in oracle.OracleState.ARRAYS}
+    wl.seed_state(arrays, [0], LAYERS, T0, "full", seed, [None] * LAYERS, None, device="cpu",
+                  plain_keys=True, dup_scores=True)
+    j = torch.arange(256, dtype=torch.int32)
+    merges, spent, rep = 0, 0.0, 0
+    while spent < budget_s:
+        if rep > 0:
+            synth.fill_normal_dup_(ost.pend_score, seed + rep, synth.PEND_SCORE, 256, 20)
+        ost.pend_pos.copy_((T0 + 256 * rep + j).view(1, 1, 1, 256).expand_as(ost.pend_pos))
+        ost.meta[0, 0] = T0 + 256 * (rep + 1)
+        ost.meta[0, 1] = 256
+        ost.meta[0, 2] = 1024
+        t0 = time.time()
+        ost.commit(-1, 0)
+        spent += time.time() - t0
+        merges += LAYERS * 4
+        rep += 1
+    return merges / spent, merges, spent
+
+
 def workload_config(world: int, launch: str) -> dict:
     """The workload both arms report (the reference arm's launch is the host)."""
     return {"workload": WORKLOAD, "B": B, "layers": LAYERS, "t0": T0,
@@ -857,9 +887,17 @@ def main():
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         v, cores, toks, dt = oracle_tokens_per_s(budget_s=12.0)
+        v1, _, toks1, dt1 = oracle_tokens_per_s(budget_s=6.0, max_threads=1)
+        mps, merges, mdt = oracle_merges_per_s(budget_s=4.0)
         cpu = {"value": v, "unit": "tok/s", "cores": cores, "kind": "oracle",
                "sample": f"{toks} whole 8-layer decode steps of {cores} sequences of the "
-                         f"workload in {dt:.1f} s"}
+                         f"workload in {dt:.1f} s",
+               "single_thread": {"value": v1, "unit": "tok/s", "cores": 1,
+                                 "sample": f"{toks1} whole 8-layer decode steps of one "
+                                           f"sequence in {dt1:.1f} s"},
+               "commit": {"value": mps, "unit": "merges/s", "cores": 1,
+                          "sample": f"{merges} merges of the commit workload (top 1024 of "
+                                    f"1280 by full sort, then the moves) in {mdt:.1f} s"}}
     # headline: the steps replayed from CUDA graphs when that pass ran, else the eager pass
     g = r["graph"]
     head_ms = g["ms"] if g else r["ms"]
