@@ -182,6 +182,15 @@ int er_advance_ex(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t
  * `stream`.  Returns ER_OK when the word was 0, else ER_EDEVICE. */
 int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream);
 
+/* Diagnostic for the failure path, no part of the method: one thread waits on
+ * a fresh mbarrier (one expected arrival) through the bounded wait that every
+ * kernel of the library uses for its pipeline barriers.  arrive = 1 completes
+ * the barrier first (the wait returns at once, nothing is recorded); arrive =
+ * 0 leaves it incomplete, so the wait gives up after ~2 s and records
+ * ER_ETIMEOUT in st's device error word; the kernel then exits and the context
+ * stays usable.  ER_EINVAL for a NULL state or another arrive value. */
+int er_wait_selftest(const er_state* st, int32_t arrive, er_stream_t stream);
+
 /* ------------------------------------------------------- hot-path steps */
 
 /* a2 — RMS-norm with gain, then rotary embedding of dims [0, 64) at each

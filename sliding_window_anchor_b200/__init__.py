@@ -149,6 +149,13 @@ def last_device_error(st: State, stream=None) -> int:
     return int(code.value)
 
 
+def wait_selftest(st: State, arrive: bool, stream=None):
+    """er_wait_selftest: a bounded device wait that completes (arrive=True) or
+    runs out (~2 s, ER_ETIMEOUT in the state's error word)."""
+    check("er_wait_selftest", lib().er_wait_selftest(st.ptr(), 1 if arrive else 0,
+                                                     stream_handle(stream, st.device)))
+
+
 def qk_norm_rope(x: torch.Tensor, gain: torch.Tensor, pos: torch.Tensor, out=None, stream=None):
     rows = x.numel() // D
     out = torch.empty_like(x) if out is None else out

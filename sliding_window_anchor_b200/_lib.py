@@ -60,6 +60,7 @@ EXPORTS = {
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "er_score_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "er_score_split_w1": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "er_wait_selftest": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_int32, ctypes.c_void_p]),
     "er_prepare_qkv_score": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                             ctypes.c_void_p]),
     "er_rma_score": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p, ctypes.c_int32,

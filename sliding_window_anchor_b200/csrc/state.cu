@@ -151,11 +151,30 @@ void profile_end(cudaStream_t st, std::pair<cudaEvent_t, cudaEvent_t> ev) {
   p.pending.push_back(ev);
 }
 
+// One thread waits on a fresh one-arrival mbarrier through the bounded wait
+// every kernel of the library uses; with arrive = 0 nothing completes the
+// barrier, so the wait must give up (~2 s) and record ER_ETIMEOUT.
+__global__ void k_wait_selftest(int32_t* err, int arrive) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbar_init();
+  if (arrive) mbar_arrive(&bar);
+  mbar_wait(&bar, 0, err);
+}
+
 }  // namespace er
 
 using namespace er;
 
 extern "C" {
+
+int er_wait_selftest(const er_state* st, int32_t arrive, er_stream_t stream) {
+  if (!st || !st->dev_error || (arrive != 0 && arrive != 1)) return ER_EINVAL;
+  k_wait_selftest<<<1, 32, 0, (cudaStream_t)stream>>>(st->dev_error, arrive);
+  count_launches(1);
+  return launch_status();
+}
 
 size_t er_state_bytes(int32_t s_max, int32_t n_layers) {
   StateLayout L;

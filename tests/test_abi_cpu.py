@@ -130,6 +130,11 @@ def test_host_validation_rejects_before_enqueue(L):
     assert L.er_swa_rma_prefill_chunk_ex(ctypes.byref(st), ctypes.byref(w), 0, 0, nul, 16, nul,
                                          nul, 0, 8, nul) == -1
     assert L.er_launch_count() == before
+    # the bounded-wait diagnostic: only arrive 0 or 1, and a state
+    before = L.er_launch_count()
+    assert L.er_wait_selftest(None, 0, nul) == -1
+    assert L.er_wait_selftest(ctypes.byref(st), 2, nul) == -1
+    assert L.er_launch_count() == before
     # the fused q/k/v + W1-term weights: NULL, unaligned or overlapping buffers are refused
     base = 1 << 40
     qkv_bytes = 12288 * 2560 * 2

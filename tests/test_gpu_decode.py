@@ -12,6 +12,7 @@ import pytest
 import torch
 
 import oracle
+import synth
 from synth import workloads as wl
 from tests import helpers as H
 
@@ -203,6 +204,32 @@ def test_out_of_range_sequence_is_recorded_not_faulted(sab):
     st.meta[1, 1] = 256
     sab.swa_rma_decode(st, gw, 0, [0, 1], x)
     assert sab.last_device_error(st) == -2
+
+
+def test_bounded_wait_runs_out_and_the_context_survives(sab):
+    """The failure path of every pipeline barrier: a wait that nothing completes
+    gives up after ~2 s, records ER_ETIMEOUT and returns; afterwards the context
+    runs the library's kernels normally (no fault, no hang)."""
+    import time
+    st = sab.State(1, 1)
+    sab.state_init(st, [0])
+    assert sab.last_device_error(st) == 0
+    sab.wait_selftest(st, arrive=True)  # a completed barrier: nothing recorded
+    assert sab.last_device_error(st) == 0
+    t0 = time.time()
+    sab.wait_selftest(st, arrive=False)
+    code = sab.last_device_error(st)
+    waited = time.time() - t0
+    assert code == -5, code  # ER_ETIMEOUT
+    assert 1.5 < waited < 30.0, waited
+    # the context is intact: norm/RoPE through the library still matches the oracle
+    x = synth.normal((64, 256), 9, synth.MISC, torch.bfloat16)
+    g = synth.normal((256,), 9, synth.MISC + 1, torch.bfloat16, scale=0.1, offset=1.0)
+    pos = torch.arange(64, dtype=torch.int32) * 977
+    got = sab.qk_norm_rope(x.cuda(), g.cuda(), pos.cuda()).cpu()
+    ref = oracle.norm_rope(x, g, pos)
+    assert (got == ref).double().mean() > 0.99
+    assert sab.last_device_error(st) == 0
 
 
 RMA_ARRAYS = ("bank_k", "bank_v", "pend_k", "pend_v", "bank_score", "pend_score", "bank_pos",
