@@ -6,13 +6,14 @@
 // this library: the RMA read is its own softmax over committed + pending
 // records, with its own q, added to the SWA output before o_proj.
 //
-// Work item = (query, KV group, branch, split).  A branch's rows are one to
-// three contiguous ranges of 512-byte K rows and V rows (window ring pieces,
-// the chunk's own rows in prefill, bank, pending); they stream through shared
-// memory in 64-row tiles.
+// Work item = (query, KV group, branch, split).  A branch's rows are one or two
+// contiguous ranges of 512-byte K rows and V rows (the window ring; bank and
+// pending); they stream through shared memory in 64-row tiles.  (A prefill
+// chunk's reads run in prefill_attn.cu.)
 //
 // Persistent kernel, one 160-thread CTA per SM:
-//   warp 4 (producer): lane 0 walks the CTA's items; for each tile it arms the
+//   warp 4 (producer): lane 0 takes the CTA's items from a work counter; for
+//     each tile it arms the
 //     stage's mbarrier with the transaction bytes and issues TMA tensor copies
 //     (cp.async.bulk.tensor.2d, no multicast) of four 64x64 boxes of K rows and
 //     four of V rows, 128-byte swizzled, plus the item's 4 query heads (one
@@ -90,9 +91,9 @@ struct Range {
   int rows;
 };
 
-// Row ranges of one item; returns the number of ranges (0..3), none empty.
-__device__ int item_ranges(const AttendParams& P, int qi, int g, int br, Range r[3]) {
-  const int seq = P.prefill ? P.seq_fixed : P.seq_ids[qi];
+// Row ranges of one item; returns the number of ranges (0..2), none empty.
+__device__ int item_ranges(const AttendParams& P, int qi, int g, int br, Range r[2]) {
+  const int seq = P.seq_ids[qi];
   if (seq < 0 || seq >= P.s_max) return 0;
   const int32_t pos0 = P.meta[seq * 4 + 0];
   const int pend = P.meta[seq * 4 + 1];
@@ -100,28 +101,14 @@ __device__ int item_ranges(const AttendParams& P, int qi, int g, int br, Range r
   const int gi = (int)grp(seq, P.layer, g, P.L);
   int n = 0;
   if (br == 0) {
-    const int w0 = gi * WIN;  // first ring row of this (sequence, layer, group)
-    if (!P.prefill) {
-      // window positions [t-1023, t], t = pos0, all already in the ring
-      const int nwin = min(pos0 + 1, WIN);
-      if (nwin > 0) r[n++] = Range{TM_WIN, w0, nwin};
-    } else {
-      const int t = pos0 + qi;
-      if (t < 0) return 0;
-      const int lo = max(0, t - (WIN - 1));
-      const int count = pos0 - lo;  // old ring positions lo..pos0-1
-      if (count > 0) {
-        const int s0 = lo % WIN;
-        const int n1 = min(count, WIN - s0);
-        r[n++] = Range{TM_WIN, w0 + s0, n1};
-        if (count > n1) r[n++] = Range{TM_WIN, w0, count - n1};
-      }
-      r[n++] = Range{TM_CHUNK, g * P.nq, qi + 1};
-    }
+    // window positions [t-1023, t], t = pos0, all already in the ring (the
+    // softmax does not depend on their order, so the ring is read as stored)
+    const int nwin = min(pos0 + 1, WIN);
+    if (nwin > 0) r[n++] = Range{TM_WIN, gi * WIN, nwin};
   } else {
     if (P.rma_off) return 0;  // the RMA switched off: an empty read, o_rma = 0
     if (bank > 0) r[n++] = Range{TM_BANK, gi * BANK, bank};
-    const int np = min(pend + (P.prefill ? qi : 0) + 1, PEND);
+    const int np = min(pend + 1, PEND);
     if (np > 0) r[n++] = Range{TM_PEND, gi * PEND, np};
   }
   return n;
@@ -147,7 +134,7 @@ struct Tile {
 struct TileIter {
   const AttendParams* P;
   int item, item_end;
-  Range r[3];
+  Range r[2];
   int nr, ri, tile_in_range, e, emit, qi, g, br;
   bool has_rows;
 
@@ -672,13 +659,6 @@ int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* 
             encode_rows(&P.tmap_v[TM_BANK], P.bank_v, groups * BANK) &&
             encode_rows(&P.tmap_k[TM_PEND], P.pend_k, groups * PEND) &&
             encode_rows(&P.tmap_v[TM_PEND], P.pend_v, groups * PEND);
-  if (P.prefill) {
-    ok = ok && encode_rows(&P.tmap_k[TM_CHUNK], P.chunk_k, (uint64_t)NG * P.nq) &&
-         encode_rows(&P.tmap_v[TM_CHUNK], P.chunk_v, (uint64_t)NG * P.nq);
-  } else {
-    P.tmap_k[TM_CHUNK] = P.tmap_k[TM_WIN];
-    P.tmap_v[TM_CHUNK] = P.tmap_v[TM_WIN];
-  }
   if (!ok) return ER_ECUDA;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -755,7 +735,7 @@ int er_swa_rma_attend(const er_state* st, int32_t layer, const int32_t* seq_ids,
   P.pend_k = st->pend_k; P.pend_v = st->pend_v;
   P.meta = st->meta; P.seq_ids = seq_ids;
   P.s_max = st->s_max; P.L = st->n_layers; P.layer = layer;
-  P.q_swa = q_swa; P.q_rma = q_rma; P.nq = B; P.prefill = 0;
+  P.q_swa = q_swa; P.q_rma = q_rma; P.nq = B;
   P.part_o = c.take<float>(attend_part_floats(B));
   P.part_ml = c.take<float>(attend_ml_floats(B));
   P.sched = c.take<int>(1);

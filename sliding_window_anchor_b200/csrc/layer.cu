@@ -175,7 +175,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     ap.pend_k = st->pend_k; ap.pend_v = st->pend_v; ap.meta = st->meta; ap.seq_ids = seq_ids;
     ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
     ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
-    ap.prefill = 0; ap.seq_fixed = -1; ap.rma_off = rma_off ? 1 : 0;
+    ap.rma_off = rma_off ? 1 : 0;
     ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.sched = W.sched; ap.err = st->dev_error;
     // k_post_proj above zeroed the work counter
     if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s)) != ER_OK) return rc;

@@ -29,9 +29,9 @@ struct PostParams {
   int32_t* err;
 };
 
-// Tensor maps of the row arrays the reads stream (2-D views [rows][256] BF16,
-// 64x64 boxes, 128-byte swizzle): K and V of window, bank, pending, chunk.
-enum { TM_WIN = 0, TM_BANK = 1, TM_PEND = 2, TM_CHUNK = 3, TM_COUNT = 4 };
+// Tensor maps of the row arrays the decode read streams (2-D views [rows][256]
+// BF16, 64x64 boxes, 128-byte swizzle): K and V of window, bank, pending.
+enum { TM_WIN = 0, TM_BANK = 1, TM_PEND = 2, TM_COUNT = 3 };
 
 struct AttendParams {
   CUtensorMap tmap_k[TM_COUNT];
@@ -42,10 +42,7 @@ struct AttendParams {
   int s_max, L, layer;
   const uint16_t* q_swa;  // [nq][16][256], normed and rotated
   const uint16_t* q_rma;  // [nq][16][256]
-  int nq;
-  int prefill;        // 0: query b = sequence seq_ids[b] at meta pos; 1: token b of seq_fixed
-  int seq_fixed;
-  const uint16_t *chunk_k, *chunk_v;  // prefill: [4][nq][256]
+  int nq;                 // query b = the token of sequence seq_ids[b] at its meta pos
   int splits;
   float* part_o;   // [items][4][256]
   float* part_ml;  // [items][4][2]
