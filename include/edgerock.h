@@ -28,13 +28,17 @@
  *  - Pointers named in a signature are DEVICE pointers unless marked (host).
  *    The caller allocates and frees all memory (state, weights, inputs,
  *    outputs, workspace); the library never allocates or frees device memory
- *    and never synchronises the stream, except er_last_device_error, which
- *    reads one word back.
+ *    itself (cuBLAS keeps its own handle memory; er_rma_score_noalloc's
+ *    scratch is a static device array) and never synchronises the stream,
+ *    except er_last_device_error, which reads one word back.
  *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  A
  *    layer call may also run part of its work (the commit, beside o_proj) on
  *    a side stream the library keeps per device, forked from and joined back
  *    to `stream` inside the call, so everything still completes in `stream`
- *    order and the call can be captured in a CUDA graph.
+ *    order and the call can be captured in a CUDA graph.  The first layer
+ *    call (and the first read or scorer call) on a device creates that
+ *    device's library resources (cuBLAS handle, side stream, events, kernel
+ *    attributes): make one such call before capturing on the device.
  *  - Return value: ER_OK, or a negative ER_E* code.  Host-side argument checks
  *    happen before anything is enqueued; a failed check enqueues nothing.
  *    Conditions only the device can see (a sequence id out of range, a full

@@ -660,14 +660,19 @@ int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* 
             encode_rows(&P.tmap_k[TM_PEND], P.pend_k, groups * PEND) &&
             encode_rows(&P.tmap_v[TM_PEND], P.pend_v, groups * PEND);
   if (!ok) return ER_ECUDA;
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(k_attend, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sizeof(AttnSmem) + 1024) != cudaSuccess)
-      return ER_ECUDA;
-    attr_done[dev] = true;
+  {
+    // the shared-memory opt-in, once per device (calls may come from several threads)
+    static std::mutex mu;
+    static bool attr_done[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ER_ECUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(k_attend, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)sizeof(AttnSmem) + 1024) != cudaSuccess)
+        return ER_ECUDA;
+      attr_done[dev] = true;
+    }
   }
   const int n_items = P.nq * NG * 2 * P.splits;
   const int grid = min(n_items, num_sms());
