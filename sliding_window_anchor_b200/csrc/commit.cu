@@ -22,7 +22,9 @@
 //     their target slots, with the score and position, four rows in flight.
 // Launches with few merges run as clusters of 8 CTAs that repeat steps 1-3
 // and split step 4 (a cluster barrier keeps every key read ahead of the first
-// bank write).
+// bank write).  The layer calls split the commit in two launches instead:
+// steps 1-3 (k_commit_plan) while the read runs, step 4 (k_commit_move) after
+// it.
 // Surviving anchors are not touched, so the write traffic is only the moved
 // records.
 #include "common.cuh"
@@ -229,6 +231,135 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
+// Step 2 in the select form (no ranked list wanted): flag[i] = 1 for the K
+// kept records (bank i < c, pending BANK + j, j < p).  flag must be cleared
+// and synchronised before; every thread of the block calls it.
+__device__ void select_kept(const CommitParams& P, size_t gi, int c, int p, int K, uint8_t* flag,
+                            int* hist, int* warp_sums, int* sel) {
+  const int tid = threadIdx.x;
+  uint64_t key5[5];  // records tid + 256*q (bank 0..1023, then pending)
+#pragma unroll
+  for (int q = 0; q < 5; ++q) {
+    const int i = tid + CT * q;
+    uint64_t kv = 0;
+    if (i < BANK) {
+      if (i < c) kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
+    } else if (i - BANK < p) {
+      kv = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
+    }
+    key5[q] = kv;
+  }
+  uint64_t prefix = 0;
+  int shift = 64;
+  if (c + p > BANK) radix_select(key5, K, hist, warp_sums, sel, &prefix, &shift);
+#pragma unroll
+  for (int q = 0; q < 5; ++q)
+    if (key5[q] != 0 && (shift >= 64 || (key5[q] >> shift) >= (prefix >> shift)))
+      flag[tid + CT * q] = 1;
+}
+
+// Step 3: from the kept flags (synchronised), the move list: winner w, in
+// ascending pending index, goes from pending slot move_src[w] to the w-th
+// evicted bank slot (ascending), or past the bank's end while it is not full.
+// Returns the number of winners; the lists are synchronised on return.
+__device__ int plan_moves(int c, int p, const uint8_t* flag, int16_t* evict_list,
+                          int16_t* move_src, int16_t* move_dst, int* warp_sums) {
+  const int tid = threadIdx.x;
+  int ev[4], nev = 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int slot = tid * 4 + q;
+    ev[q] = (slot < c && !flag[slot]) ? 1 : 0;
+    nev += ev[q];
+  }
+  int total_evict = 0;
+  int er = block_scan_excl(nev, warp_sums, &total_evict);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (ev[q]) evict_list[er++] = (int16_t)(tid * 4 + q);
+  int total_win = 0;
+  const int wn = (tid < p && flag[BANK + tid]) ? 1 : 0;
+  const int w_rank = block_scan_excl(wn, warp_sums, &total_win);
+  __syncthreads();
+  if (wn) {
+    const int dst = w_rank < total_evict ? (int)evict_list[w_rank] : c + (w_rank - total_evict);
+    move_src[w_rank] = (int16_t)tid;
+    move_dst[w_rank] = (int16_t)dst;
+  }
+  __syncthreads();
+  return total_win;
+}
+
+// Step 4 for the winners this block's warps own: warp `mover` of `movers`
+// takes winners mover, mover + movers, ...; 16 bytes per lane per row, MV rows
+// per warp in flight (every load issued before the first store).  The lists
+// are in shared memory.
+__device__ void move_winners(const CommitParams& P, size_t gi, int total_win,
+                             const int16_t* move_src, const int16_t* move_dst, int mover,
+                             int movers) {
+  constexpr int MV = 4;
+  const int lane = threadIdx.x & 31;
+  for (int w0 = mover; w0 < total_win; w0 += MV * movers) {
+    uint4 kr[MV], vr[MV];
+    int src[MV];
+#pragma unroll
+    for (int q = 0; q < MV; ++q) {
+      const int w = w0 + q * movers;
+      src[q] = w < total_win ? (int)move_src[w] : -1;
+      kr[q] = vr[q] = make_uint4(0, 0, 0, 0);
+      if (src[q] >= 0) {
+        kr[q] = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + src[q]) * D)[lane];
+        vr[q] = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + src[q]) * D)[lane];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < MV; ++q) {
+      if (src[q] < 0) continue;
+      const int dst = move_dst[w0 + q * movers];
+      reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + dst) * D)[lane] = kr[q];
+      reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + dst) * D)[lane] = vr[q];
+      if (lane == 0) {
+        P.bank_score[gi * BANK + dst] = P.pend_score[gi * PEND + src[q]];
+        P.bank_pos[gi * BANK + dst] = P.pend_pos[gi * PEND + src[q]];
+      }
+    }
+  }
+}
+
+// Metadata of a block's run of sequences, read in one parallel load so that
+// the (many) sequences with nothing to commit cost no serial global-memory
+// latency.  Threads tid < nb fill slot tid.
+__device__ __forceinline__ void load_run(const CommitParams& P, int b0, int nb, int* blk_seq,
+                                         int* blk_c, int* blk_p) {
+  const int tid = threadIdx.x;
+  if (tid < nb) {
+    const int seq = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b0 + tid];
+    blk_seq[tid] = seq;
+    blk_c[tid] = 0;
+    blk_p[tid] = 0;
+    if (seq >= 0 && seq < P.s_max) {
+      blk_c[tid] = P.meta[seq * 4 + 2];
+      blk_p[tid] = P.meta[seq * 4 + 1] + P.p_add;
+    }
+  }
+}
+
+// The checks every form of the commit makes for sequence slot bi: returns true
+// when (seq, c, p) is a merge to run.
+__device__ __forceinline__ bool merge_due(const CommitParams& P, int seq, int c, int p) {
+  const int tid = threadIdx.x;
+  if (seq < 0 || seq >= P.s_max) {
+    if (tid == 0 && blockIdx.y == 0) set_dev_error(P.err, ER_EINVAL);
+    return false;
+  }
+  if (P.only_if_full && p != PEND) return false;
+  if (c < 0 || c > BANK || p < 0 || p > PEND) {
+    if (tid == 0) set_dev_error(P.err, ER_ECAPACITY);
+    return false;
+  }
+  return true;
+}
+
 __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
   __shared__ uint64_t skey[NSORT];
   __shared__ uint16_t ssrc[NSORT];
@@ -247,60 +378,25 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
   // and move list, and moves its share of the winners (rank r takes winners
   // r*8+warp, r*8+warp + 8*ranks, ...)
   const int rank = (int)cluster_ctarank(), nranks = (int)cluster_nctarank();
-  // each cluster owns a run of `per_block` listed sequences; their metadata is read
-  // in one parallel load, so the (many) sequences with nothing to commit cost
-  // no serial global-memory latency
+  // each cluster owns a run of `per_block` listed sequences
   const int b0 = (blockIdx.x / nranks) * P.per_block;
   const int nb = min(P.per_block, P.n - b0);
-  if (tid < nb) {
-    const int seq = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b0 + tid];
-    blk_seq[tid] = seq;
-    if (seq >= 0 && seq < P.s_max) {
-      blk_c[tid] = P.meta[seq * 4 + 2];
-      blk_p[tid] = P.meta[seq * 4 + 1] + P.p_add;
-    }
-  }
+  load_run(P, b0, nb, blk_seq, blk_c, blk_p);
   __syncthreads();
   for (int bi = 0; bi < nb; ++bi) {
     const int b = b0 + bi;
     const int seq = blk_seq[bi];
-    if (seq < 0 || seq >= P.s_max) {
-      if (tid == 0 && blockIdx.y == 0) set_dev_error(P.err, ER_EINVAL);
-      continue;
-    }
     const int c = blk_c[bi];
     const int p = blk_p[bi];
-    if (P.only_if_full && p != PEND) continue;
-    if (c < 0 || c > BANK || p < 0 || p > PEND) {
-      if (tid == 0) set_dev_error(P.err, ER_ECAPACITY);
-      continue;
-    }
+    if (!merge_due(P, seq, c, p)) continue;
     const size_t gi = grp(seq, l, g, P.L);
 
     const int K = min(BANK, c + p);
     for (int i = tid; i < BANK + PEND; i += CT) flag[i] = 0;
+    __syncthreads();  // flags cleared before they are set
     if (P.kept == nullptr) {
       // only the kept set is needed: radix-select the K-th largest key
-      uint64_t key5[5];  // records tid + 256*q (bank 0..1023, then pending)
-#pragma unroll
-      for (int q = 0; q < 5; ++q) {
-        const int i = tid + CT * q;
-        uint64_t kv = 0;
-        if (i < BANK) {
-          if (i < c) kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
-        } else if (i - BANK < p) {
-          kv = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
-        }
-        key5[q] = kv;
-      }
-      uint64_t prefix = 0;
-      int shift = 64;
-      if (c + p > BANK) radix_select(key5, K, hist, warp_sums, sel, &prefix, &shift);
-      __syncthreads();  // flags cleared before they are set
-#pragma unroll
-      for (int q = 0; q < 5; ++q)
-        if (key5[q] != 0 && (shift >= 64 || (key5[q] >> shift) >= (prefix >> shift)))
-          flag[tid + CT * q] = 1;
+      select_kept(P, gi, c, p, K, flag, hist, warp_sums, sel);
     } else {
       // the ranked list is wanted: full bitonic sort, elements 8*tid .. 8*tid+7
       uint64_t key[EPT];
@@ -316,7 +412,6 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
         src[e] = (uint32_t)i;
       }
       sort2048(key, src, skey, ssrc);
-      __syncthreads();  // flags cleared before they are set
       // rank r = 8*tid + e
 #pragma unroll
       for (int e = 0; e < EPT; ++e)
@@ -331,66 +426,86 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
       }
     }
     __syncthreads();
-
-    // evicted bank slots, ascending (4 slots per thread)
-    int ev[4], nev = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int slot = tid * 4 + q;
-      ev[q] = (slot < c && !flag[slot]) ? 1 : 0;
-      nev += ev[q];
-    }
-    int total_evict = 0;
-    int er = block_scan_excl(nev, warp_sums, &total_evict);
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (ev[q]) evict_list[er++] = (int16_t)(tid * 4 + q);
-    // pending winners, ascending pending index (one per thread)
-    int total_win = 0;
-    const int wn = (tid < p && flag[BANK + tid]) ? 1 : 0;
-    const int w_rank = block_scan_excl(wn, warp_sums, &total_win);
-    __syncthreads();
-    if (wn) {
-      const int dst =
-          w_rank < total_evict ? (int)evict_list[w_rank] : c + (w_rank - total_evict);
-      move_src[w_rank] = (int16_t)tid;
-      move_dst[w_rank] = (int16_t)dst;
-    }
-    __syncthreads();
-
+    const int total_win = plan_moves(c, p, flag, evict_list, move_src, move_dst, warp_sums);
     // no CTA of the cluster writes the bank before every CTA has read this merge's keys
     cluster_sync_all();
-    // move rows: one warp per winner, 16 bytes per lane per row; MV winners per warp
-    // in flight (every load issued before the first store)
-    constexpr int MV = 4;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int movers = CW * nranks;
-    for (int w0 = rank * CW + warp; w0 < total_win; w0 += MV * movers) {
-      uint4 kr[MV], vr[MV];
-      int src[MV];
-#pragma unroll
-      for (int q = 0; q < MV; ++q) {
-        const int w = w0 + q * movers;
-        src[q] = w < total_win ? (int)move_src[w] : -1;
-        kr[q] = vr[q] = make_uint4(0, 0, 0, 0);
-        if (src[q] >= 0) {
-          kr[q] = reinterpret_cast<const uint4*>(P.pend_k + (gi * PEND + src[q]) * D)[lane];
-          vr[q] = reinterpret_cast<const uint4*>(P.pend_v + (gi * PEND + src[q]) * D)[lane];
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < MV; ++q) {
-        if (src[q] < 0) continue;
-        const int dst = move_dst[w0 + q * movers];
-        reinterpret_cast<uint4*>(P.bank_k + (gi * BANK + dst) * D)[lane] = kr[q];
-        reinterpret_cast<uint4*>(P.bank_v + (gi * BANK + dst) * D)[lane] = vr[q];
-        if (lane == 0) {
-          P.bank_score[gi * BANK + dst] = P.pend_score[gi * PEND + src[q]];
-          P.bank_pos[gi * BANK + dst] = P.pend_pos[gi * PEND + src[q]];
-        }
-      }
-    }
+    move_winners(P, gi, total_win, move_src, move_dst, rank * CW + (tid >> 5), CW * nranks);
     __syncthreads();  // shared arrays are reused by the next sequence
+  }
+}
+
+// The layer calls' commit in two launches: k_commit_plan (steps 1-3, the move
+// lists into `plan`) runs beside the read, which leaves the keys and the bank
+// alone; k_commit_move (step 4) runs after the read, beside o_proj.  One block
+// per (run of SPB sequences, layer, group) plans; MOVE_CTAS blocks per run
+// share the moves.
+constexpr int MOVE_CTAS = 8;
+
+__global__ void __launch_bounds__(CT, 4) k_commit_plan(CommitParams P, MovePlan* plan) {
+  __shared__ uint8_t flag[BANK + PEND];
+  __shared__ int16_t evict_list[BANK];
+  __shared__ int16_t move_src[PEND], move_dst[PEND];
+  __shared__ int warp_sums[CW];
+  __shared__ int blk_seq[SPB], blk_c[SPB], blk_p[SPB];
+  __shared__ int hist[256];
+  __shared__ int sel[4];
+  const int lg = blockIdx.y, l = P.layer0 + lg / NG, g = lg % NG;
+  const int nlg = P.nlayers * NG;
+  const int tid = threadIdx.x;
+  const int b0 = blockIdx.x * SPB;
+  const int nb = min(SPB, P.n - b0);
+  load_run(P, b0, nb, blk_seq, blk_c, blk_p);
+  __syncthreads();
+  for (int bi = 0; bi < nb; ++bi) {
+    MovePlan& mp = plan[(size_t)(b0 + bi) * nlg + lg];
+    const int seq = blk_seq[bi];
+    const int c = blk_c[bi];
+    const int p = blk_p[bi];
+    if (!merge_due(P, seq, c, p)) {
+      if (tid == 0) mp.n = 0;
+      continue;
+    }
+    const size_t gi = grp(seq, l, g, P.L);
+    for (int i = tid; i < BANK + PEND; i += CT) flag[i] = 0;
+    __syncthreads();
+    select_kept(P, gi, c, p, min(BANK, c + p), flag, hist, warp_sums, sel);
+    __syncthreads();
+    const int total_win = plan_moves(c, p, flag, evict_list, move_src, move_dst, warp_sums);
+    for (int w = tid; w < total_win; w += CT) {
+      mp.src[w] = move_src[w];
+      mp.dst[w] = move_dst[w];
+    }
+    if (tid == 0) mp.n = total_win;
+    __syncthreads();  // shared arrays are reused by the next sequence
+  }
+}
+
+__global__ void __launch_bounds__(CT, 4) k_commit_move(CommitParams P, const MovePlan* plan) {
+  __shared__ int16_t move_src[PEND], move_dst[PEND];
+  __shared__ int blk_seq[SPB], blk_n[SPB];
+  const int lg = blockIdx.y, l = P.layer0 + lg / NG, g = lg % NG;
+  const int nlg = P.nlayers * NG;
+  const int tid = threadIdx.x;
+  const int run = blockIdx.x / MOVE_CTAS, r = blockIdx.x % MOVE_CTAS;
+  const int b0 = run * SPB;
+  const int nb = min(SPB, P.n - b0);
+  if (tid < nb) {
+    blk_seq[tid] = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b0 + tid];
+    blk_n[tid] = plan[(size_t)(b0 + tid) * nlg + lg].n;
+  }
+  __syncthreads();
+  for (int bi = 0; bi < nb; ++bi) {
+    const int n = blk_n[bi];
+    if (n <= 0) continue;  // planned as a merge only for a valid, full sequence
+    const MovePlan& mp = plan[(size_t)(b0 + bi) * nlg + lg];
+    for (int w = tid; w < n; w += CT) {
+      move_src[w] = mp.src[w];
+      move_dst[w] = mp.dst[w];
+    }
+    __syncthreads();
+    move_winners(P, grp(blk_seq[bi], l, g, P.L), n, move_src, move_dst,
+                 r * CW + (tid >> 5), CW * MOVE_CTAS);
+    __syncthreads();  // the lists are reused by the next sequence
   }
 }
 
@@ -426,6 +541,34 @@ int launch_commit(const CommitParams& P, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, k_commit, Q) != cudaSuccess) return ER_ECUDA;
+  count_launches(1);
+  return launch_status();
+}
+
+// The layer calls' commit (only_if_full, no ranked list): plan beside the read,
+// move after it.  plan: [n][nlayers * 4] MovePlan, caller scratch.
+size_t commit_plan_bytes(int n, int nlayers) {
+  return (size_t)n * nlayers * NG * sizeof(MovePlan);
+}
+
+int launch_commit_plan(const CommitParams& P, MovePlan* plan, cudaStream_t st) {
+  if (P.n <= 0) return ER_OK;
+  if (!P.only_if_full || P.kept || !plan) return ER_EINVAL;
+  CommitParams Q = P;
+  Q.per_block = SPB;
+  const int runs = (P.n + SPB - 1) / SPB;
+  k_commit_plan<<<dim3(runs, P.nlayers * NG), CT, 0, st>>>(Q, plan);
+  count_launches(1);
+  return launch_status();
+}
+
+int launch_commit_move(const CommitParams& P, const MovePlan* plan, cudaStream_t st) {
+  if (P.n <= 0) return ER_OK;
+  if (!plan) return ER_EINVAL;
+  CommitParams Q = P;
+  Q.per_block = SPB;
+  const int runs = (P.n + SPB - 1) / SPB;
+  k_commit_move<<<dim3(runs * MOVE_CTAS, P.nlayers * NG), CT, 0, st>>>(Q, plan);
   count_launches(1);
   return launch_status();
 }

@@ -25,7 +25,9 @@ const float* score_partials(const void* scratch, int n);
 int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st);
 int launch_attend(const AttendParams& P, float* o_swa, float* o_rma, uint16_t* o_sum,
                   bool zero_sched, cudaStream_t st);
-int launch_commit(const CommitParams& P, cudaStream_t st);
+size_t commit_plan_bytes(int n, int nlayers);
+int launch_commit_plan(const CommitParams& P, MovePlan* plan, cudaStream_t st);
+int launch_commit_move(const CommitParams& P, const MovePlan* plan, cudaStream_t st);
 size_t attend_part_floats(int nq);
 size_t attend_ml_floats(int nq);
 size_t prefill_out_floats(int T);
@@ -48,6 +50,7 @@ struct LayerWs {
   int* sched;                // decode: the read's work counter
   float* pf_out;             // prefill: FP32 branch outputs [2][T][4096]
   uint16_t* o_sum;
+  MovePlan* plan;            // the commit's move lists, one per (sequence, group)
   size_t bytes;
 };
 
@@ -65,19 +68,23 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   w.sched = prefill ? nullptr : c.take<int>(1);
   w.pf_out = prefill ? c.take<float>(prefill_out_floats(nq)) : nullptr;
   w.o_sum = c.take<uint16_t>((size_t)nq * OIN);
+  w.plan = reinterpret_cast<MovePlan*>(
+      c.take<unsigned char>(commit_plan_bytes(prefill ? 1 : nq, 1)));
   w.bytes = c.used();
   return w;
 }
 
-// Steps of a layer call that run beside library GEMMs on a side stream: the
-// commit beside o_proj (anchor rows vs the read output) and, in a prefill
-// chunk, the scorer beside the q/k/v projection (both only read x).  A side stream per device takes them
-// between a fork and a join on the caller's stream, so the call's work still
-// completes in the caller's stream order (and stays capturable).
+// Steps of a layer call that run beside other work on a side stream: the
+// commit's planning beside the read (it reads only scores and positions, which
+// the read leaves alone) and its row moves beside o_proj (anchor rows vs the
+// read output), and, in a prefill chunk with unprepared weights, the scorer
+// beside the q/k/v projection (both only read x).  A side stream per device
+// takes them between forks and a join on the caller's stream, so the call's
+// work still completes in the caller's stream order (and stays capturable).
 struct Side {
   std::mutex mu;
   cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, fork2 = nullptr, join = nullptr;
 };
 Side g_side[64];
 
@@ -89,6 +96,7 @@ Side* side_for_current_device() {
   if (!sd.stream) {
     if (cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking) != cudaSuccess ||
         cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sd.fork2, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) != cudaSuccess)
       return nullptr;
   }
@@ -164,11 +172,33 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   pp.chunk_k = W.chunk_k; pp.chunk_v = W.chunk_v; pp.err = st->dev_error;
   pp.sched_reset = W.sched;
   if ((rc = launch_post_proj(pp, rma_off, s)) != ER_OK) return rc;
+  // a7, planned: the layer's commit where the block is now full (decided on the
+  // device) works out its kept set and move lists on the side stream while the
+  // reads run; the rows move after them, beside a6 (the shared o_proj)
+  CommitParams cp{};
+  cp.bank_k = st->bank_k; cp.bank_v = st->bank_v; cp.pend_k = st->pend_k; cp.pend_v = st->pend_v;
+  cp.bank_score = st->bank_score; cp.pend_score = st->pend_score;
+  cp.bank_pos = st->bank_pos; cp.pend_pos = st->pend_pos;
+  cp.meta = st->meta; cp.seq_ids = seq_ids; cp.seq_fixed = seq_fixed;
+  cp.n = prefill ? 1 : nq; cp.s_max = st->s_max; cp.L = st->n_layers;
+  cp.layer0 = layer; cp.nlayers = 1; cp.p_add = prefill ? nq : 1; cp.only_if_full = 1;
+  cp.kept = nullptr; cp.err = st->dev_error;
+  // the events are re-recorded by every call: hold the side stream from the
+  // first fork to the join
+  std::unique_lock<std::mutex> lock(sd->mu, std::defer_lock);
+  int rc_plan = ER_OK;
+  if (!rma_off) {
+    lock.lock();
+    if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
+        cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
+      return ER_ECUDA;
+    rc_plan = launch_commit_plan(cp, W.plan, sd->stream);
+  }
   // a5 / a8: both reads, merged into bf16(o_swa + o_rma)
+  int rc_read;
   if (prefill) {
-    if ((rc = launch_prefill_attend(st, layer, seq_fixed, nq, W.q_swa, W.q_rma, W.chunk_k,
-                                    W.chunk_v, W.pf_out, W.o_sum, rma_off, s)) != ER_OK)
-      return rc;
+    rc_read = launch_prefill_attend(st, layer, seq_fixed, nq, W.q_swa, W.q_rma, W.chunk_k,
+                                    W.chunk_v, W.pf_out, W.o_sum, rma_off, s);
   } else {
     AttendParams ap{};
     ap.win_k = st->win_k; ap.win_v = st->win_v; ap.bank_k = st->bank_k; ap.bank_v = st->bank_v;
@@ -178,30 +208,25 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     ap.rma_off = rma_off ? 1 : 0;
     ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.sched = W.sched; ap.err = st->dev_error;
     // k_post_proj above zeroed the work counter
-    if ((rc = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s)) != ER_OK) return rc;
+    rc_read = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s);
   }
-  // a7: commit this layer where the block is now full (decided on the device),
-  // beside a6, the shared o_proj (disjoint data)
-  if (rma_off) return gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
-  CommitParams cp{};
-  cp.bank_k = st->bank_k; cp.bank_v = st->bank_v; cp.pend_k = st->pend_k; cp.pend_v = st->pend_v;
-  cp.bank_score = st->bank_score; cp.pend_score = st->pend_score;
-  cp.bank_pos = st->bank_pos; cp.pend_pos = st->pend_pos;
-  cp.meta = st->meta; cp.seq_ids = seq_ids; cp.seq_fixed = seq_fixed;
-  cp.n = prefill ? 1 : nq; cp.s_max = st->s_max; cp.L = st->n_layers;
-  cp.layer0 = layer; cp.nlayers = 1; cp.p_add = prefill ? nq : 1; cp.only_if_full = 1;
-  cp.kept = nullptr; cp.err = st->dev_error;
-  std::lock_guard<std::mutex> lock(sd->mu);  // the events are re-recorded by every call
-  if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
-      cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
-    return ER_ECUDA;
-  const int rc_commit = launch_commit(cp, sd->stream);
-  const int rc_proj = gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
-  // join: the caller's stream waits for the commit whatever happened above
-  if (cudaEventRecord(sd->join, sd->stream) != cudaSuccess ||
-      cudaStreamWaitEvent(s, sd->join, 0) != cudaSuccess)
-    return ER_ECUDA;
-  return rc_commit != ER_OK ? rc_commit : rc_proj;
+  if (rma_off) return rc_read != ER_OK ? rc_read : gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
+  // the moves wait for the reads (they overwrite evicted anchor rows); after a
+  // failed launch nothing moves, but the side stream still joins
+  int rc_move = ER_OK;
+  bool joined_ok = cudaEventRecord(sd->fork2, s) == cudaSuccess &&
+                   cudaStreamWaitEvent(sd->stream, sd->fork2, 0) == cudaSuccess;
+  if (joined_ok && rc_plan == ER_OK && rc_read == ER_OK)
+    rc_move = launch_commit_move(cp, W.plan, sd->stream);
+  const int rc_proj =
+      rc_read == ER_OK ? gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s) : ER_OK;
+  // join: the caller's stream waits for the side stream whatever happened above
+  joined_ok = cudaEventRecord(sd->join, sd->stream) == cudaSuccess &&
+              cudaStreamWaitEvent(s, sd->join, 0) == cudaSuccess && joined_ok;
+  if (!joined_ok) return ER_ECUDA;
+  for (int r : {rc_plan, rc_read, rc_move, rc_proj})
+    if (r != ER_OK) return r;
+  return ER_OK;
 }
 
 }  // namespace

@@ -56,6 +56,14 @@ struct AttendParams {
   int32_t* err;
 };
 
+// One merge's move list (the layer calls' two-launch commit): winner w moves
+// from pending slot src[w] to bank slot dst[w]; n = 0 when nothing commits.
+struct MovePlan {
+  int32_t n;
+  int16_t src[256];
+  int16_t dst[256];
+};
+
 struct CommitParams {
   uint16_t *bank_k, *bank_v;
   const uint16_t *pend_k, *pend_v;
