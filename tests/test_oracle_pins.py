@@ -354,6 +354,49 @@ def test_commit_keeps_anchor_contents_when_pending_loses():
         assert torch.equal(getattr(st, n), getattr(before, n))
 
 
+def test_commits_compose_to_one_top_k_over_the_stream():
+    """Commits after every block of 256 keep, in the end, exactly the top 1024 of
+    all records ever appended (for a total order, top-k(top-k(A) | B) =
+    top-k(A | B)), and every kept slot still holds its own record's rows."""
+    gen = np.random.default_rng(3)
+    st = oracle.OracleState(1, 1)
+    st.meta[0] = torch.tensor([0, 0, 0, 0])
+    allrec = [[] for _ in range(4)]
+    pos0 = 5000
+    for blk in range(12):
+        for g in range(4):
+            sc = gen.standard_normal(256).astype(np.float32)
+            if blk > 0:  # exact ties with earlier records and inside the block
+                prev = np.array([r[0] for r in allrec[g]], dtype=np.float32)
+                idx = gen.integers(0, 256, 13)
+                sc[idx] = prev[gen.integers(0, len(prev), 13)]
+            sc[gen.integers(0, 256, 3)] = sc[0]
+            sc[7] = -0.0 if blk % 2 else 0.0
+            sc[11] = np.float32("nan") if blk % 3 == 0 else np.float32("-inf")
+            pos = pos0 + blk * 256 + np.arange(256, dtype=np.int32)
+            st.pend_score[0, 0, g] = torch.from_numpy(sc)
+            st.pend_pos[0, 0, g] = torch.from_numpy(pos)
+            # each record's K and V rows carry its position (exact in BF16 below 256)
+            tag = torch.from_numpy(((pos % 199) + g).astype(np.float32)).to(torch.bfloat16)
+            st.pend_k[0, 0, g] = tag[:, None].expand(256, 256)
+            st.pend_v[0, 0, g] = -tag[:, None].expand(256, 256)
+            allrec[g] += list(zip(sc.tolist(), pos.tolist()))
+        st.meta[0, 1] = 256
+        st.commit(-1, 0)
+        assert int(st.meta[0, 1]) == 0 and int(st.meta[0, 2]) == min(1024, 256 * (blk + 1))
+    for g in range(4):
+        want = sorted(allrec[g], key=lambda r: _order_key(r[0], r[1]))[:1024]
+        got = st.bank_pos[0, 0, g].tolist()
+        assert sorted(got) == sorted(q for _, q in want), g
+        tags = st.bank_k[0, 0, g, :, 0].float()
+        assert torch.equal(tags, torch.tensor([(q % 199) + g for q in got], dtype=torch.float32))
+        assert torch.equal(st.bank_v[0, 0, g, :, 5].float(), -tags)
+        by_pos = {q: sc for sc, q in allrec[g]}
+        for i, q in enumerate(got):
+            a, b = float(st.bank_score[0, 0, g, i]), by_pos[q]
+            assert a == b or (math.isnan(a) and math.isnan(b))
+
+
 # -------------------------------------------------------------- decode path
 
 def _weights(seed, layer=0):
