@@ -15,7 +15,7 @@
 //   warp 4 (producer): lane 0 takes the CTA's items from a work counter; for
 //     each tile it arms the
 //     stage's mbarrier with the transaction bytes and issues TMA tensor copies
-//     (cp.async.bulk.tensor.2d, no multicast) of four 64x64 boxes of K rows and
+//     (cp.async.bulk.tensor.2d, into this CTA only) of four 64x64 boxes of K rows and
 //     four of V rows, 128-byte swizzled, plus the item's 4 query heads (one
 //     plain bulk copy) with its first tile; 3-stage ring.
 //   warps 0..3 (consumers): each takes 16 rows (keys) of every tile.  The

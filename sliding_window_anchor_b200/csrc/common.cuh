@@ -126,8 +126,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
   return true;
 }
 
-// Contiguous global -> shared bulk copy (TMA engine, no tensor map, no
-// multicast), completion signalled on `bar` as transaction bytes.
+// Contiguous global -> shared bulk copy (TMA engine, no tensor map, into this
+// CTA only), completion signalled on `bar` as transaction bytes.
 // dst/src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
                                          uint64_t* bar) {

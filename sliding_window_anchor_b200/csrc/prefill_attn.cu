@@ -38,8 +38,8 @@
 //               rescaled in TMEM (after the previous PV has completed).  At the
 //               end O / l and (m, l) go out in FP32 through a staging tile.
 // Both CTAs' loads count on the even CTA's barriers; each softmax warp of
-// both CTAs arrives (once per tile) on the even CTA's P-ready barrier.  No copy is
-// multicast.  An item's key tiles are split over NSPLIT pairs; a second
+// both CTAs arrives (once per tile) on the even CTA's P-ready barrier.  Every copy
+// lands in one CTA only.  An item's key tiles are split over NSPLIT pairs; a second
 // kernel merges the splits of each branch by their (m, l), adds the two
 // branches and rounds to BF16 for o_proj, and moves the chunk's window rows
 // into the ring (after every read of the chunk).

@@ -1,8 +1,8 @@
 // tc.cuh — 5th-generation tensor-core (tcgen05) building blocks for sm_100a:
 // TMEM allocation, UMMA shared-memory and instruction descriptors, the
 // single-thread MMA issue, its completion commit onto an mbarrier, TMEM loads,
-// and TMA tensor-map helpers.  Hand-written PTX; one CTA, no clusters, no
-// multicast.
+// and TMA tensor-map helpers.  Hand-written PTX; every copy lands in one
+// CTA.
 #pragma once
 
 #include <cuda.h>
@@ -232,7 +232,8 @@ __device__ __forceinline__ void commit_pair(uint32_t bar) {
 }
 
 // A TMA box into this CTA's shared memory whose transaction bytes count on the
-// mbarrier at shared::cluster address `bar` (the even CTA's), no multicast.
+// mbarrier at shared::cluster address `bar` (the even CTA's); the data lands
+// in this CTA only.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y,
                                                  uint32_t bar) {
   asm volatile(
