@@ -494,13 +494,23 @@ __global__ void k_prefill_combine(const float* __restrict__ out, const float2* _
   const int d0 = (idx % (D / 8)) * 8;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   for (int br = 0; br < nbr; ++br) {
+    // every split's (m, l) and partial row are loaded up front (all in bounds),
+    // so the loads overlap; a split without keys (l = 0) is skipped, never
+    // multiplied, whatever its row holds
     float2 v[NSPLIT];
-    float M = -INFINITY;
+    float4 x0[NSPLIT], x1[NSPLIT];
 #pragma unroll
     for (int sp = 0; sp < NSPLIT; ++sp) {
       v[sp] = ml[(size_t)(br * NSPLIT + sp) * T * NH + row];
-      if (v[sp].y > 0.f) M = fmaxf(M, v[sp].x);
+      const float4* src = reinterpret_cast<const float4*>(
+          out + ((size_t)(br * NSPLIT + sp) * T * NH + row) * D + d0);
+      x0[sp] = src[0];
+      x1[sp] = src[1];
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int sp = 0; sp < NSPLIT; ++sp)
+      if (v[sp].y > 0.f) M = fmaxf(M, v[sp].x);
     float w[NSPLIT], wsum = 0.f;
 #pragma unroll
     for (int sp = 0; sp < NSPLIT; ++sp) {
@@ -512,11 +522,10 @@ __global__ void k_prefill_combine(const float* __restrict__ out, const float2* _
     for (int sp = 0; sp < NSPLIT; ++sp) {
       if (w[sp] == 0.f) continue;
       const float ws = w[sp] * inv;
-      const float4* src = reinterpret_cast<const float4*>(
-          out + ((size_t)(br * NSPLIT + sp) * T * NH + row) * D + d0);
-      const float4 x0 = src[0], x1 = src[1];
-      acc[0] += ws * x0.x; acc[1] += ws * x0.y; acc[2] += ws * x0.z; acc[3] += ws * x0.w;
-      acc[4] += ws * x1.x; acc[5] += ws * x1.y; acc[6] += ws * x1.z; acc[7] += ws * x1.w;
+      acc[0] += ws * x0[sp].x; acc[1] += ws * x0[sp].y;
+      acc[2] += ws * x0[sp].z; acc[3] += ws * x0[sp].w;
+      acc[4] += ws * x1[sp].x; acc[5] += ws * x1[sp].y;
+      acc[6] += ws * x1[sp].z; acc[7] += ws * x1[sp].w;
     }
   }
   uint4 pk;
