@@ -211,7 +211,7 @@ __device__ __forceinline__ int row_col(int hs) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(256) k_post_proj(PostParams P) {
+__global__ void __launch_bounds__(256, 8) k_post_proj(PostParams P) {
   __shared__ float2 s_cs[32];  // the rotation of this token's position
   __shared__ int s_tok[4];     // seq, t, p_idx, valid
   grid_dep_trigger();  // a prefill read may set itself up meanwhile (it waits for us)
