@@ -173,8 +173,11 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   pp.sched_reset = W.sched;
   if ((rc = launch_post_proj(pp, rma_off, s)) != ER_OK) return rc;
   // a7, planned: the layer's commit where the block is now full (decided on the
-  // device) works out its kept set and move lists on the side stream while the
-  // reads run; the rows move after them, beside a6 (the shared o_proj)
+  // device) works out its kept set and move lists on the side stream -- in a
+  // decode batch while the reads run (a long, dynamically scheduled kernel that
+  // absorbs the shared SMs), in a prefill chunk after its reads (short, with a
+  // fixed CTA per tile: sharing SMs lengthened it) beside the combine and
+  // o_proj -- and the rows move after the reads, beside a6 (the shared o_proj)
   CommitParams cp{};
   cp.bank_k = st->bank_k; cp.bank_v = st->bank_v; cp.pend_k = st->pend_k; cp.pend_v = st->pend_v;
   cp.bank_score = st->bank_score; cp.pend_score = st->pend_score;
@@ -189,10 +192,12 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   int rc_plan = ER_OK;
   if (!rma_off) {
     lock.lock();
-    if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
-        cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
-      return ER_ECUDA;
-    rc_plan = launch_commit_plan(cp, W.plan, sd->stream);
+    if (!prefill) {
+      if (cudaEventRecord(sd->fork, s) != cudaSuccess ||
+          cudaStreamWaitEvent(sd->stream, sd->fork, 0) != cudaSuccess)
+        return ER_ECUDA;
+      rc_plan = launch_commit_plan(cp, W.plan, sd->stream);
+    }
   }
   // a5 / a8: both reads, merged into bf16(o_swa + o_rma)
   int rc_read;
@@ -216,6 +221,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   int rc_move = ER_OK;
   bool joined_ok = cudaEventRecord(sd->fork2, s) == cudaSuccess &&
                    cudaStreamWaitEvent(sd->stream, sd->fork2, 0) == cudaSuccess;
+  if (prefill && joined_ok && rc_read == ER_OK)
+    rc_plan = launch_commit_plan(cp, W.plan, sd->stream);
   if (joined_ok && rc_plan == ER_OK && rc_read == ER_OK)
     rc_move = launch_commit_move(cp, W.plan, sd->stream);
   const int rc_proj =
