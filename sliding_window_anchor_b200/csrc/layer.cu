@@ -215,7 +215,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     // k_post_proj above zeroed the work counter
     rc_read = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s);
   }
-  if (rma_off) return rc_read != ER_OK ? rc_read : gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
+  if (rma_off)
+    return rc_read != ER_OK ? rc_read : gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
   // the moves wait for the reads (they overwrite evicted anchor rows); after a
   // failed launch nothing moves, but the side stream still joins
   int rc_move = ER_OK;
