@@ -339,8 +339,9 @@ const char* er_error_string(int code);
 uint64_t er_launch_count(void);
 
 /* When enabled, launches of the read kernels (the a5 decode read and the a8
- * prefill read) are bracketed by CUDA events on their own stream; er_profile_read returns the summed milliseconds and the
- * number of timed launches since the last reset (it synchronises the events).
+ * prefill read) are bracketed by CUDA events on their own stream;
+ * er_profile_read returns the summed milliseconds and the number of timed
+ * launches since the last reset (it synchronises the events).
  * Host-side bookkeeping only; not thread-safe. */
 int er_profile_enable(int enable);
 int er_profile_read(double* ms_total, int64_t* launches, int reset);

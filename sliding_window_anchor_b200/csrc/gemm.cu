@@ -1,6 +1,7 @@
 // gemm.cu — the plain BF16 projections (a1: x·W_qkvᵀ, a6: o·W_oᵀ), FP32
-// accumulation, BF16 output (or FP32 for a1 fused with the scorer's W1·x).  These are library GEMMs (cuBLAS) with no fused
-// epilogue; the norm/RoPE and state writes that follow run in k_post_proj.
+// accumulation, BF16 output (or FP32 for a1 fused with the scorer's W1·x).
+// These are library GEMMs (cuBLAS) with no fused epilogue; the norm/RoPE and
+// state writes that follow run in k_post_proj.
 #include <cublas_v2.h>
 
 #include <mutex>

@@ -485,7 +485,8 @@ __global__ void k_prefill_combine(const float* __restrict__ out, const float2* _
       if (t >= 0) {
         const size_t row = grp(rw.seq, rw.layer, g, rw.L) * WIN + (size_t)(t % WIN);
         const uint4* src =
-            reinterpret_cast<const uint4*>((is_v ? rw.chunk_v : rw.chunk_k) + ((size_t)g * T + tok) * D);
+            reinterpret_cast<const uint4*>((is_v ? rw.chunk_v : rw.chunk_k) +
+                                           ((size_t)g * T + tok) * D);
         reinterpret_cast<uint4*>((is_v ? rw.win_v : rw.win_k) + row * D)[lane] = src[lane];
       }
     }
