@@ -25,7 +25,8 @@ __all__ = ["State", "LayerWeights", "qk_norm_rope", "rma_score", "rma_append_pen
            "rma_commit", "swa_rma_attend", "swa_rma_decode", "swa_rma_prefill_chunk",
            "advance", "state_init", "last_device_error", "launch_count", "profile_enable",
            "profile_read", "decode_workspace_bytes", "prefill_workspace_bytes",
-           "attend_workspace_bytes", "score_workspace_bytes", "rma_score_noalloc", "ERError"]
+           "attend_workspace_bytes", "score_workspace_bytes", "rma_score_noalloc",
+           "wait_selftest", "ERError"]
 
 
 class State:
