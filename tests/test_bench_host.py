@@ -58,3 +58,42 @@ def test_algorithmic_bytes_follow_the_pending_fill():
     per_group_fixed = 2 * 4 * 512 + 2 * 4 * 1024
     assert b0 == 4 * ((2048 + 256) * 1024 + per_group_fixed)
     assert b1 == 4 * ((2048 + 1) * 1024 + per_group_fixed)
+
+
+def _run_reference(env_extra=None):
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, **(env_extra or {}))
+    return subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1",
+                           "--warmup", "0"], cwd=root, env=env, capture_output=True, text=True,
+                          timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    """The reference arm is the oracle on the host cores: one JSON line with the
+    base contract's keys, the impl tag, a cpu_baseline describing the run and an
+    e2e block that moves no bytes."""
+    r = _run_reference()
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "tok/s"
+    assert d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == bench.WORKLOAD
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tok/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    """Under torchrun only rank 0 runs and prints the reference line."""
+    r = _run_reference({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert not any(l.startswith("{") for l in r.stdout.splitlines())
