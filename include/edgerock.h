@@ -39,6 +39,11 @@
  *    call (and the first read or scorer call) on a device creates that
  *    device's library resources (cuBLAS handle, side stream, events, kernel
  *    attributes): make one such call before capturing on the device.
+ *  - A workspace (`ws`) is a call's scratch; in the layer calls it also holds
+ *    the read's work counter and the commit's move lists, which live from the
+ *    call's first kernel to its last.  Calls that may run at the same time
+ *    (other streams, other threads) need workspaces of their own; calls
+ *    ordered on one stream can share one.
  *  - Return value: ER_OK, or a negative ER_E* code.  Host-side argument checks
  *    happen before anything is enqueued; a failed check enqueues nothing.
  *    Conditions only the device can see (a sequence id out of range, a full
