@@ -590,3 +590,62 @@ def test_position_shift_invariance():
         _, o_swa, _ = st.decode_layer(ow, 0, 0, x, want_branches=True)
         outs.append(o_swa)
     assert (outs[0] - outs[1]).abs().max() < 2e-2
+
+
+# ---------------------------------------------------------- pending append
+
+def test_append_pending_writes_only_the_next_slot_of_each_group():
+    # neodrop.ai "内存还会跌吗？…" §三段记忆，只记值得记的: each token becomes one candidate
+    # record per KV group, appended behind the ones already pending; the counters are
+    # not touched by the append (the step's advance moves them)
+    g = torch.Generator().manual_seed(77)
+    st = oracle.OracleState(3, 2)
+    for n in oracle.OracleState.ARRAYS:
+        t = getattr(st, n)
+        if t.dtype == torch.bfloat16 or t.dtype == torch.float32:
+            t.copy_(torch.randn(t.shape, generator=g).to(t.dtype))
+        else:
+            t.copy_(torch.randint(-5, 10**6, t.shape, generator=g, dtype=torch.int32))
+    st.meta.copy_(torch.tensor([[9000, 5, 1024, 0], [100, 0, 0, 0], [40000, 255, 1024, 0]],
+                               dtype=torch.int32))
+    before = {n: getattr(st, n).clone() for n in oracle.OracleState.ARRAYS}
+    seqs = [2, 0]  # batch row b belongs to sequence seqs[b]; not in row order on purpose
+    k = torch.randn(2, 4, 256, generator=g).to(torch.bfloat16)
+    v = torch.randn(2, 4, 256, generator=g).to(torch.bfloat16)
+    s = torch.randn(2, 4, generator=g, dtype=torch.float32)
+    pos = torch.tensor([40000, 9000], dtype=torch.int32)
+    st.append_pending(1, seqs, k, v, s, pos)
+    expect = {n: t.clone() for n, t in before.items()}
+    for b, seq in enumerate(seqs):
+        p = int(before["meta"][seq, 1])
+        for grp in range(4):
+            expect["pend_k"][seq, 1, grp, p] = k[b, grp]
+            expect["pend_v"][seq, 1, grp, p] = v[b, grp]
+            expect["pend_score"][seq, 1, grp, p] = s[b, grp]
+            expect["pend_pos"][seq, 1, grp, p] = pos[b]
+    for n in oracle.OracleState.ARRAYS:
+        assert torch.equal(getattr(st, n), expect[n]), n
+    # slot 255 of sequence 2 really was written (the last slot of a block)
+    assert torch.equal(st.pend_k[2, 1, 3, 255], k[0, 3])
+
+
+def test_append_pending_equals_the_record_a_decode_step_appends():
+    # the record a decode step appends is the token's k_rma (normed, rotated at its
+    # position), v_rma, the group's FP32 score and the position: build it here from the
+    # pinned pieces and append it to a copy of the same state
+    ow, w, st = _seeded(55, 4096, "uniform")
+    p = int(st.meta[0, 1])
+    assert 0 < p < 255
+    t = int(st.meta[0, 0])
+    x = synth.normal((2560,), 55, synth.MISC, torch.bfloat16)
+    st_b = st.clone()
+    st.decode_layer(ow, 0, 0, x)
+    proj = oracle.linear_bf16(w["w_qkv"], x)
+    k = oracle.norm_rope(proj[10240:11264].view(4, 256), w["k_norm_rma"], t).view(1, 4, 256)
+    v = proj[11264:12288].view(1, 4, 256)
+    s = oracle.score(w["w1"], w["w2"], x)
+    st_b.append_pending(0, [0], k, v, s, torch.tensor([t], dtype=torch.int32))
+    for n in ("pend_k", "pend_v", "pend_score", "pend_pos", "bank_k", "bank_v", "bank_score",
+              "bank_pos", "meta"):
+        assert torch.equal(getattr(st, n), getattr(st_b, n)), n
+    assert int(st.pend_pos[0, 0, 2, p]) == t
