@@ -30,7 +30,8 @@
  *    outputs, workspace); the library never allocates or frees device memory
  *    itself (cuBLAS keeps its own handle memory; er_rma_score_noalloc's
  *    scratch is a static device array) and never synchronises the stream,
- *    except er_last_device_error, which reads one word back.
+ *    except er_last_device_error and er_last_call_error, which read one word
+ *    back.
  *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  A
  *    layer call may also run part of its work (the commit, beside o_proj) on
  *    a side stream the library keeps per device, forked from and joined back
@@ -39,6 +40,10 @@
  *    call (and the first read or scorer call) on a device creates that
  *    device's library resources (cuBLAS handle, side stream, events, kernel
  *    attributes): make one such call before capturing on the device.
+ *  - Those per-device resources, and the device addresses of the library's
+ *    fixed device arrays, are made once per device and process and are not
+ *    made again after cudaDeviceReset: do not call the library on a device
+ *    that was reset in the same process.
  *  - A workspace (`ws`) is a call's scratch; in the layer calls it also holds
  *    the read's work counter and the commit's move lists, which live from the
  *    call's first kernel to its last.  Calls that may run at the same time
@@ -47,9 +52,11 @@
  *  - Return value: ER_OK, or a negative ER_E* code.  Host-side argument checks
  *    happen before anything is enqueued; a failed check enqueues nothing.
  *    Conditions only the device can see (a sequence id out of range, a full
- *    pending block, a prefill chunk crossing the block boundary) skip the
- *    affected sequence and record the first such code in the state's device
- *    error word (read with er_last_device_error).  No kernel traps.
+ *    pending block, a prefill chunk crossing the block boundary, a bounded
+ *    wait that gave up) skip the affected work and record the first such
+ *    code in a device error word: the state's (read with
+ *    er_last_device_error), or, for the calls that take no state, the
+ *    library's own word (read with er_last_call_error).  No kernel traps.
  *  - BF16 values are raw bfloat16 bit patterns (er_bf16).
  */
 #ifndef EDGEROCK_H
@@ -162,13 +169,17 @@ size_t er_state_bytes(int32_t s_max, int32_t n_layers);
  * small, base is unaligned, or sizes are out of range. */
 int er_state_carve(void* base, size_t bytes, int32_t s_max, int32_t n_layers, er_state* out);
 
-/* Empties the listed sequences: meta := {0, 0, 0, 0}.  seq_ids: device
- * int32 [n].  Row contents are left as they are (unread until written). */
+/* Empties the listed sequences: meta := {0, 0, 0, 0}, i.e. the stream start
+ * of [F-mem]: a window, bank and pending block of fixed capacity, all empty.
+ * seq_ids: device int32 [n].  Row contents are left as they are (unread until
+ * written). */
 int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stream_t stream);
 
 /* End of one step of T tokens for the listed sequences, after every layer's
- * call: pos += T; pend_count += T, and a block that reached 256 (which every
- * layer has committed) empties: pend_count := 0, bank_count := min(1024,
+ * call [N-rma]: every token left one candidate per group in the pending
+ * block, and a block of 256 is merged into a bank of at most 1024.  So:
+ * pos += T; pend_count += T, and a block that reached 256 (which every layer
+ * has committed) empties: pend_count := 0, bank_count := min(1024,
  * bank_count + 256).  T in 1..256. */
 int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
                er_stream_t stream);
@@ -187,17 +198,27 @@ int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
 int er_advance_ex(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
                   uint32_t flags, er_stream_t stream);
 
-/* Copies the device error word to *code (host) and clears it; synchronises
- * `stream`.  Returns ER_OK when the word was 0, else ER_EDEVICE. */
+/* Copies the state's device error word to *code (host) and clears it;
+ * synchronises `stream`.  Returns ER_OK when the word was 0, else ER_EDEVICE.
+ * (The capacities that the device checks are those of [F-mem]: a full
+ * pending block or a chunk crossing it reports ER_ECAPACITY here.) */
 int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream);
+
+/* The same for the library's own error word, which the calls that take no
+ * state record into: er_rma_score (and er_rma_score_ex with dev_error NULL),
+ * er_rma_score_noalloc, and er_wait_selftest with st NULL.  One word per
+ * device, shared by every such call in the process: it holds the first code
+ * recorded since the last read.  Synchronises `stream`. */
+int er_last_call_error(int32_t* code, er_stream_t stream);
 
 /* Diagnostic for the failure path, no part of the method: one thread waits on
  * a fresh mbarrier (one expected arrival) through the bounded wait that every
  * kernel of the library uses for its pipeline barriers.  arrive = 1 completes
  * the barrier first (the wait returns at once, nothing is recorded); arrive =
  * 0 leaves it incomplete, so the wait gives up after ~2 s and records
- * ER_ETIMEOUT in st's device error word; the kernel then exits and the context
- * stays usable.  ER_EINVAL for a NULL state or another arrive value. */
+ * ER_ETIMEOUT in st's device error word (st NULL: the library's own word, read
+ * by er_last_call_error); the kernel then exits and the context stays usable.
+ * ER_EINVAL for another arrive value. */
 int er_wait_selftest(const er_state* st, int32_t arrive, er_stream_t stream);
 
 /* ------------------------------------------------------- hot-path steps */
@@ -235,6 +256,13 @@ int er_prepare_qkv_score(const er_bf16* w_qkv, const float* w1, er_bf16* out,
 int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
                  size_t ws_bytes, er_stream_t stream);
 
+/* er_rma_score with an explicit device error word: a bounded wait inside the
+ * scorer that gives up (its scores are then not valid) records ER_ETIMEOUT in
+ * *dev_error (a caller-owned device int32, e.g. a state's dev_error; NULL
+ * means the library's own word, as for er_rma_score). */
+int er_rma_score_ex(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
+                    size_t ws_bytes, int32_t* dev_error, er_stream_t stream);
+
 /* a3 without caller scratch.  The pages describe nothing like this; it exists
  * for callers that cannot hand the library any device memory beyond the
  * inputs and outputs, so cannot provide er_rma_score's workspace: for example
@@ -253,7 +281,9 @@ int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* 
  *  - Every call shares the one array: calls whose work overlaps on the GPU
  *    (different streams, or different threads on one device) race and give
  *    wrong scores; serialise them.  The array keeps the last call's contents;
- *    no part of it needs to start at zero. */
+ *    no part of it needs to start at zero.
+ *  - A bounded wait that gives up records ER_ETIMEOUT in the library's own
+ *    error word (a fixed device word too), read with er_last_call_error. */
 #define ER_SCORE_NOALLOC_MAX_TOKENS 256
 int er_rma_score_noalloc(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s,
                          er_stream_t stream);
@@ -298,7 +328,8 @@ int er_swa_rma_attend(const er_state* st, int32_t layer, const int32_t* seq_ids,
                       void* ws, size_t ws_bytes, er_stream_t stream);
 
 /* a1–a7 — one decode step of one layer for B sequences (one token each at
- * its meta pos): q/k/v projections of both branches, norm + RoPE, scores,
+ * its meta pos), the SWA∥RMA layer of [F-arch] with the memory rules of
+ * [N-rma]: q/k/v projections of both branches, norm + RoPE, scores,
  * window write (slot pos % 1024), pending append, the two reads,
  * out = W_o · bf16(o_swa + o_rma), and the commit of this layer for every
  * sequence whose block this token fills (pend_count + 1 == 256), decided on
@@ -310,7 +341,9 @@ int er_swa_rma_decode(const er_state* st, const er_layer_weights* w, int32_t lay
                       void* ws, size_t ws_bytes, er_stream_t stream);
 
 /* a8 — a prefill chunk of T tokens (1..256) of one sequence (state row
- * seq_id, a host int) at positions pos..pos+T-1.  Requires
+ * seq_id, a host int) at positions pos..pos+T-1: the layer of [F-arch] run
+ * causally over a chunk, each token appending its candidate [N-rma] within
+ * the capacities of [F-mem].  Requires
  * pend_count + T <= 256 (checked on the device).  Token i reads, causally,
  * window positions [t-1023, t] (old ring entries and the chunk's own tokens)
  * and the bank plus pending slots [0, pend_count + i]; the chunk enters the

@@ -26,7 +26,7 @@ __all__ = ["State", "LayerWeights", "qk_norm_rope", "rma_score", "rma_append_pen
            "advance", "state_init", "last_device_error", "launch_count", "profile_enable",
            "profile_read", "decode_workspace_bytes", "prefill_workspace_bytes",
            "attend_workspace_bytes", "score_workspace_bytes", "rma_score_noalloc",
-           "wait_selftest", "ERError"]
+           "wait_selftest", "last_call_error", "ERError"]
 
 
 class State:
@@ -150,11 +150,22 @@ def last_device_error(st: State, stream=None) -> int:
     return int(code.value)
 
 
-def wait_selftest(st: State, arrive: bool, stream=None):
+def last_call_error(stream=None) -> int:
+    """The library's own error word (the calls that take no state), read and cleared."""
+    code = ctypes.c_int32(0)
+    rc = lib().er_last_call_error(ctypes.byref(code), stream_handle(stream))
+    if rc not in (_lib.ER_OK, _lib.ER_EDEVICE):
+        raise ERError("er_last_call_error", rc)
+    return int(code.value)
+
+
+def wait_selftest(st, arrive: bool, stream=None):
     """er_wait_selftest: a bounded device wait that completes (arrive=True) or
-    runs out (~2 s, ER_ETIMEOUT in the state's error word)."""
-    check("er_wait_selftest", lib().er_wait_selftest(st.ptr(), 1 if arrive else 0,
-                                                     stream_handle(stream, st.device)))
+    runs out (~2 s, ER_ETIMEOUT in the state's error word, or in the library's
+    own word when st is None)."""
+    check("er_wait_selftest", lib().er_wait_selftest(
+        st.ptr() if st is not None else None, 1 if arrive else 0,
+        stream_handle(stream, st.device if st is not None else None)))
 
 
 def qk_norm_rope(x: torch.Tensor, gain: torch.Tensor, pos: torch.Tensor, out=None, stream=None):
@@ -171,13 +182,16 @@ def score_workspace_bytes(n: int) -> int:
     return int(lib().er_score_workspace_bytes(n))
 
 
-def rma_score(w: LayerWeights, x: torch.Tensor, ws=None, stream=None):
+def rma_score(w: LayerWeights, x: torch.Tensor, ws=None, stream=None, dev_error=None):
+    """FP32 scores [n, 4].  dev_error: an optional device int32 tensor that receives
+    a device-side error code (default: the library's own word, last_call_error)."""
     n = x.numel() // HIDDEN
     s = torch.empty(n, NG, dtype=torch.float32, device=x.device)
     ws = _ws(score_workspace_bytes(n), x.device, ws)
-    check("er_rma_score", lib().er_rma_score(w.ptr(), dev_ptr(x, torch.bfloat16, "x"), n,
-                                             dev_ptr(s), dev_ptr(ws), ws.numel(),
-                                             stream_handle(stream, x.device)))
+    err = dev_ptr(dev_error, torch.int32, "dev_error") if dev_error is not None else None
+    check("er_rma_score_ex", lib().er_rma_score_ex(w.ptr(), dev_ptr(x, torch.bfloat16, "x"), n,
+                                                   dev_ptr(s), dev_ptr(ws), ws.numel(), err,
+                                                   stream_handle(stream, x.device)))
     return s
 
 

@@ -56,6 +56,7 @@ EXPORTS = {
                                      ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p]),
     "er_last_device_error": (ctypes.c_int, [ctypes.POINTER(CState),
                                             ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
+    "er_last_call_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
     "er_qk_norm_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "er_score_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
@@ -66,6 +67,9 @@ EXPORTS = {
     "er_rma_score": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p, ctypes.c_int32,
                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                     ctypes.c_void_p]),
+    "er_rma_score_ex": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p,
+                                       ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]),
     "er_rma_score_noalloc": (ctypes.c_int, [ctypes.POINTER(CWeights), ctypes.c_void_p,
                                             ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p]),
     "er_rma_append_pending": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_int32,

@@ -167,6 +167,7 @@ inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 void count_launches(int n);                 // bookkeeping for er_launch_count
 int launch_status();                        // ER_OK or ER_ECUDA after a launch
 int num_sms();                              // SMs of the current device (cached)
+int32_t* call_error_word();                 // device address of the stateless calls' error word
 
 // Workspace carving: 256-byte aligned sub-buffers.  With a null base the
 // returned "pointers" are the byte offsets themselves (layout computation).

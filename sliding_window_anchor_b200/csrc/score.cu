@@ -400,9 +400,10 @@ int er_rma_score_noalloc(const er_layer_weights* w, const er_bf16* x, int32_t n,
     }
     scratch = g_noalloc_ptr[dev];
   }
+  int32_t* err = call_error_word();  // also a fixed device word: nothing allocated
+  if (!err) return ER_ECUDA;
   // every scratch word a call reads was written earlier in the same call: nothing to clear
-  return launch_score(w->w1, w->w1_split, w->w2, x, n, s, scratch, nullptr,
-                      (cudaStream_t)stream);
+  return launch_score(w->w1, w->w1_split, w->w2, x, n, s, scratch, err, (cudaStream_t)stream);
 }
 
 size_t er_score_workspace_bytes(int32_t n) {
@@ -410,15 +411,22 @@ size_t er_score_workspace_bytes(int32_t n) {
   return score_scratch_bytes(n);
 }
 
-int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
-                 size_t ws_bytes, er_stream_t stream) {
+int er_rma_score_ex(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
+                    size_t ws_bytes, int32_t* dev_error, er_stream_t stream) {
   if (!w || n < 0 || (n > 0 && (!w->w1 || !w->w2 || !x || !s || !ws))) return ER_EINVAL;
   if (n == 0) return ER_OK;
   if (!aligned16(w->w1) || !aligned16(ws) || !aligned16(x) ||
       (w->w1_split && !aligned16(w->w1_split)))
     return ER_EINVAL;
   if (ws_bytes < er_score_workspace_bytes(n)) return ER_ECAPACITY;
-  return launch_score(w->w1, w->w1_split, w->w2, x, n, s, ws, nullptr, (cudaStream_t)stream);
+  int32_t* err = dev_error ? dev_error : call_error_word();
+  if (!err) return ER_ECUDA;
+  return launch_score(w->w1, w->w1_split, w->w2, x, n, s, ws, err, (cudaStream_t)stream);
+}
+
+int er_rma_score(const er_layer_weights* w, const er_bf16* x, int32_t n, float* s, void* ws,
+                 size_t ws_bytes, er_stream_t stream) {
+  return er_rma_score_ex(w, x, n, s, ws, ws_bytes, nullptr, stream);
 }
 
 }  // extern "C"

@@ -165,15 +165,62 @@ __global__ void k_wait_selftest(int32_t* err, int arrive) {
 
 }  // namespace er
 
+// The error word of the calls that take no state (the standalone scorers): a
+// fixed device word inside the library, one per GPU that loads it.  Host code
+// cannot hand its name to a kernel (on the host it only stands in for the
+// symbol), so call_error_word() looks its device address up once per device.
+static __device__ __align__(16) int32_t g_call_error[4];
+
+namespace er {
+namespace {
+std::mutex g_call_error_mu;
+int32_t* g_call_error_ptr[64] = {nullptr};
+}  // namespace
+
+int32_t* call_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_call_error_mu);
+  if (!g_call_error_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_call_error) != cudaSuccess || !p) return nullptr;
+    g_call_error_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  return g_call_error_ptr[dev];
+}
+
+namespace {
+// Copies a device error word to the host, clears it, waits for both.
+int read_and_clear(int32_t* word, int32_t* code, cudaStream_t s) {
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, word, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return ER_ECUDA;
+  if (cudaMemsetAsync(word, 0, sizeof(int32_t), s) != cudaSuccess) return ER_ECUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ER_ECUDA;
+  *code = h;
+  return h == 0 ? ER_OK : ER_EDEVICE;
+}
+}  // namespace
+}  // namespace er
+
 using namespace er;
 
 extern "C" {
 
 int er_wait_selftest(const er_state* st, int32_t arrive, er_stream_t stream) {
-  if (!st || !st->dev_error || (arrive != 0 && arrive != 1)) return ER_EINVAL;
-  k_wait_selftest<<<1, 32, 0, (cudaStream_t)stream>>>(st->dev_error, arrive);
+  if ((st && !st->dev_error) || (arrive != 0 && arrive != 1)) return ER_EINVAL;
+  int32_t* err = st ? st->dev_error : call_error_word();
+  if (!err) return ER_ECUDA;
+  k_wait_selftest<<<1, 32, 0, (cudaStream_t)stream>>>(err, arrive);
   count_launches(1);
   return launch_status();
+}
+
+int er_last_call_error(int32_t* code, er_stream_t stream) {
+  if (!code) return ER_EINVAL;
+  int32_t* word = call_error_word();
+  if (!word) return ER_ECUDA;
+  return read_and_clear(word, code, (cudaStream_t)stream);
 }
 
 size_t er_state_bytes(int32_t s_max, int32_t n_layers) {
@@ -231,15 +278,7 @@ int er_advance(const er_state* st, const int32_t* seq_ids, int32_t n, int32_t T,
 
 int er_last_device_error(const er_state* st, int32_t* code, er_stream_t stream) {
   if (!st || !st->dev_error || !code) return ER_EINVAL;
-  int32_t h = 0;
-  cudaStream_t s = (cudaStream_t)stream;
-  if (cudaMemcpyAsync(&h, st->dev_error, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
-      cudaSuccess)
-    return ER_ECUDA;
-  if (cudaMemsetAsync(st->dev_error, 0, sizeof(int32_t), s) != cudaSuccess) return ER_ECUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return ER_ECUDA;
-  *code = h;
-  return h == 0 ? ER_OK : ER_EDEVICE;
+  return read_and_clear(st->dev_error, code, (cudaStream_t)stream);
 }
 
 const char* er_error_string(int code) {

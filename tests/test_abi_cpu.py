@@ -130,10 +130,19 @@ def test_host_validation_rejects_before_enqueue(L):
     assert L.er_swa_rma_prefill_chunk_ex(ctypes.byref(st), ctypes.byref(w), 0, 0, nul, 16, nul,
                                          nul, 0, 8, nul) == -1
     assert L.er_launch_count() == before
-    # the bounded-wait diagnostic: only arrive 0 or 1, and a state
+    # the bounded-wait diagnostic: only arrive 0 or 1 (with a state or, NULL, the
+    # library's own word); a state without an error word is refused
     before = L.er_launch_count()
-    assert L.er_wait_selftest(None, 0, nul) == -1
+    assert L.er_wait_selftest(None, 2, nul) == -1
     assert L.er_wait_selftest(ctypes.byref(st), 2, nul) == -1
+    no_word = CState()
+    ctypes.memmove(ctypes.byref(no_word), ctypes.byref(st), ctypes.sizeof(st))
+    no_word.dev_error = None
+    assert L.er_wait_selftest(ctypes.byref(no_word), 0, nul) == -1
+    # the scorer with an explicit error word checks its arguments the same way
+    assert L.er_rma_score_ex(None, nul, 1, nul, nul, 0, nul, nul) == -1
+    assert L.er_rma_score_ex(ctypes.byref(w), nul, 0, nul, nul, 0, nul, nul) == 0
+    assert L.er_last_call_error(None, nul) == -1
     assert L.er_launch_count() == before
     # the fused q/k/v + W1-term weights: NULL, unaligned or overlapping buffers are refused
     base = 1 << 40

@@ -6,6 +6,7 @@ the same generator numbers.  Bars: the stated |Δ| <= 1e-2 + 1e-2·|oracle| on
 every layer output, and kept anchor sets equal except where two records'
 scores differ by less than 1e-5 relative at the keep/evict boundary.
 """
+import time
 from concurrent.futures import ThreadPoolExecutor
 
 import pytest
@@ -230,6 +231,29 @@ def test_bounded_wait_runs_out_and_the_context_survives(sab):
     ref = oracle.norm_rope(x, g, pos)
     assert (got == ref).double().mean() > 0.99
     assert sab.last_device_error(st) == 0
+
+
+def test_stateless_calls_report_a_wait_that_gave_up(sab):
+    """The calls that take no state (the standalone scorers) record into the
+    library's own error word: a bounded wait run out through it is reported by
+    er_last_call_error, which then reads clear; the scorer with an explicit word
+    records nothing on a normal call and its scores are unchanged."""
+    assert sab.last_call_error() in (0, -5)  # clear whatever an earlier test left
+    sab.wait_selftest(None, arrive=True)
+    assert sab.last_call_error() == 0
+    t0 = time.time()
+    sab.wait_selftest(None, arrive=False)
+    assert sab.last_call_error() == -5  # ER_ETIMEOUT
+    assert 1.5 < time.time() - t0 < 30.0
+    assert sab.last_call_error() == 0
+    seed = 321
+    gw, wdev = H.gpu_weights(seed, 0)
+    x = synth.normal((64, 2560), seed, synth.MISC, torch.bfloat16, "cuda")
+    word = torch.zeros(4, dtype=torch.int32, device="cuda")
+    s_ex = sab.rma_score(gw, x, dev_error=word)
+    s_lib = sab.rma_score(gw, x)
+    assert torch.equal(s_ex, s_lib)
+    assert int(word[0]) == 0 and sab.last_call_error() == 0
 
 
 RMA_ARRAYS = ("bank_k", "bank_v", "pend_k", "pend_v", "bank_score", "pend_score", "bank_pos",
