@@ -47,6 +47,8 @@ def parse():
                     help="skip the decode pass with the RMA switched off (the ablation)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph pass (one captured graph per decode step)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the B=1 (one layer) and B=64 (8 layers) decode configurations")
     ap.add_argument("--prefill-chunks", type=int, default=512,
                     help="256-token chunks of the prefill stream (512 = 131072 tokens)")
     ap.add_argument("--kernel", default="step",
@@ -394,39 +396,26 @@ def run_ours(args, rank, world, local_rank):
     pf = None
     if not args.no_prefill_bench and rank == 0:
         pf = prefill_bench(dev, args.prefill_chunks)
+    cfgs = None
+    if not args.no_configs and rank == 0:
+        cfgs = {r["workload"]: r for r in (decode_config_bench(dev, 0),
+                                           decode_config_bench(dev, 2))}
     return dict(ms=ms, launches=launches, clocks=clk, attend_ms=attend_ms, attend_n=attend_n,
                 fills=fills, commits=commits, e2e=e2e, commit_microbench=cm, prefill=pf,
-                graph=graph, rma_off=rma_off)
+                graph=graph, rma_off=rma_off, configs=cfgs)
 
 
 # ------------------------------------------------------- commit microbench
 
-def seed_commit_workload(st, seed, rep, dev):
-    """The commit workload: every (sequence, layer, group) holds a full bank and a
-    full pending block; scores N(0,1) with ~5% exact ties inside each merge; K/V
-    rows N(0,1).  Repetition r re-seeds the pending block (scores, positions
-    t0+256r+j) on top of the bank the previous repetition left."""
-    import torch
-    import synth
-    from synth import workloads as wl
-    n, L = st.s_max, st.n_layers
-    if rep == 0:
-        wl.seed_state(st.arrays(), range(n), L, T0, "full", seed, [None] * L, None, device=dev,
-                      plain_keys=True, dup_scores=True)
-    else:
-        synth.fill_normal_dup_(st.pend_score, seed + rep, synth.PEND_SCORE, 256, 20)
-    j = torch.arange(256, dtype=torch.int32, device=dev)
-    st.pend_pos.copy_((T0 + 256 * rep + j).view(1, 1, 1, 256).expand_as(st.pend_pos))
-    st.meta[:, 0] = T0 + 256 * (rep + 1)
-    st.meta[:, 1] = 256
-    st.meta[:, 2] = 1024
-
-
 def commit_microbench(st, dev, reps=3):
     """Times er_rma_commit(layer=-1) over every sequence: B x 8 layers x 4 groups
-    independent top-1024-of-1280 merges.  Algorithmic bytes per merge: the 1280
-    keys (score + position, 8 B each) read, plus each moved record's K and V row
-    read and written (2 x 1 KiB) with its score and position (2 x 8 B)."""
+    independent top-1024-of-1280 merges of the commit workload.  Every repetition
+    is a fresh workload (scores N(0,1) with ~5% exact ties, bank and pending full;
+    synth.workloads.seed_commit_workload), the first one untimed.  Algorithmic bytes
+    per merge: the 1280 keys (score + position, 8 B each) read, plus each moved
+    record's K and V row read and written (2 x 1 KiB) with its score and position
+    (2 x 8 B).  The same seeds are checked bit-exact against the oracle by
+    tests/test_gpu_steps.py::test_commit_full_size_workload_matches_oracle."""
     import torch
     import sliding_window_anchor_b200 as sab
     from synth import workloads as wl
@@ -435,7 +424,7 @@ def commit_microbench(st, dev, reps=3):
     merges = st.s_max * st.n_layers * 4
     times, moved = [], []
     for rep in range(reps + 1):
-        seed_commit_workload(st, seed, rep, dev)
+        wl.seed_commit_workload(st.arrays(), range(st.s_max), st.n_layers, T0, seed, rep, dev)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
@@ -446,7 +435,7 @@ def commit_microbench(st, dev, reps=3):
             raise RuntimeError("device error in the commit microbench")
         if rep > 0:  # the first repetition is the warm-up
             times.append(e0.elapsed_time(e1))
-            moved.append(int((st.bank_pos >= T0 + 256 * rep).sum()))
+            moved.append(int((st.bank_pos >= T0).sum()))  # pending positions are T0..T0+255
     i = sorted(range(reps), key=lambda k: times[k])[reps // 2]
     ms, m = times[i], moved[i]
     alg = merges * 1280 * 8 + m * (2 * 1024 + 16)
@@ -454,8 +443,11 @@ def commit_microbench(st, dev, reps=3):
     return {"workload": f"commit_b{st.s_max}_l{st.n_layers}", "merges": merges, "ms": ms,
             "merges_per_s": merges / (ms / 1e3),
             "sequence_commits_per_s": st.s_max / (ms / 1e3),
-            "moved_records": m, "alg_bytes": alg, "achieved_gbs": alg / (ms / 1e3) / 1e9,
-            "frac": alg / (ms / 1e3) / 1e9 / hbm, "peak_gbs": hbm, "peak_kind": kind}
+            "moved_records": m, "moved_per_merge": m / merges, "alg_bytes": alg,
+            "achieved_gbs": alg / (ms / 1e3) / 1e9,
+            "frac": alg / (ms / 1e3) / 1e9 / hbm, "peak_gbs": hbm, "peak_kind": kind,
+            "reps": reps, "note": "median of the timed repetitions, each a freshly seeded "
+                                  "workload (i.i.d. scores, ~5% ties)"}
 
 
 def prefill_attention_flops(t0: int, T: int, c: int, p0: int) -> int:
@@ -554,6 +546,101 @@ def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2,
             "graph": None if graph_ms is None else {
                 "ms": graph_ms, "tok_per_s": chunks * T / (graph_ms / 1e3),
                 "note": "same chunks replayed from one captured CUDA graph per chunk"}}
+
+
+# bytes every decode layer step reads from the weights: the fused q/k/v + W1-term
+# matrix (13056 x 2560 BF16), W_o (2560 x 4096 BF16), W2 and the four gains
+WEIGHT_BYTES_PER_LAYER = 13056 * 2560 * 2 + 2560 * 4096 * 2 + 4 * 256 * 4 + 4 * 256 * 2
+
+
+def decode_config_bench(dev, cfg_index: int, n_x: int = 16, warmup: int = 3):
+    """One spec decode configuration end to end on the device: its state
+    seeded as the tests seed it, then all of its steps (a1-a7 per layer, device-
+    gated commits, the advance) replayed from CUDA graphs (one per distinct input
+    buffer, inputs resident).  Reports tok/s, ms/step and the fraction of the byte
+    floor (every layer step reads its weights once and its state rows once, at the
+    measured HBM bandwidth); an eager pass times the read kernel's launches."""
+    import torch
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+    cfg, seed = wl.CONFIGS[cfg_index], wl.seed_of(cfg_index)
+    Bc, L, steps, t0 = cfg["B"], cfg["n_layers"], cfg["steps"], cfg["t0"]
+    weights = [sab.LayerWeights.from_dict(wl.make_weights(seed, l, device=dev))
+               for l in range(L)]
+    st = sab.State(Bc, L, device=dev)
+
+    def normrope(x, g, pos):
+        return sab.qk_norm_rope(x.contiguous(), g, pos.to(torch.int32).contiguous())
+
+    fills = wl.seed_state(st.arrays(), range(Bc), L, t0, cfg["pend"], seed,
+                          [w.t for w in weights], normrope, device=dev).cpu().tolist()
+    snap = st.blob.clone()
+    ids = torch.arange(Bc, dtype=torch.int32, device=dev)
+    ws = torch.empty(sab.decode_workspace_bytes(Bc), dtype=torch.uint8, device=dev)
+    n_x = min(n_x, steps)
+    xs = [[wl.make_x(seed, l, s, range(Bc), device=dev) for l in range(L)] for s in range(n_x)]
+    outs = [torch.empty(Bc, 2560, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(s):
+        for l in range(L):
+            sab.swa_rma_decode(st, weights[l], l, ids, xs[s % n_x][l], out=outs[l], ws=ws)
+        sab.advance(st, ids)
+
+    # eager pass over the first steps: the read kernel's own launches, timed
+    for s in range(warmup):
+        step(s)
+    torch.cuda.synchronize(dev)
+    k_eager = min(steps, 32)
+    sab.profile_read(reset=True)
+    sab.profile_enable(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for s in range(k_eager):
+        step(s)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    sab.profile_enable(False)
+    a_ms, a_n = sab.profile_read(reset=True)
+    eager_ms = e0.elapsed_time(e1)
+    a_alg = algorithmic_read_bytes(fills, warmup, k_eager) * L
+    # the whole configuration from its seeded start, replayed from graphs
+    st.blob.copy_(snap)
+    stream_g = torch.cuda.Stream(dev)
+    graphs = []
+    for s in range(n_x):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream_g):
+            step(s)
+        graphs.append(g)
+    st.blob.copy_(snap)  # capture launches nothing; restore anyway
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for s in range(steps):
+        graphs[s % n_x].replay()
+    g1.record(stream)
+    torch.cuda.synchronize(dev)
+    del graphs
+    if sab.last_device_error(st) != 0:
+        raise RuntimeError(f"device error in the config {cfg_index} bench")
+    ms = g0.elapsed_time(g1)
+    hbm, kind = peaks()
+    state_bytes = algorithmic_read_bytes(fills, 0, steps) * L
+    floor_bytes = state_bytes + steps * L * WEIGHT_BYTES_PER_LAYER
+    floor_ms = floor_bytes / (hbm * 1e9) * 1e3
+    commits = sum(1 for f in fills for s in range(steps) if (f + s) % 256 == 255)
+    per_read = a_ms / a_n if a_n else None
+    return {"workload": cfg["name"], "B": Bc, "layers": L, "t0": t0, "steps": steps,
+            "tok_per_s": Bc * steps / (ms / 1e3), "ms_per_step": ms / steps,
+            "ms_per_layer_step": ms / (steps * L), "commits": commits,
+            "floor_ms_per_step": floor_ms / steps, "floor_frac": floor_ms / ms,
+            "floor_bytes_per_step": floor_bytes / steps,
+            "eager_ms_per_step": eager_ms / k_eager,
+            "attend_avg_launch_ms": per_read,
+            "attend_frac": (a_alg / a_n) / (per_read / 1e3) / 1e9 / hbm if a_n else None,
+            "peak_gbs": hbm, "peak_kind": kind,
+            "launch": "one CUDA graph per step (inputs resident, %d buffers)" % n_x}
 
 
 SWEEP_BATCHES = (1, 2, 4, 8, 16, 32, 64, 96, 128, 160, 192, 224, 256, 288, 320, 352, 384, 448,
@@ -786,26 +873,16 @@ def oracle_tokens_per_s(budget_s=12.0, max_threads=8):
 
 def oracle_merges_per_s(budget_s=4.0):
     """The oracle's commit (a full sort of the 1280 records, then the moves) on the
-    commit workload, one thread: one sequence x 8 layers x 4 groups per call, the
-    pending block re-filled (scores with ~5% ties, fresh positions) before each."""
-    import torch
+    commit workload, one thread: one sequence x 8 layers x 4 groups per call, each a
+    freshly seeded repetition (as the GPU microbench seeds them)."""
     import oracle
-    import synth
     from synth import workloads as wl
     seed = wl.seed_of(1)
     ost = oracle.OracleState(1, LAYERS)
     arrays = {n: getattr(ost, n) for n in oracle.OracleState.ARRAYS}
-    wl.seed_state(arrays, [0], LAYERS, T0, "full", seed, [None] * LAYERS, None, device="cpu",
-                  plain_keys=True, dup_scores=True)
-    j = torch.arange(256, dtype=torch.int32)
     merges, spent, rep = 0, 0.0, 0
     while spent < budget_s:
-        if rep > 0:
-            synth.fill_normal_dup_(ost.pend_score, seed + rep, synth.PEND_SCORE, 256, 20)
-        ost.pend_pos.copy_((T0 + 256 * rep + j).view(1, 1, 1, 256).expand_as(ost.pend_pos))
-        ost.meta[0, 0] = T0 + 256 * (rep + 1)
-        ost.meta[0, 1] = 256
-        ost.meta[0, 2] = 1024
+        wl.seed_commit_workload(arrays, [rep % 512], LAYERS, T0, seed, rep, "cpu")
         t0 = time.time()
         ost.commit(-1, 0)
         spent += time.time() - t0
@@ -901,6 +978,7 @@ def main():
     # headline: the steps replayed from CUDA graphs when that pass ran, else the eager pass
     g = r["graph"]
     head_ms = g["ms"] if g else r["ms"]
+    step_bytes = alg / args.steps + LAYERS * WEIGHT_BYTES_PER_LAYER
     head_launches = g["launches_per_step"] * args.steps if g else r["launches"]
     secs = head_ms / 1e3
     line = {
@@ -915,7 +993,15 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "k_attend", "achieved": achieved, "peak": hbm,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / hbm,
                      "traffic": traffic, "alg_bytes_per_launch": per_launch,
-                     "avg_launch_ms": avg_ms, "launches": r["attend_n"]},
+                     "avg_launch_ms": avg_ms, "launches": r["attend_n"],
+                     "above_peak": achieved > hbm,
+                     "peak_test": "a read+write device copy (b.copy_(a), 1 Gi BF16 elements); "
+                                  "a read-only stream can exceed it",
+                     "step": {"bytes": step_bytes, "ms": head_ms / args.steps,
+                              "achieved": step_bytes / (head_ms / args.steps / 1e3) / 1e9,
+                              "frac": step_bytes / (head_ms / args.steps / 1e3) / 1e9 / hbm,
+                              "note": "the whole step: state rows of all reads plus every "
+                                      "layer's weights, over the step time"}},
         "cpu_baseline": cpu,
         "e2e": r["e2e"],
         "gpu_launches": head_launches,
@@ -923,6 +1009,7 @@ def main():
         "commit_microbench": r["commit_microbench"],
         "prefill": r["prefill"],
         "rma_off": r["rma_off"],
+        "configs": r["configs"],
         "eager": {"value": whole_job_tokens_per_s(world, B, args.steps, r["ms"]),
                   "ms_per_step": r["ms"] / args.steps, "gpu_launches": r["launches"],
                   "note": "the same steps launched call by call through the binding; "

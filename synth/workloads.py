@@ -202,3 +202,45 @@ def seed_state(arrays: dict, seqs, n_layers: int, t0: int, pend_mode: str, seed:
     meta[:, 2] = BANK
     meta[:, 3] = 0
     return fills
+
+
+# ------------------------------------------------------- commit workload
+
+def seed_commit_workload(arrays: dict, seqs, n_layers: int, t0: int, seed: int, rep: int,
+                         device="cpu") -> None:
+    """The commit microbench workload, repetition `rep`: every (sequence, layer,
+    group) holds a full bank (positions stratified below t0-1024) and a full pending
+    block (positions t0..t0+255), scores N(0,1) with ~5% exact ties inside each
+    merge, meta {t0+256, 256, 1024, 0}.  rep 0 also fills the K/V rows with N(0,1)
+    (plain, un-normed); a later repetition draws fresh scores (stream keyed by
+    seed and rep) and restores the positions and metadata, leaving the K/V rows as
+    they are (their contents do not change which records a merge keeps or moves)."""
+    seqs = list(seqs)
+    n, L = len(seqs), n_layers
+    if rep == 0:
+        seed_state(arrays, seqs, L, t0, "full", seed, [None] * L, None, device=device,
+                   plain_keys=True, dup_scores=True)
+    else:
+        seed_r = seed + 7919 * rep
+        ident = seqs == list(range(n))
+        per = L * NG * (BANK + PEND)
+        sc = torch.empty(n, L, NG, BANK + PEND, dtype=torch.float32, device=device)
+        width = max(1, (t0 - WIN) // BANK)
+        if ident:
+            synth.fill_normal_dup_(sc, seed_r, synth.BANK_SCORE, BANK + PEND, 20)
+            synth.fill_strata_(arrays["bank_pos"], seed, synth.BANK_POS, BANK, width)
+        else:
+            for i, s in enumerate(seqs):
+                synth.fill_normal_dup_(sc[i], seed_r, synth.BANK_SCORE, BANK + PEND, 20,
+                                       index0=s * per)
+                synth.fill_strata_(arrays["bank_pos"][i], seed, synth.BANK_POS, BANK, width,
+                                   index0=s * L * NG * BANK)
+        arrays["bank_score"].copy_(sc[..., :BANK])
+        arrays["pend_score"].copy_(sc[..., BANK:])
+    j = torch.arange(PEND, dtype=torch.int32, device=device)
+    arrays["pend_pos"].copy_((t0 + j).view(1, 1, 1, PEND).expand_as(arrays["pend_pos"]))
+    meta = arrays["meta"]
+    meta[:, 0] = t0 + PEND
+    meta[:, 1] = PEND
+    meta[:, 2] = BANK
+    meta[:, 3] = 0

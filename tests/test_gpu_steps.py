@@ -258,30 +258,30 @@ def test_attend_many_queries_one_split(sab):
 
 def test_commit_full_size_workload_matches_oracle(sab):
     """The commit microbench workload at full size (512 sequences x 8 layers x 4 groups,
-    bank and pending full, ~5% exact score ties, plain K/V rows), one commit of every
-    layer; sampled sequences bit-exact against the oracle on the same seeded rows."""
+    bank and pending full, ~5% exact score ties, plain K/V rows), seeded as the bench
+    seeds it: repetition 0, then three repetitions with fresh scores (the timed ones).
+    After every commit of every layer, sampled sequences are bit-exact against the
+    oracle on the same seeded rows: every state array after repetition 0; the scores,
+    positions and metadata (which records are kept and in which slot) after the later
+    ones; and each later merge moves about 205 records on average."""
     seed, n, L, t0 = wl.seed_of(1), 512, 8, 32768
-
-    def seed_rows(arrays, seqs, device):
-        wl.seed_state(arrays, seqs, L, t0, "full", seed, [None] * L, None, device=device,
-                      plain_keys=True, dup_scores=True)
-        j = torch.arange(256, dtype=torch.int32, device=device)
-        arrays["pend_pos"].copy_((t0 + j).view(1, 1, 1, 256).expand_as(arrays["pend_pos"]))
-        arrays["meta"][:, 0] = t0 + 256
-        arrays["meta"][:, 1] = 256
-        arrays["meta"][:, 2] = 1024
-
     st = sab.State(n, L)
-    seed_rows(st.arrays(), range(n), "cuda")
     ids = torch.arange(n, dtype=torch.int32, device="cuda")
-    sab.rma_commit(st, -1, ids)
-    assert sab.last_device_error(st) == 0
-    for seq in (0, 257, 511):
-        ost = oracle.OracleState(1, L)
-        seed_rows({k: getattr(ost, k) for k in oracle.OracleState.ARRAYS}, [seq], "cpu")
-        ost.commit(-1, 0)
-        grow = H.download_row(st, seq)
-        for k in oracle.OracleState.ARRAYS:
-            assert torch.equal(grow[k], getattr(ost, k)[0]), (seq, k)
+    keys = ("bank_score", "pend_score", "bank_pos", "pend_pos", "meta")
+    for rep in range(4):
+        wl.seed_commit_workload(st.arrays(), range(n), L, t0, seed, rep, "cuda")
+        sab.rma_commit(st, -1, ids)
+        assert sab.last_device_error(st) == 0
+        for seq in (0, 257, 511):
+            ost = oracle.OracleState(1, L, kv=(rep == 0))
+            wl.seed_commit_workload({k: getattr(ost, k) for k in oracle.OracleState.ARRAYS},
+                                    [seq], L, t0, seed, rep, "cpu")
+            ost.commit(-1, 0)
+            grow = H.download_row(st, seq)
+            for k in (oracle.OracleState.ARRAYS if rep == 0 else keys):
+                assert torch.equal(grow[k], getattr(ost, k)[0]), (rep, seq, k)
+        if rep > 0:
+            moved = int((st.bank_pos >= t0).sum()) / (n * L * 4)
+            assert 195.0 < moved < 215.0, (rep, moved)
     del st
     torch.cuda.empty_cache()

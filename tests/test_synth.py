@@ -51,3 +51,27 @@ def test_workload_weights_shapes():
     pos = wl.window_positions(4096)
     assert sorted(pos.tolist()) == list(range(3072, 4096))
     assert all(int(p) % 1024 == s for s, p in enumerate(pos))
+
+
+def test_commit_workload_rows_do_not_depend_on_which_rows_are_seeded():
+    # a sampled sequence seeded alone gets the same keys as in the full batch, for the
+    # first repetition and a later one (the oracle side seeds sampled rows alone)
+    import oracle
+    from synth import workloads as wl
+    full = oracle.OracleState(6, 2, kv=False)
+    part = oracle.OracleState(2, 2, kv=False)
+    arrs = lambda o: {n: getattr(o, n) for n in oracle.OracleState.ARRAYS}
+    for rep in (1, 2):
+        wl.seed_commit_workload(arrs(full), range(6), 2, 32768, 99, rep)
+        wl.seed_commit_workload(arrs(part), [1, 4], 2, 32768, 99, rep)
+        for n in ("bank_score", "pend_score", "bank_pos", "pend_pos", "meta"):
+            assert torch.equal(getattr(full, n)[[1, 4]], getattr(part, n)), (rep, n)
+    # fresh scores per repetition, ~5% exact ties inside a merge
+    a = oracle.OracleState(1, 1, kv=False)
+    wl.seed_commit_workload(arrs(a), [0], 1, 32768, 99, 1)
+    s1 = torch.cat([a.bank_score[0, 0, 0], a.pend_score[0, 0, 0]])
+    wl.seed_commit_workload(arrs(a), [0], 1, 32768, 99, 2)
+    s2 = torch.cat([a.bank_score[0, 0, 0], a.pend_score[0, 0, 0]])
+    assert not torch.equal(s1, s2)
+    dup = 1280 - torch.unique(s1).numel()
+    assert 20 <= dup <= 120, dup
