@@ -28,18 +28,20 @@
  *  - Pointers named in a signature are DEVICE pointers unless marked (host).
  *    The caller allocates and frees all memory (state, weights, inputs,
  *    outputs, workspace); the library never allocates or frees device memory
- *    itself (cuBLAS keeps its own handle memory; er_rma_score_noalloc's
- *    scratch is a static device array) and never synchronises the stream,
+ *    itself (er_rma_score_noalloc's scratch and the library's error word are
+ *    fixed device arrays) and never synchronises the stream,
  *    except er_last_device_error and er_last_call_error, which read one word
  *    back.
  *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  A
- *    layer call may also run part of its work (the commit, beside o_proj) on
- *    a side stream the library keeps per device, forked from and joined back
- *    to `stream` inside the call, so everything still completes in `stream`
- *    order and the call can be captured in a CUDA graph.  The first layer
- *    call (and the first read or scorer call) on a device creates that
- *    device's library resources (cuBLAS handle, side stream, events, kernel
- *    attributes): make one such call before capturing on the device.
+ *    layer call may also run part of its work (the commit, beside the read
+ *    and o_proj) on a side stream that the library assigns to each caller
+ *    stream (16 per device; past 16 caller streams, some share one), forked
+ *    from and joined back to `stream` inside the call, so everything still
+ *    completes in `stream` order and the call can be captured in a CUDA
+ *    graph; calls on different caller streams do not wait on each other.
+ *    The first layer call on a device creates that device's side streams and
+ *    events, and the first call of each kind its kernel attributes: make one
+ *    such call on the device before capturing on it.
  *  - Those per-device resources, and the device addresses of the library's
  *    fixed device arrays, are made once per device and process and are not
  *    made again after cudaDeviceReset: do not call the library on a device
@@ -120,7 +122,27 @@ typedef struct er_state {
   int32_t *dev_error;
   int32_t s_max;
   int32_t n_layers;
+  int32_t pool; /* 1: the pooled anchor layout (ER_STATE_POOL), 0: the layout above */
 } er_state;
+
+/* The pooled anchor layout (a variant of the commit that moves no K/V row).
+ * The committed bank and the pending block of a group share ONE pool of 1280
+ * rows, with the same K/V bytes as bank + pending:
+ *   bank_k, bank_v BF16  [s_max][n_layers][4][1280][256]  pool rows
+ *   bank_score     FP32  [s_max][n_layers][4][1280]       score of the record in a slot
+ *   bank_pos       INT32 [s_max][n_layers][4][1280]       its source position, or
+ *                                                         0x7FFFFFFF for a free slot
+ *   pend_pos       INT32 [s_max][n_layers][4][256]        slot list: pending record j
+ *                                                         of the block lives in pool
+ *                                                         slot pend_pos[j]
+ *   pend_k, pend_v, pend_score: NULL.
+ * A record never moves once written.  A commit ranks the records of the
+ * occupied slots exactly as in the other layout and keeps the same records
+ * [F-arch], [N-rma]; it marks the slots of the evicted ones free and lists
+ * the 256 lowest free slots (ascending) as the next block's slots.  The reads
+ * take the whole pool of a group and skip free slots and records a query may
+ * not see (source position above the query's).  meta is unchanged. */
+#define ER_STATE_POOL 1u
 
 /* One SWA∥RMA layer's weights (device, caller-owned), nn.Linear layout [out][in]:
  *   w_qkv BF16 [12288][2560]: rows q_swa 0..4095 | k_swa 4096..5119 | v_swa 5120..6143 |
@@ -139,7 +161,7 @@ typedef struct er_state {
  *                             When set, the layer calls take a1 and the W1·x
  *                             product of a3 from ONE GEMM over it (FP32 output;
  *                             the projections are then rounded to BF16, the same
- *                             values a BF16-output GEMM gives) and apply SiLU and
+ *                             values a BF16-output er_linear gives) and apply SiLU and
  *                             W2 in the norm/RoPE kernel, so no separate scorer
  *                             launch runs (calls with ER_FLAG_RMA_OFF score
  *                             nothing and project from w_qkv with BF16 output).
@@ -169,10 +191,17 @@ size_t er_state_bytes(int32_t s_max, int32_t n_layers);
  * small, base is unaligned, or sizes are out of range. */
 int er_state_carve(void* base, size_t bytes, int32_t s_max, int32_t n_layers, er_state* out);
 
+/* The same with layout flags: 0, or ER_STATE_POOL for the pooled anchor layout
+ * (other bits: 0 bytes / ER_EINVAL). */
+size_t er_state_bytes_ex(int32_t s_max, int32_t n_layers, uint32_t flags);
+int er_state_carve_ex(void* base, size_t bytes, int32_t s_max, int32_t n_layers, uint32_t flags,
+                      er_state* out);
+
 /* Empties the listed sequences: meta := {0, 0, 0, 0}, i.e. the stream start
  * of [F-mem]: a window, bank and pending block of fixed capacity, all empty.
- * seq_ids: device int32 [n].  Row contents are left as they are (unread until
- * written). */
+ * In the pooled layout it also marks every pool slot free and lists slots
+ * 0..255 for the first block.  seq_ids: device int32 [n].  Row contents are
+ * left as they are (unread until written). */
 int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stream_t stream);
 
 /* End of one step of T tokens for the listed sequences, after every layer's
@@ -229,6 +258,22 @@ int er_wait_selftest(const er_state* st, int32_t arrive, er_stream_t stream);
  * [n_rows][256] (may alias); gain: BF16 [256]; pos: INT32 [n_rows]. */
 int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, const er_bf16* gain,
                     const int32_t* pos, er_stream_t stream);
+
+/* a1 / a6 — the layer's dense projections on their own [F-arch]: y = x · wᵀ
+ * with x BF16 [T][K] and w BF16 [F][K] (row-major, the nn.Linear layout), FP32
+ * accumulation on the tensor cores; y is BF16 (y_fp32 = 0, round to nearest
+ * even) or FP32 (y_fp32 = 1), [T][ldy] with ldy >= F.  The layer calls use
+ * it for x·W_qkvᵀ (F = 12288, or 13056 with the scorer's W1 terms, K = 2560)
+ * and for the shared o_proj (F = 2560, K = 4096).  F a multiple of 256, K of
+ * 64, T >= 0; x, w, y 16-byte aligned; ws 256-byte aligned, at least
+ * er_linear_workspace_bytes(T, F, K) (0 for bad sizes), reusable by calls
+ * ordered on one stream.  The summation order is fixed for given (T, F, K):
+ * the same inputs give the same bits.  A bounded wait that gives up records
+ * ER_ETIMEOUT in *dev_error (NULL: the library's own word). */
+size_t er_linear_workspace_bytes(int32_t T, int32_t F, int32_t K);
+int er_linear(const er_bf16* x, int32_t T, const er_bf16* w, int32_t F, int32_t K, void* y,
+              int32_t y_fp32, int32_t ldy, void* ws, size_t ws_bytes, int32_t* dev_error,
+              er_stream_t stream);
 
 /* a3 — retention scores [F-arch], [N-rma]: s = W2 · SiLU(W1 · x) with FP32
  * accuracy: W1 is taken as three BF16 terms hi + mid + lo (residual below

@@ -26,7 +26,8 @@ __all__ = ["State", "LayerWeights", "qk_norm_rope", "rma_score", "rma_append_pen
            "advance", "state_init", "last_device_error", "launch_count", "profile_enable",
            "profile_read", "decode_workspace_bytes", "prefill_workspace_bytes",
            "attend_workspace_bytes", "score_workspace_bytes", "rma_score_noalloc",
-           "wait_selftest", "last_call_error", "ERError"]
+           "wait_selftest", "last_call_error", "linear", "linear_workspace_bytes",
+           "ERError"]
 
 
 class State:
@@ -36,27 +37,36 @@ class State:
     ARRAYS = ("win_k", "win_v", "bank_k", "bank_v", "pend_k", "pend_v", "bank_score",
               "pend_score", "bank_pos", "pend_pos", "meta")
 
-    def __init__(self, s_max: int, n_layers: int = 8, device="cuda"):
+    def __init__(self, s_max: int, n_layers: int = 8, device="cuda", pool: bool = False):
+        """pool=True: the pooled anchor layout (ER_STATE_POOL): bank_k / bank_v /
+        bank_score / bank_pos hold 1280 pool slots per group, pend_pos the groups'
+        256-entry slot lists, and there are no pend_k / pend_v / pend_score."""
         L = lib()
-        nbytes = L.er_state_bytes(s_max, n_layers)
+        flags = _lib.ER_STATE_POOL if pool else 0
+        nbytes = L.er_state_bytes_ex(s_max, n_layers, flags)
         if nbytes == 0:
             raise ValueError("bad state size")
-        self.s_max, self.n_layers = s_max, n_layers
+        self.s_max, self.n_layers, self.pool = s_max, n_layers, pool
         self.device = torch.device(device)
         self.blob = torch.zeros(nbytes, dtype=torch.uint8, device=self.device)
         self.c = _lib.CState()
-        check("er_state_carve", L.er_state_carve(ctypes.c_void_p(self.blob.data_ptr()), nbytes,
-                                                 s_max, n_layers, ctypes.byref(self.c)))
+        check("er_state_carve_ex", L.er_state_carve_ex(ctypes.c_void_p(self.blob.data_ptr()),
+                                                       nbytes, s_max, n_layers, flags,
+                                                       ctypes.byref(self.c)))
         base = self.blob.data_ptr()
         g = (s_max, n_layers, NG)
+        nb = BANK + PEND if pool else BANK
         spec = {
             "win_k": (torch.bfloat16, g + (WIN, D)), "win_v": (torch.bfloat16, g + (WIN, D)),
-            "bank_k": (torch.bfloat16, g + (BANK, D)), "bank_v": (torch.bfloat16, g + (BANK, D)),
-            "pend_k": (torch.bfloat16, g + (PEND, D)), "pend_v": (torch.bfloat16, g + (PEND, D)),
-            "bank_score": (torch.float32, g + (BANK,)), "pend_score": (torch.float32, g + (PEND,)),
-            "bank_pos": (torch.int32, g + (BANK,)), "pend_pos": (torch.int32, g + (PEND,)),
+            "bank_k": (torch.bfloat16, g + (nb, D)), "bank_v": (torch.bfloat16, g + (nb, D)),
+            "bank_score": (torch.float32, g + (nb,)), "bank_pos": (torch.int32, g + (nb,)),
+            "pend_pos": (torch.int32, g + (PEND,)),
             "meta": (torch.int32, (s_max, 4)), "dev_error": (torch.int32, (4,)),
         }
+        if not pool:
+            spec.update({"pend_k": (torch.bfloat16, g + (PEND, D)),
+                         "pend_v": (torch.bfloat16, g + (PEND, D)),
+                         "pend_score": (torch.float32, g + (PEND,))})
         for name, (dt, shape) in spec.items():
             off = getattr(self.c, name) - base
             n = 1
@@ -69,7 +79,37 @@ class State:
         return ctypes.byref(self.c)
 
     def arrays(self):
+        if self.pool:
+            raise ValueError("the pooled layout has no pending arrays; see pool_from_plain")
         return {n: getattr(self, n) for n in self.ARRAYS}
+
+    def pool_from_plain(self, plain: "State", rows=None):
+        """Fill this pooled state's rows from a state in the plain layout holding the
+        same records: pool slots 0..1023 take the bank slots, 1024..1279 the pending
+        block (slot list 1024 + j), slots past the counts are free.  Copies only."""
+        if not self.pool or plain.pool:
+            raise ValueError("pool_from_plain copies a plain state into a pooled one")
+        rows = range(min(self.s_max, plain.s_max)) if rows is None else rows
+        free = 0x7FFFFFFF
+        for r in rows:
+            c, p = int(plain.meta[r, 2]), int(plain.meta[r, 1])
+            self.win_k[r].copy_(plain.win_k[r])
+            self.win_v[r].copy_(plain.win_v[r])
+            self.bank_k[r, :, :, :BANK].copy_(plain.bank_k[r])
+            self.bank_k[r, :, :, BANK:].copy_(plain.pend_k[r])
+            self.bank_v[r, :, :, :BANK].copy_(plain.bank_v[r])
+            self.bank_v[r, :, :, BANK:].copy_(plain.pend_v[r])
+            self.bank_score[r, :, :, :BANK].copy_(plain.bank_score[r])
+            self.bank_score[r, :, :, BANK:].copy_(plain.pend_score[r])
+            self.bank_pos[r, :, :, :BANK].copy_(plain.bank_pos[r])
+            self.bank_pos[r, :, :, BANK:].copy_(plain.pend_pos[r])
+            self.bank_pos[r, :, :, c:BANK] = free
+            self.bank_pos[r, :, :, BANK + p:] = free
+            self.bank_score[r, :, :, c:BANK] = 0.0
+            self.bank_score[r, :, :, BANK + p:] = 0.0
+            self.pend_pos[r].copy_(torch.arange(BANK, BANK + PEND, dtype=torch.int32,
+                                                device=self.device).expand_as(self.pend_pos[r]))
+            self.meta[r].copy_(plain.meta[r])
 
 
 class LayerWeights:
@@ -175,6 +215,27 @@ def qk_norm_rope(x: torch.Tensor, gain: torch.Tensor, pos: torch.Tensor, out=Non
         dev_ptr(x, torch.bfloat16, "x"), dev_ptr(out, torch.bfloat16, "out"), rows,
         dev_ptr(gain, torch.bfloat16, "gain"), dev_ptr(pos, torch.int32, "pos"),
         stream_handle(stream, x.device)))
+    return out
+
+
+def linear_workspace_bytes(T: int, F: int, K: int) -> int:
+    return int(lib().er_linear_workspace_bytes(T, F, K))
+
+
+def linear(x: torch.Tensor, w: torch.Tensor, fp32_out: bool = False, out=None, ws=None,
+           stream=None, dev_error=None):
+    """y = x · wᵀ on the tensor cores (er_linear): x BF16 [T, K], w BF16 [F, K];
+    y BF16 (or FP32 with fp32_out) [T, F]."""
+    T, K = x.shape
+    F = w.shape[0]
+    dt = torch.float32 if fp32_out else torch.bfloat16
+    out = torch.empty(T, F, dtype=dt, device=x.device) if out is None else out
+    ws = _ws(linear_workspace_bytes(max(T, 1), F, K), x.device, ws)
+    err = dev_ptr(dev_error, torch.int32, "dev_error") if dev_error is not None else None
+    check("er_linear", lib().er_linear(
+        dev_ptr(x, torch.bfloat16, "x"), T, dev_ptr(w, torch.bfloat16, "w"), F, K,
+        dev_ptr(out, dt, "out"), 1 if fp32_out else 0, out.stride(0), dev_ptr(ws), ws.numel(),
+        err, stream_handle(stream, x.device)))
     return out
 
 

@@ -31,10 +31,11 @@ class CState(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("win_k", "win_v", "bank_k", "bank_v", "pend_k",
                                                "pend_v", "bank_score", "pend_score", "bank_pos",
                                                "pend_pos", "meta", "dev_error")] + [
-        ("s_max", ctypes.c_int32), ("n_layers", ctypes.c_int32)]
+        ("s_max", ctypes.c_int32), ("n_layers", ctypes.c_int32), ("pool", ctypes.c_int32)]
 
 
 ER_FLAG_RMA_OFF = 1  # the RMA switched off (the pages' ablation)
+ER_STATE_POOL = 1    # the pooled anchor layout (a commit that moves no K/V row)
 
 
 class CWeights(ctypes.Structure):
@@ -48,6 +49,10 @@ EXPORTS = {
     "er_state_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32]),
     "er_state_carve": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32,
                                       ctypes.c_int32, ctypes.POINTER(CState)]),
+    "er_state_bytes_ex": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32, ctypes.c_uint32]),
+    "er_state_carve_ex": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32,
+                                         ctypes.c_int32, ctypes.c_uint32,
+                                         ctypes.POINTER(CState)]),
     "er_state_init": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_void_p, ctypes.c_int32,
                                      ctypes.c_void_p]),
     "er_advance": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_void_p, ctypes.c_int32,
@@ -59,6 +64,12 @@ EXPORTS = {
     "er_last_call_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
     "er_qk_norm_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "er_linear_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32,
+                                                     ctypes.c_int32]),
+    "er_linear": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                                 ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                 ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+                                 ctypes.c_void_p]),
     "er_score_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "er_score_split_w1": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "er_wait_selftest": (ctypes.c_int, [ctypes.POINTER(CState), ctypes.c_int32, ctypes.c_void_p]),

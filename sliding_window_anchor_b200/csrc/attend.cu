@@ -66,6 +66,7 @@ struct TileDesc {
   int rows;
   int flags;
   int item;
+  int row;  // the tile's first row in its tensor-mapped array
 };
 
 struct __align__(1024) AttnSmem {
@@ -107,6 +108,11 @@ __device__ int item_ranges(const AttendParams& P, int qi, int g, int br, Range r
     if (nwin > 0) r[n++] = Range{TM_WIN, gi * WIN, nwin};
   } else {
     if (P.rma_off) return 0;  // the RMA switched off: an empty read, o_rma = 0
+    if (P.pool) {
+      // the whole pool of the group; free slots and later records are masked
+      r[n++] = Range{TM_BANK, gi * POOL, POOL};
+      return n;
+    }
     if (bank > 0) r[n++] = Range{TM_BANK, gi * BANK, bank};
     const int np = min(pend + 1, PEND);
     if (np > 0) r[n++] = Range{TM_PEND, gi * PEND, np};
@@ -294,6 +300,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
         S.desc[stage].rows = t.rows;
         S.desc[stage].flags = t.flags;
         S.desc[stage].item = t.item;
+        S.desc[stage].row = t.row;
         if (bytes) mbar_arrive_expect_tx(&S.full[stage], bytes);
         else mbar_arrive(&S.full[stage]);
         if (qbytes)
@@ -355,6 +362,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
   for (int i = 0; i < 8; ++i) keep[i] = 0.f;
 
   int item = 0, qi = 0, g = 0, br = 0;
+  int32_t tq = 0;  // pooled layout: the query's position (records after it are masked)
   while (true) {
     bool end = false;
     uint32_t qb[16][2];  // Qᵀ B fragments for the 16 k-steps (heads >= 4 are zero)
@@ -385,6 +393,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
         int split;
         item = d.item;
         item_coords(P, item, &qi, &g, &br, &split);
+        if (P.pool) {
+          const int seq = P.seq_ids[qi];
+          tq = (seq >= 0 && seq < P.s_max) ? P.meta[seq * 4 + 0] : -1;
+        }
         const uint16_t* q = S.q[stage];
 #pragma unroll
         for (int kk = 0; kk < 16; ++kk) {
@@ -419,11 +431,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
         }
         // s[i]: keys gq (i<2) / gq+8 (i>=2), heads 2cq + (i&1); base-2 logits
         float s[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int key = (i < 2) ? gq : gq + 8;
-          s[i] = (key < nrows) ? (sa[i] + sb[i]) * kLog2eOver16 : -INFINITY;
+        bool vis[2] = {gq < nrows, gq + 8 < nrows};
+        if (P.pool && br) {
+          // pool slots: a free slot, or a record after the query, is not read
+          const int32_t* pp = P.bank_pos + d.row + row0;
+          vis[0] = vis[0] && pp[gq] <= tq;
+          vis[1] = vis[1] && pp[gq + 8] <= tq;
         }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          s[i] = vis[i >> 1] ? (sa[i] + sb[i]) * kLog2eOver16 : -INFINITY;
         // ---- online softmax for this lane's two heads (8 lanes share each pair)
         float alpha[2], pv[4];
 #pragma unroll
@@ -653,12 +670,13 @@ int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* 
   AttendParams P = P0;
   P.splits = attend_splits(P.nq);
   const uint64_t groups = (uint64_t)P.s_max * P.L * NG;
+  const uint64_t bank_rows = P.pool ? (uint64_t)POOL : (uint64_t)BANK;
   bool ok = encode_rows(&P.tmap_k[TM_WIN], P.win_k, groups * WIN) &&
             encode_rows(&P.tmap_v[TM_WIN], P.win_v, groups * WIN) &&
-            encode_rows(&P.tmap_k[TM_BANK], P.bank_k, groups * BANK) &&
-            encode_rows(&P.tmap_v[TM_BANK], P.bank_v, groups * BANK) &&
-            encode_rows(&P.tmap_k[TM_PEND], P.pend_k, groups * PEND) &&
-            encode_rows(&P.tmap_v[TM_PEND], P.pend_v, groups * PEND);
+            encode_rows(&P.tmap_k[TM_BANK], P.bank_k, groups * bank_rows) &&
+            encode_rows(&P.tmap_v[TM_BANK], P.bank_v, groups * bank_rows) &&
+            (P.pool || (encode_rows(&P.tmap_k[TM_PEND], P.pend_k, groups * PEND) &&
+                        encode_rows(&P.tmap_v[TM_PEND], P.pend_v, groups * PEND)));
   if (!ok) return ER_ECUDA;
   {
     // the shared-memory opt-in, once per device (calls may come from several threads)
@@ -745,6 +763,8 @@ int er_swa_rma_attend(const er_state* st, int32_t layer, const int32_t* seq_ids,
   P.part_ml = c.take<float>(attend_ml_floats(B));
   P.sched = c.take<int>(1);
   P.err = st->dev_error;
+  P.pool = st->pool;
+  P.bank_pos = st->bank_pos;
   return launch_attend(P, o_swa, o_rma, nullptr, true, (cudaStream_t)stream);
 }
 

@@ -232,8 +232,9 @@ __device__ __forceinline__ void cluster_sync_all() {
 }
 
 // Step 2 in the select form (no ranked list wanted): flag[i] = 1 for the K
-// kept records (bank i < c, pending BANK + j, j < p).  flag must be cleared
-// and synchronised before; every thread of the block calls it.
+// kept records (bank i < c, pending BANK + j, j < p; in the pooled layout the
+// occupied pool slots i).  flag must be cleared and synchronised before; every
+// thread of the block calls it.
 __device__ void select_kept(const CommitParams& P, size_t gi, int c, int p, int K, uint8_t* flag,
                             int* hist, int* warp_sums, int* sel) {
   const int tid = threadIdx.x;
@@ -242,7 +243,11 @@ __device__ void select_kept(const CommitParams& P, size_t gi, int c, int p, int 
   for (int q = 0; q < 5; ++q) {
     const int i = tid + CT * q;
     uint64_t kv = 0;
-    if (i < BANK) {
+    if (P.pool) {
+      // pool slot i: a record unless free
+      const int32_t pos = P.bank_pos[gi * POOL + i];
+      if (pos != FREE_POS) kv = rec_key(P.bank_score[gi * POOL + i], pos);
+    } else if (i < BANK) {
       if (i < c) kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
     } else if (i - BANK < p) {
       kv = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
@@ -288,6 +293,48 @@ __device__ int plan_moves(int c, int p, const uint8_t* flag, int16_t* evict_list
   }
   __syncthreads();
   return total_win;
+}
+
+// Step 3 in the pooled layout: the evicted records' slots (occupied, not kept,
+// ascending) into evict_list, and the next block's slot list (the 256 lowest
+// slots free after the merge, ascending) into slot_list.  Returns the number
+// evicted; the lists are synchronised on return.
+__device__ int plan_pool(const CommitParams& P, size_t gi, const uint8_t* flag,
+                         int16_t* evict_list, int16_t* slot_list, int* warp_sums) {
+  const int tid = threadIdx.x;
+  int ev[5], fr[5], nev = 0, nfr = 0;
+#pragma unroll
+  for (int q = 0; q < 5; ++q) {
+    const int slot = tid * 5 + q;
+    const bool occ = P.bank_pos[gi * POOL + slot] != FREE_POS;
+    ev[q] = (occ && !flag[slot]) ? 1 : 0;
+    fr[q] = (!occ || ev[q]) ? 1 : 0;
+    nev += ev[q];
+    nfr += fr[q];
+  }
+  int total_ev = 0, total_fr = 0;
+  int er = block_scan_excl(nev, warp_sums, &total_ev);
+  int fi = block_scan_excl(nfr, warp_sums, &total_fr);
+#pragma unroll
+  for (int q = 0; q < 5; ++q) {
+    if (ev[q]) evict_list[er++] = (int16_t)(tid * 5 + q);
+    if (fr[q]) {
+      if (fi < PEND) slot_list[fi] = (int16_t)(tid * 5 + q);
+      ++fi;
+    }
+  }
+  __syncthreads();
+  return total_ev;
+}
+
+// Step 4 in the pooled layout: free the evicted slots and install the slot list.
+__device__ void apply_pool(const CommitParams& P, size_t gi, int n_ev, const int16_t* evict_list,
+                           const int16_t* slot_list) {
+  for (int w = threadIdx.x; w < n_ev; w += CT) {
+    P.bank_pos[gi * POOL + evict_list[w]] = FREE_POS;
+    P.bank_score[gi * POOL + evict_list[w]] = 0.f;
+  }
+  for (int j = threadIdx.x; j < PEND; j += CT) P.slots[gi * PEND + j] = slot_list[j];
 }
 
 // Step 4 for the winners this block's warps own: warp `mover` of `movers`
@@ -405,9 +452,16 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
       for (int e = 0; e < EPT; ++e) {
         const int i = tid * EPT + e;
         uint64_t kv = 0;
-        if (i < c) kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
-        else if (i >= BANK && i < BANK + p)
+        if (P.pool) {
+          if (i < POOL) {
+            const int32_t pos = P.bank_pos[gi * POOL + i];
+            if (pos != FREE_POS) kv = rec_key(P.bank_score[gi * POOL + i], pos);
+          }
+        } else if (i < c) {
+          kv = rec_key(P.bank_score[gi * BANK + i], P.bank_pos[gi * BANK + i]);
+        } else if (i >= BANK && i < BANK + p) {
           kv = rec_key(P.pend_score[gi * PEND + (i - BANK)], P.pend_pos[gi * PEND + (i - BANK)]);
+        }
         key[e] = kv;
         src[e] = (uint32_t)i;
       }
@@ -426,6 +480,14 @@ __global__ void __launch_bounds__(CT, 4) k_commit(CommitParams P) {
       }
     }
     __syncthreads();
+    if (P.pool) {
+      // nothing moves: free the evicted slots, list the next block's slots
+      const int n_ev = plan_pool(P, gi, flag, evict_list, move_dst, warp_sums);
+      cluster_sync_all();
+      if (rank == 0) apply_pool(P, gi, n_ev, evict_list, move_dst);
+      __syncthreads();
+      continue;
+    }
     const int total_win = plan_moves(c, p, flag, evict_list, move_src, move_dst, warp_sums);
     // no CTA of the cluster writes the bank before every CTA has read this merge's keys
     cluster_sync_all();
@@ -462,7 +524,10 @@ __global__ void __launch_bounds__(CT, 4) k_commit_plan(CommitParams P, MovePlan*
     const int c = blk_c[bi];
     const int p = blk_p[bi];
     if (!merge_due(P, seq, c, p)) {
-      if (tid == 0) mp.n = 0;
+      if (tid == 0) {
+        mp.n = 0;
+        mp.commit = 0;
+      }
       continue;
     }
     const size_t gi = grp(seq, l, g, P.L);
@@ -470,19 +535,33 @@ __global__ void __launch_bounds__(CT, 4) k_commit_plan(CommitParams P, MovePlan*
     __syncthreads();
     select_kept(P, gi, c, p, min(BANK, c + p), flag, hist, warp_sums, sel);
     __syncthreads();
+    if (P.pool) {
+      const int n_ev = plan_pool(P, gi, flag, evict_list, move_dst, warp_sums);
+      for (int w = tid; w < n_ev; w += CT) mp.src[w] = evict_list[w];
+      for (int j = tid; j < PEND; j += CT) mp.dst[j] = move_dst[j];
+      if (tid == 0) {
+        mp.n = n_ev;
+        mp.commit = 1;
+      }
+      __syncthreads();
+      continue;
+    }
     const int total_win = plan_moves(c, p, flag, evict_list, move_src, move_dst, warp_sums);
     for (int w = tid; w < total_win; w += CT) {
       mp.src[w] = move_src[w];
       mp.dst[w] = move_dst[w];
     }
-    if (tid == 0) mp.n = total_win;
+    if (tid == 0) {
+      mp.n = total_win;
+      mp.commit = 1;
+    }
     __syncthreads();  // shared arrays are reused by the next sequence
   }
 }
 
 __global__ void __launch_bounds__(CT, 4) k_commit_move(CommitParams P, const MovePlan* plan) {
   __shared__ int16_t move_src[PEND], move_dst[PEND];
-  __shared__ int blk_seq[SPB], blk_n[SPB];
+  __shared__ int blk_seq[SPB], blk_n[SPB], blk_commit[SPB];
   const int lg = blockIdx.y, l = P.layer0 + lg / NG, g = lg % NG;
   const int nlg = P.nlayers * NG;
   const int tid = threadIdx.x;
@@ -492,8 +571,20 @@ __global__ void __launch_bounds__(CT, 4) k_commit_move(CommitParams P, const Mov
   if (tid < nb) {
     blk_seq[tid] = P.seq_fixed >= 0 ? P.seq_fixed : P.seq_ids[b0 + tid];
     blk_n[tid] = plan[(size_t)(b0 + tid) * nlg + lg].n;
+    blk_commit[tid] = plan[(size_t)(b0 + tid) * nlg + lg].commit;
   }
   __syncthreads();
+  if (P.pool) {
+    // nothing moves: the first CTA of each run frees the evicted slots and
+    // installs the slot lists
+    if (r == 0)
+      for (int bi = 0; bi < nb; ++bi) {
+        if (!blk_commit[bi]) continue;
+        const MovePlan& mp = plan[(size_t)(b0 + bi) * nlg + lg];
+        apply_pool(P, grp(blk_seq[bi], l, g, P.L), blk_n[bi], mp.src, mp.dst);
+      }
+    return;
+  }
   for (int bi = 0; bi < nb; ++bi) {
     const int n = blk_n[bi];
     if (n <= 0) continue;  // planned as a merge only for a valid, full sequence
@@ -578,7 +669,11 @@ int launch_commit_move(const CommitParams& P, const MovePlan* plan, cudaStream_t
 struct AppendParams {
   uint16_t *pend_k, *pend_v;
   float* pend_score;
-  int32_t* pend_pos;
+  int32_t* pend_pos;  // pooled layout: the slot lists
+  int pool;
+  uint16_t *bank_k, *bank_v;
+  float* bank_score;
+  int32_t* bank_pos;
   const int32_t* meta;
   const int32_t* seq_ids;
   int n, s_max, L, layer;
@@ -605,6 +700,21 @@ __global__ void __launch_bounds__(256) k_append(AppendParams P) {
   const size_t gi = grp(seq, P.layer, g, P.L);
   const uint4* srcp =
       reinterpret_cast<const uint4*>((w < 4 ? P.k : P.v) + ((size_t)b * NG + g) * D);
+  if (P.pool) {
+    // the record's pool slot comes from the group's slot list
+    const int slot = P.pend_pos[gi * PEND + p];
+    if (slot < 0 || slot >= POOL) {
+      if (lane == 0) set_dev_error(P.err, ER_ECAPACITY);
+      return;
+    }
+    uint4* dstp = reinterpret_cast<uint4*>((w < 4 ? P.bank_k : P.bank_v) + (gi * POOL + slot) * D);
+    dstp[lane] = srcp[lane];
+    if (w < 4 && lane == 0) {
+      P.bank_score[gi * POOL + slot] = P.s[b * NG + g];
+      P.bank_pos[gi * POOL + slot] = P.pos[b];
+    }
+    return;
+  }
   uint4* dstp = reinterpret_cast<uint4*>((w < 4 ? P.pend_k : P.pend_v) + (gi * PEND + p) * D);
   dstp[lane] = srcp[lane];
   if (w < 4 && lane == 0) {
@@ -635,6 +745,7 @@ int er_rma_commit(const er_state* st, int32_t layer, const int32_t* seq_ids, int
   P.nlayers = layer < 0 ? st->n_layers : 1;
   P.p_add = 0; P.only_if_full = 0;
   P.kept = kept; P.err = st->dev_error;
+  P.pool = st->pool; P.slots = st->pend_pos;
   cudaStream_t s = (cudaStream_t)stream;
   int rc = launch_commit(P, s);
   if (rc != ER_OK || layer >= 0) return rc;
@@ -653,6 +764,8 @@ int er_rma_append_pending(const er_state* st, int32_t layer, const int32_t* seq_
   AppendParams P;
   P.pend_k = st->pend_k; P.pend_v = st->pend_v;
   P.pend_score = st->pend_score; P.pend_pos = st->pend_pos;
+  P.pool = st->pool; P.bank_k = st->bank_k; P.bank_v = st->bank_v;
+  P.bank_score = st->bank_score; P.bank_pos = st->bank_pos;
   P.meta = st->meta; P.seq_ids = seq_ids;
   P.n = n; P.s_max = st->s_max; P.L = st->n_layers; P.layer = layer;
   P.k = k; P.v = v; P.s = s; P.pos = pos; P.err = st->dev_error;

@@ -25,6 +25,10 @@ constexpr int QKV = ER_QKV_ROWS;        // 12288
 constexpr int QKVS = ER_QKV_SCORE_ROWS; // 13056: q/k/v rows + the 3 x 256 W1-term rows
 constexpr int OIN = ER_O_IN;            // 4096
 constexpr int ROW_BYTES = D * 2;        // one BF16 K or V row
+// The pooled state layout: bank and pending block share 1280 rows per group; a
+// free pool slot holds this position (above every stream position).
+constexpr int POOL = BANK + PEND;       // 1280
+constexpr int32_t FREE_POS = 0x7FFFFFFF;
 
 // Column offsets of the six projections inside one [QKV] projection row.
 constexpr int OFF_Q_SWA = 0, OFF_K_SWA = 4096, OFF_V_SWA = 5120;

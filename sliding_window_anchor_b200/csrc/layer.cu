@@ -7,6 +7,7 @@
 // filled.  A prefill chunk writes its window rows only after every token read,
 // because the chunk's early tokens still see ring positions its late tokens
 // would overwrite (the prefill read kernel's second launch moves them).
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -14,10 +15,9 @@
 
 namespace er {
 
-int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
-                  cudaStream_t st);
-int gemm_bf16_xwt_f32(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
-                      int ldy, cudaStream_t st);
+size_t proj_workspace_bytes(int T, int F, int K);
+int launch_proj(const uint16_t* X, int T, const uint16_t* W, int F, int K, uint16_t* yb,
+                int ldb, int nbf, float* yf, int ldf, void* ws, int32_t* err, cudaStream_t st);
 int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
                  int n, float* s, void* scratch, int32_t* err, cudaStream_t st);
 size_t score_scratch_bytes(int n);
@@ -42,7 +42,8 @@ namespace er {
 namespace {
 
 struct LayerWs {
-  void* proj;  // BF16 [nq][12288], or FP32 [nq][13056] with the fused weights
+  uint16_t* proj;  // BF16 [nq][12288]: the six projections
+  float* w1_sums;  // FP32 [nq][768]: the three W1-term sums (fused weights)
   unsigned char* score_scratch;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
@@ -51,13 +52,15 @@ struct LayerWs {
   float* pf_out;             // prefill: FP32 branch outputs [2][T][4096]
   uint16_t* o_sum;
   MovePlan* plan;            // the commit's move lists, one per (sequence, group)
+  unsigned char* proj_ws;    // the projections' partial sums and flags (one GEMM at a time)
   size_t bytes;
 };
 
 LayerWs carve_ws(void* base, int nq, bool prefill) {
   Carver c(base);
   LayerWs w;
-  w.proj = c.take<float>((size_t)nq * QKVS);
+  w.proj = c.take<uint16_t>((size_t)nq * QKV);
+  w.w1_sums = c.take<float>((size_t)nq * (QKVS - QKV));
   w.score_scratch = c.take<unsigned char>(score_scratch_bytes(nq));
   w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
@@ -70,6 +73,10 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   w.o_sum = c.take<uint16_t>((size_t)nq * OIN);
   w.plan = reinterpret_cast<MovePlan*>(
       c.take<unsigned char>(commit_plan_bytes(prefill ? 1 : nq, 1)));
+  size_t pw = proj_workspace_bytes(nq, QKVS, HID);
+  pw = std::max(pw, proj_workspace_bytes(nq, QKV, HID));
+  pw = std::max(pw, proj_workspace_bytes(nq, HID, OIN));
+  w.proj_ws = c.take<unsigned char>(pw);
   w.bytes = c.used();
   return w;
 }
@@ -78,29 +85,53 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
 // commit's planning beside the read (it reads only scores and positions, which
 // the read leaves alone) and its row moves beside o_proj (anchor rows vs the
 // read output), and, in a prefill chunk with unprepared weights, the scorer
-// beside the q/k/v projection (both only read x).  A side stream per device
-// takes them between forks and a join on the caller's stream, so the call's
-// work still completes in the caller's stream order (and stays capturable).
+// beside the q/k/v projection (both only read x).  Each caller stream has a
+// side stream and fork/join events of its own, taken between forks and a join
+// on the caller's stream, so a call's work still completes in the caller's
+// stream order (and stays capturable), and calls on different caller streams
+// share nothing: no lock is held across them and no stream waits on another
+// caller's work.
 struct Side {
-  std::mutex mu;
+  std::mutex mu;  // the events are re-recorded by every call that uses this entry
+  cudaStream_t caller = nullptr;
+  bool bound = false;
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr, fork2 = nullptr, join = nullptr;
 };
-Side g_side[64];
+constexpr int kSidesPerDevice = 16;
+struct DeviceSides {
+  bool made = false;
+  Side side[kSidesPerDevice];
+};
+DeviceSides g_sides[64];
+std::mutex g_side_mu;
 
-Side* side_for_current_device() {
+// The side resources of `caller` on the current device.  The device's pool is
+// made by its first layer call (before any capture); later calls only bind a
+// caller stream to a free entry, or, past 16 caller streams, share one.
+Side* side_for(cudaStream_t caller) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  Side& sd = g_side[dev];
-  std::lock_guard<std::mutex> lock(sd.mu);
-  if (!sd.stream) {
-    if (cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&sd.fork2, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) != cudaSuccess)
-      return nullptr;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  DeviceSides& ds = g_sides[dev];
+  if (!ds.made) {
+    for (Side& sd : ds.side)
+      if (cudaStreamCreateWithFlags(&sd.stream, cudaStreamNonBlocking) != cudaSuccess ||
+          cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&sd.fork2, cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) != cudaSuccess)
+        return nullptr;
+    ds.made = true;
   }
-  return &sd;
+  for (Side& sd : ds.side)
+    if (sd.bound && sd.caller == caller) return &sd;
+  for (Side& sd : ds.side)
+    if (!sd.bound) {
+      sd.bound = true;
+      sd.caller = caller;
+      return &sd;
+    }
+  return &ds.side[(reinterpret_cast<uintptr_t>(caller) >> 4) % kSidesPerDevice];
 }
 
 bool weights_ok(const er_layer_weights* w) {
@@ -120,24 +151,30 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   LayerWs W = carve_ws(ws, nq, prefill);
   if (ws_bytes < W.bytes) return ER_ECAPACITY;
   int rc;
-  Side* sd = side_for_current_device();
+  Side* sd = side_for(s);
   if (!sd) return ER_ECUDA;
   // with the RMA off nothing is scored: the plain BF16 projection is cheaper
   const bool fused = w->w_qkv_score != nullptr && !rma_off;
-  uint16_t* proj_bf = static_cast<uint16_t*>(W.proj);
-  float* proj_f = static_cast<float*>(W.proj);
+  uint16_t* proj_bf = W.proj;
+  int32_t* err = st->dev_error;
   if (fused) {
-    // a1 and a3's W1·x in one GEMM, FP32 out
-    if ((rc = gemm_bf16_xwt_f32(x, w->w_qkv_score, proj_f, nq, QKVS, HID, QKVS, s)) != ER_OK)
+    // a1 and a3's W1·x in one GEMM: the projections rounded to BF16, the W1-term
+    // sums kept in FP32
+    if ((rc = launch_proj(x, nq, w->w_qkv_score, QKVS, HID, proj_bf, QKV, QKV, W.w1_sums,
+                          QKVS - QKV, W.proj_ws, err, s)) != ER_OK)
       return rc;
   } else if (rma_off) {
     // a1: all six projections in one GEMM
-    if ((rc = gemm_bf16_xwt(x, w->w_qkv, proj_bf, nq, QKV, HID, s)) != ER_OK) return rc;
+    if ((rc = launch_proj(x, nq, w->w_qkv, QKV, HID, proj_bf, QKV, QKV, nullptr, 0, W.proj_ws,
+                          err, s)) != ER_OK)
+      return rc;
   } else if (!prefill) {
     // a1, then a3 (FP32 scores; the partials stay in the scratch, k_post_proj
     // adds them).  Measured: beside a batch's a1 GEMM, which fills the GPU, the
     // scorer slowed the decode step, so here they run in turn.
-    if ((rc = gemm_bf16_xwt(x, w->w_qkv, proj_bf, nq, QKV, HID, s)) != ER_OK) return rc;
+    if ((rc = launch_proj(x, nq, w->w_qkv, QKV, HID, proj_bf, QKV, QKV, nullptr, 0, W.proj_ws,
+                          err, s)) != ER_OK)
+      return rc;
     if ((rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr, W.score_scratch,
                            st->dev_error, s)) != ER_OK)
       return rc;
@@ -149,7 +186,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
       return ER_ECUDA;
     const int rc_score = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr,
                                       W.score_scratch, st->dev_error, sd->stream);
-    const int rc_proj = gemm_bf16_xwt(x, w->w_qkv, proj_bf, nq, QKV, HID, s);
+    const int rc_proj =
+        launch_proj(x, nq, w->w_qkv, QKV, HID, proj_bf, QKV, QKV, nullptr, 0, W.proj_ws, err, s);
     if (cudaEventRecord(sd->join, sd->stream) != cudaSuccess ||
         cudaStreamWaitEvent(s, sd->join, 0) != cudaSuccess)
       return ER_ECUDA;
@@ -157,8 +195,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   }
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
-  pp.proj = fused ? nullptr : proj_bf;
-  pp.proj_f32 = fused ? proj_f : nullptr;
+  pp.proj = proj_bf;
+  pp.w1_sums = fused ? W.w1_sums : nullptr;
   pp.s_part = fused ? nullptr : score_partials(W.score_scratch, nq);
   pp.w2 = w->w2;
   pp.nq = nq;
@@ -167,6 +205,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   pp.q_swa = W.q_swa; pp.q_rma = W.q_rma;
   pp.win_k = st->win_k; pp.win_v = st->win_v; pp.pend_k = st->pend_k; pp.pend_v = st->pend_v;
   pp.pend_score = st->pend_score; pp.pend_pos = st->pend_pos;
+  pp.pool = st->pool; pp.bank_k = st->bank_k; pp.bank_v = st->bank_v;
+  pp.bank_score = st->bank_score; pp.bank_pos = st->bank_pos;
   pp.meta = st->meta; pp.seq_ids = seq_ids; pp.s_max = st->s_max; pp.L = st->n_layers;
   pp.layer = layer; pp.prefill = prefill ? 1 : 0; pp.seq_fixed = seq_fixed;
   pp.chunk_k = W.chunk_k; pp.chunk_v = W.chunk_v; pp.err = st->dev_error;
@@ -186,6 +226,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   cp.n = prefill ? 1 : nq; cp.s_max = st->s_max; cp.L = st->n_layers;
   cp.layer0 = layer; cp.nlayers = 1; cp.p_add = prefill ? nq : 1; cp.only_if_full = 1;
   cp.kept = nullptr; cp.err = st->dev_error;
+  cp.pool = st->pool; cp.slots = st->pend_pos;
   // the events are re-recorded by every call: hold the side stream from the
   // first fork to the join
   std::unique_lock<std::mutex> lock(sd->mu, std::defer_lock);
@@ -211,12 +252,15 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     ap.s_max = st->s_max; ap.L = st->n_layers; ap.layer = layer;
     ap.q_swa = W.q_swa; ap.q_rma = W.q_rma; ap.nq = nq;
     ap.rma_off = rma_off ? 1 : 0;
+    ap.pool = st->pool; ap.bank_pos = st->bank_pos;
     ap.part_o = W.part_o; ap.part_ml = W.part_ml; ap.sched = W.sched; ap.err = st->dev_error;
     // k_post_proj above zeroed the work counter
     rc_read = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s);
   }
   if (rma_off)
-    return rc_read != ER_OK ? rc_read : gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s);
+    return rc_read != ER_OK ? rc_read
+                            : launch_proj(W.o_sum, nq, w->w_o, HID, OIN, out, HID, HID,
+                                          nullptr, 0, W.proj_ws, err, s);
   // the moves wait for the reads (they overwrite evicted anchor rows); after a
   // failed launch nothing moves, but the side stream still joins
   int rc_move = ER_OK;
@@ -227,7 +271,10 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   if (joined_ok && rc_plan == ER_OK && rc_read == ER_OK)
     rc_move = launch_commit_move(cp, W.plan, sd->stream);
   const int rc_proj =
-      rc_read == ER_OK ? gemm_bf16_xwt(W.o_sum, w->w_o, out, nq, HID, OIN, s) : ER_OK;
+      rc_read == ER_OK
+          ? launch_proj(W.o_sum, nq, w->w_o, HID, OIN, out, HID, HID, nullptr, 0, W.proj_ws, err,
+                        s)
+          : ER_OK;
   // join: the caller's stream waits for the side stream whatever happened above
   joined_ok = cudaEventRecord(sd->join, sd->stream) == cudaSuccess &&
               cudaStreamWaitEvent(s, sd->join, 0) == cudaSuccess && joined_ok;

@@ -165,15 +165,27 @@ __device__ __forceinline__ void post_row(const PostParams& P, int hs, int lane, 
     if (!state_ok) return;
     const int g = (hs < 44) ? hs - 40 : hs - 44;
     const size_t gi = grp(seq, P.layer, g, P.L);
-    dst = ((hs < 44) ? P.pend_k : P.pend_v) + (gi * PEND + p_idx) * D;
+    // the pending record's home: its slot of the pending block, or, in the pooled
+    // layout, the pool slot the group's slot list names for it
+    size_t rec = gi * PEND + p_idx;
+    if (P.pool) {
+      const int slot = P.pend_pos[gi * PEND + p_idx];
+      if (slot < 0 || slot >= POOL) {
+        if (lane == 0) set_dev_error(P.err, ER_ECAPACITY);
+        return;
+      }
+      rec = gi * POOL + slot;
+    }
+    dst = ((hs < 44) ? (P.pool ? P.bank_k : P.pend_k) : (P.pool ? P.bank_v : P.pend_v)) +
+          rec * D;
     if (hs < 44) {
       float sc = 0.f;
-      if (P.proj_f32) {
+      if (P.w1_sums) {
         // the score of group g from the fused GEMM: h_j = hi_j + mid_j + lo_j (the
         // three W1-term sums, smallest first), s_g = sum_j W2[g][j] SiLU(h_j);
         // lane covers j = 8 lane .. 8 lane + 7, then a fixed-order warp sum
         const float4* hrow =
-            reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + QKV) + lane * 2;
+            reinterpret_cast<const float4*>(P.w1_sums + (size_t)qi * (QKVS - QKV)) + lane * 2;
         const float4* w2g = reinterpret_cast<const float4*>(P.w2 + g * 256) + lane * 2;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -191,8 +203,13 @@ __device__ __forceinline__ void post_row(const PostParams& P, int hs, int lane, 
         for (int q = 0; q < 4; ++q) sc += P.s_part[((size_t)q * P.nq + qi) * NG + g];
       }
       if (lane == 0) {
-        P.pend_score[gi * PEND + p_idx] = sc;
-        P.pend_pos[gi * PEND + p_idx] = t;
+        if (P.pool) {
+          P.bank_score[rec] = sc;
+          P.bank_pos[rec] = t;
+        } else {
+          P.pend_score[rec] = sc;
+          P.pend_pos[rec] = t;
+        }
       }
     }
   }
@@ -243,17 +260,7 @@ __global__ void __launch_bounds__(256, 8) k_post_proj(PostParams P) {
   // its latency overlaps warp 0's metadata and rotations.
   grid_dep_wait();
   float v[8];
-  const int col = row_col(hs);
-  if (P.proj_f32) {
-    // FP32 sums of the fused GEMM, rounded to BF16 as a BF16-output GEMM would
-    const float4* src =
-        reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + col) + lane * 2;
-    const float4 a = src[0], b = src[1];
-    v[0] = bf1(f2bf(a.x)); v[1] = bf1(f2bf(a.y)); v[2] = bf1(f2bf(a.z)); v[3] = bf1(f2bf(a.w));
-    v[4] = bf1(f2bf(b.x)); v[5] = bf1(f2bf(b.y)); v[6] = bf1(f2bf(b.z)); v[7] = bf1(f2bf(b.w));
-  } else {
-    load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
-  }
+  load8(P.proj + (size_t)qi * QKV + row_col(hs) + lane * 8, v);
   __syncthreads();
   if (!s_tok[3]) {  // the same for the whole block
     if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);

@@ -9,8 +9,8 @@
 namespace er {
 
 struct PostParams {
-  const uint16_t* proj;      // [nq][12288] BF16 (separate scorer), or
-  const float* proj_f32;     // [nq][13056] FP32: q/k/v sums, then hi/mid/lo W1-term sums
+  const uint16_t* proj;      // [nq][12288] BF16: the six projections
+  const float* w1_sums;      // fused scorer: [nq][768] FP32 hi/mid/lo W1-term sums (or NULL)
   const float* s_part;       // separate scorer: [4 hidden quarters][nq][4] partial scores
   const float* w2;           // fused: W2 [4][256] FP32
   int nq;
@@ -18,7 +18,11 @@ struct PostParams {
   uint16_t *q_swa, *q_rma;  // [nq][16][256] each
   uint16_t *win_k, *win_v, *pend_k, *pend_v;
   float* pend_score;
-  int32_t* pend_pos;
+  int32_t* pend_pos;           // pooled layout: the groups' slot lists
+  int pool;                    // the pooled layout: records go to bank_* at their slot
+  uint16_t *bank_k, *bank_v;
+  float* bank_score;
+  int32_t* bank_pos;
   const int32_t* meta;
   const int32_t* seq_ids;
   int s_max, L, layer;
@@ -52,14 +56,19 @@ struct AttendParams {
   float *o_swa, *o_rma;  // FP32 [nq][16][256] (standalone read), or
   uint16_t* o_sum;       // BF16 [nq][4096] = bf16(o_swa + o_rma) (layer path)
   int rma_off;           // the RMA read sees no records (o_rma = 0)
+  int pool;              // pooled layout: the RMA read takes a group's 1280 pool slots
+  const int32_t* bank_pos;  // pooled layout: per slot the source position (free: FREE_POS)
   int* sched;            // work counter, 0 at launch (the CTAs take units from it)
   int32_t* err;
 };
 
 // One merge's move list (the layer calls' two-launch commit): winner w moves
 // from pending slot src[w] to bank slot dst[w]; n = 0 when nothing commits.
+// In the pooled layout: src[0..n) are the pool slots of the evicted records
+// and dst[0..256) the next block's slot list; commit = 1 when the merge ran.
 struct MovePlan {
   int32_t n;
+  int32_t commit;
   int16_t src[256];
   int16_t dst[256];
 };
@@ -81,6 +90,8 @@ struct CommitParams {
   int per_block;     // sequences per block (set at launch)
   int32_t* kept;     // optional [n][nlayers][4][1024]
   int32_t* err;
+  int pool;          // the pooled layout: bank_* hold 1280 slots, pend_pos the slot lists
+  int32_t* slots;    // pooled layout: [s_max][L][4][256] slot lists (the state's pend_pos)
 };
 
 }  // namespace er

@@ -112,6 +112,8 @@ struct PrefillParams {
   CUtensorMap tmap_v[4];  // the same V rows; box 64 dims x 128 rows
   const int32_t* meta;
   int seq, s_max, L, layer, T;
+  int pool;                 // pooled layout: the RMA read takes the group's 1280 pool slots
+  const int32_t* bank_pos;  // pooled layout: each slot's source position (free: FREE_POS)
   float* out;   // FP32 [2 branches][NSPLIT][T][16][256]: each split's O / l
   float2* ml;   // [2][NSPLIT][T][16]: each split's (running maximum m in log2 units, l)
   int32_t* err;
@@ -120,8 +122,10 @@ struct PrefillParams {
 __device__ __forceinline__ bool warp_all(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 // The key tiles one work item (tokens i0 .. i0+63) reads, in streaming order.
+// In the pooled layout the RMA tiles are the group's 10 pool tiles (kind
+// KIND_BANK over the pool rows), masked by each slot's source position.
 __device__ int build_tiles(PTile* tl, int br, int g, int i0, int T, int t0, int p0, int c,
-                           int gi) {
+                           int gi, int pool) {
   const int i_last = min(T, i0 + PAIR_TOK) - 1;
   int n = 0;
   if (br == 0) {
@@ -142,6 +146,8 @@ __device__ int build_tiles(PTile* tl, int br, int g, int i0, int T, int t0, int 
     }
     for (int ct = 0; ct * PKT <= i_last; ++ct)
       tl[n++] = {KIND_CHUNK, g * T + ct * PKT, ct * PKT, ct * PKT + PKT - 1 <= i0 ? 1 : 0};
+  } else if (pool) {
+    for (int bt = 0; bt < POOL / PKT; ++bt) tl[n++] = {KIND_BANK, gi * POOL + bt * PKT, bt * PKT, 0};
   } else {
     for (int bt = 0; bt * PKT < c; ++bt)
       tl[n++] = {KIND_BANK, gi * BANK + bt * PKT, bt * PKT, bt * PKT + PKT <= c ? 1 : 0};
@@ -192,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
     int nt = 0;
     if (meta_ok) {
       // this pair's contiguous share of the item's tiles (both CTAs build the same list)
-      const int all = build_tiles(S.tiles, br, g, i0, T, t0, p0, c, gi);
+      const int all = build_tiles(S.tiles, br, g, i0, T, t0, p0, c, gi, P.pool);
       const int tb = all * split / NSPLIT, te = all * (split + 1) / NSPLIT;
       for (int j = tb; j < te; ++j) S.tiles[j - tb] = S.tiles[j];
       nt = te - tb;
@@ -335,7 +341,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
 
       const PTile tl = S.tiles[j];
       if (!tl.full) {
-        if (tl.kind == KIND_RING) {
+        if (P.pool && tl.kind == KIND_BANK) {
+          // a free slot, or a record after this query, is not read
+          const int4* pp = reinterpret_cast<const int4*>(P.bank_pos + tl.row0);
+#pragma unroll
+          for (int k4 = 0; k4 < PKT / 4; ++k4) {
+            const int4 q4 = pp[k4];
+            if (q4.x > t) s[4 * k4 + 0] = -INFINITY;
+            if (q4.y > t) s[4 * k4 + 1] = -INFINITY;
+            if (q4.z > t) s[4 * k4 + 2] = -INFINITY;
+            if (q4.w > t) s[4 * k4 + 3] = -INFINITY;
+          }
+        } else if (tl.kind == KIND_RING) {
           const int ub = tl.base - t0;
 #pragma unroll
           for (int k = 0; k < PKT; ++k)
@@ -574,9 +591,13 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   const uint32_t qb[4] = {64, 4, 1, PQ_TOK};
   bool ok = encode_bf16(&P.tmap_q[0], q_swa, 4, qd, qs, qb) &&
             encode_bf16(&P.tmap_q[1], q_rma, 4, qd, qs, qb);
-  const uint16_t* kb[4] = {st->win_k, chunk_k, st->bank_k, st->pend_k};
-  const uint16_t* vb[4] = {st->win_v, chunk_v, st->bank_v, st->pend_v};
-  const uint64_t rows[4] = {rows_win, (uint64_t)NG * T, rows_win, rows_pend};
+  // the pooled layout has no pending arrays: its pool (bank) map stands in for
+  // the unused pending one
+  const uint64_t rows_bank =
+      (uint64_t)st->s_max * st->n_layers * NG * (st->pool ? POOL : BANK);
+  const uint16_t* kb[4] = {st->win_k, chunk_k, st->bank_k, st->pool ? st->bank_k : st->pend_k};
+  const uint16_t* vb[4] = {st->win_v, chunk_v, st->bank_v, st->pool ? st->bank_v : st->pend_v};
+  const uint64_t rows[4] = {rows_win, (uint64_t)NG * T, rows_bank, rows_pend};
   for (int m = 0; m < 4; ++m)
     ok = ok && encode_bf16_2d(&P.tmap_k[m], kb[m], D, rows[m], ROW_BYTES, 64, KH) &&
          encode_bf16_2d(&P.tmap_v[m], vb[m], D, rows[m], ROW_BYTES, 64, PKT);
@@ -587,6 +608,8 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
   P.L = st->n_layers;
   P.layer = layer;
   P.T = T;
+  P.pool = st->pool;
+  P.bank_pos = st->bank_pos;
   P.out = out;
   P.ml = reinterpret_cast<float2*>(out + (size_t)2 * NSPLIT * T * OIN);
   P.err = st->dev_error;

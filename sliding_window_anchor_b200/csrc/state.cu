@@ -40,27 +40,49 @@ struct StateLayout {
   size_t win, bank, pend, bscore, pscore, bpos, ppos, meta, err, total;
 };
 
-bool layout_of(int32_t s_max, int32_t n_layers, StateLayout* L) {
+// pool = 0: the bank (1024 rows per group) and the pending block (256) apart;
+// pool = 1: one pool of 1280 rows per group holding both, with a 256-entry
+// slot list per group in place of the pending arrays (same K/V bytes).
+bool layout_of(int32_t s_max, int32_t n_layers, int pool, StateLayout* L) {
   // row indices of every array stay below 2^31 (TMA coordinates are 32-bit): 4096
   // sequences are 288 GiB of state, more than one GPU holds
   if (s_max < 1 || s_max > 4096 || n_layers < 1 || n_layers > ER_MAX_LAYERS) return false;
   Carver c(nullptr);
   size_t g = (size_t)s_max * n_layers * NG;
+  const size_t bank_rows = pool ? (size_t)POOL : (size_t)BANK;
   L->win = (size_t)c.take<uint16_t>(g * WIN * D);
-  size_t win_v = (size_t)c.take<uint16_t>(g * WIN * D);
-  L->bank = (size_t)c.take<uint16_t>(g * BANK * D);
-  size_t bank_v = (size_t)c.take<uint16_t>(g * BANK * D);
-  L->pend = (size_t)c.take<uint16_t>(g * PEND * D);
-  size_t pend_v = (size_t)c.take<uint16_t>(g * PEND * D);
-  (void)win_v; (void)bank_v; (void)pend_v;
-  L->bscore = (size_t)c.take<float>(g * BANK);
-  L->pscore = (size_t)c.take<float>(g * PEND);
-  L->bpos = (size_t)c.take<int32_t>(g * BANK);
-  L->ppos = (size_t)c.take<int32_t>(g * PEND);
+  c.take<uint16_t>(g * WIN * D);  // win_v
+  L->bank = (size_t)c.take<uint16_t>(g * bank_rows * D);
+  c.take<uint16_t>(g * bank_rows * D);  // bank_v
+  L->pend = pool ? 0 : (size_t)c.take<uint16_t>(g * PEND * D);
+  if (!pool) c.take<uint16_t>(g * PEND * D);  // pend_v
+  L->bscore = (size_t)c.take<float>(g * bank_rows);
+  L->pscore = pool ? 0 : (size_t)c.take<float>(g * PEND);
+  L->bpos = (size_t)c.take<int32_t>(g * bank_rows);
+  L->ppos = (size_t)c.take<int32_t>(g * PEND);  // pool: the slot list
   L->meta = (size_t)c.take<int32_t>((size_t)s_max * 4);
   L->err = (size_t)c.take<int32_t>(64);
   L->total = c.used();
   return true;
+}
+
+// The pooled layout's stream start: every pool slot free (position FREE_POS),
+// the first block's records going to slots 0..255.
+// A read weighs a skipped record by exactly 0, which a NaN in its V row would
+// still spoil, so the V rows of the pool start at zero too.
+__global__ void k_pool_init(float* score, int32_t* pos, int32_t* slots, uint16_t* bank_v,
+                            const int32_t* seq_ids, int n, int s_max, int L) {
+  const int b = blockIdx.x, lg = blockIdx.y;
+  const int seq = seq_ids[b];
+  if (seq < 0 || seq >= s_max) return;  // recorded by k_state_init
+  const size_t gi = (size_t)seq * L * NG + lg;
+  for (int i = threadIdx.x; i < POOL; i += blockDim.x) {
+    score[gi * POOL + i] = 0.f;
+    pos[gi * POOL + i] = FREE_POS;
+  }
+  for (int j = threadIdx.x; j < PEND; j += blockDim.x) slots[gi * PEND + j] = j;
+  uint4* v = reinterpret_cast<uint4*>(bank_v + gi * POOL * D);
+  for (int i = threadIdx.x; i < POOL * D / 8; i += blockDim.x) v[i] = make_uint4(0, 0, 0, 0);
 }
 
 __global__ void k_state_init(int32_t* meta, const int32_t* seq_ids, int n, int s_max,
@@ -223,40 +245,60 @@ int er_last_call_error(int32_t* code, er_stream_t stream) {
   return read_and_clear(word, code, (cudaStream_t)stream);
 }
 
-size_t er_state_bytes(int32_t s_max, int32_t n_layers) {
+size_t er_state_bytes_ex(int32_t s_max, int32_t n_layers, uint32_t flags) {
   StateLayout L;
-  return layout_of(s_max, n_layers, &L) ? L.total : 0;
+  if (flags & ~ER_STATE_POOL) return 0;
+  return layout_of(s_max, n_layers, (flags & ER_STATE_POOL) ? 1 : 0, &L) ? L.total : 0;
 }
 
-int er_state_carve(void* base, size_t bytes, int32_t s_max, int32_t n_layers, er_state* out) {
+size_t er_state_bytes(int32_t s_max, int32_t n_layers) {
+  return er_state_bytes_ex(s_max, n_layers, 0u);
+}
+
+int er_state_carve_ex(void* base, size_t bytes, int32_t s_max, int32_t n_layers, uint32_t flags,
+                      er_state* out) {
   StateLayout L;
-  if (!base || !out || !layout_of(s_max, n_layers, &L)) return ER_EINVAL;
+  const int pool = (flags & ER_STATE_POOL) ? 1 : 0;
+  if ((flags & ~ER_STATE_POOL) || !base || !out || !layout_of(s_max, n_layers, pool, &L))
+    return ER_EINVAL;
   if (((uintptr_t)base & 255u) != 0 || bytes < L.total) return ER_EINVAL;
   char* b = (char*)base;
   size_t g = (size_t)s_max * n_layers * NG;
+  const size_t bank_rows = pool ? (size_t)POOL : (size_t)BANK;
   out->win_k = (er_bf16*)(b + L.win);
   out->win_v = out->win_k + g * WIN * D;
   out->bank_k = (er_bf16*)(b + L.bank);
-  out->bank_v = out->bank_k + g * BANK * D;
-  out->pend_k = (er_bf16*)(b + L.pend);
-  out->pend_v = out->pend_k + g * PEND * D;
+  out->bank_v = out->bank_k + g * bank_rows * D;
+  out->pend_k = pool ? nullptr : (er_bf16*)(b + L.pend);
+  out->pend_v = pool ? nullptr : out->pend_k + g * PEND * D;
   out->bank_score = (float*)(b + L.bscore);
-  out->pend_score = (float*)(b + L.pscore);
+  out->pend_score = pool ? nullptr : (float*)(b + L.pscore);
   out->bank_pos = (int32_t*)(b + L.bpos);
   out->pend_pos = (int32_t*)(b + L.ppos);
   out->meta = (int32_t*)(b + L.meta);
   out->dev_error = (int32_t*)(b + L.err);
   out->s_max = s_max;
   out->n_layers = n_layers;
+  out->pool = pool;
   return ER_OK;
+}
+
+int er_state_carve(void* base, size_t bytes, int32_t s_max, int32_t n_layers, er_state* out) {
+  return er_state_carve_ex(base, bytes, s_max, n_layers, 0u, out);
 }
 
 int er_state_init(const er_state* st, const int32_t* seq_ids, int32_t n, er_stream_t stream) {
   if (!st || !st->meta || (n > 0 && !seq_ids) || n < 0) return ER_EINVAL;
   if (n == 0) return ER_OK;
-  k_state_init<<<(n + 127) / 128, 128, 0, (cudaStream_t)stream>>>(st->meta, seq_ids, n,
-                                                                   st->s_max, st->dev_error);
+  cudaStream_t s = (cudaStream_t)stream;
+  k_state_init<<<(n + 127) / 128, 128, 0, s>>>(st->meta, seq_ids, n, st->s_max, st->dev_error);
   count_launches(1);
+  if (st->pool) {
+    k_pool_init<<<dim3(n, st->n_layers * NG), 256, 0, s>>>(st->bank_score, st->bank_pos,
+                                                          st->pend_pos, st->bank_v, seq_ids, n,
+                                                          st->s_max, st->n_layers);
+    count_launches(1);
+  }
   return launch_status();
 }
 

@@ -144,6 +144,18 @@ def test_host_validation_rejects_before_enqueue(L):
     assert L.er_rma_score_ex(ctypes.byref(w), nul, 0, nul, nul, 0, nul, nul) == 0
     assert L.er_last_call_error(None, nul) == -1
     assert L.er_launch_count() == before
+    # the projection GEMM: sizes, alignment and workspace are checked before any launch
+    before = L.er_launch_count()
+    assert L.er_linear_workspace_bytes(1, 300, 2560) == 0
+    assert L.er_linear_workspace_bytes(512, 13056, 2560) > 0
+    assert L.er_linear(ok, 4, ok, 300, 2560, ok, 0, 300, ok, 1 << 30, nul, nul) == -1
+    assert L.er_linear(ok, 4, ok, 2560, 100, ok, 0, 2560, ok, 1 << 30, nul, nul) == -1
+    assert L.er_linear(ok, 4, ok, 2560, 2560, ok, 2, 2560, ok, 1 << 30, nul, nul) == -1
+    assert L.er_linear(ok, 4, ok, 2560, 2560, ok, 0, 2000, ok, 1 << 30, nul, nul) == -1
+    assert L.er_linear(fake, 4, ok, 2560, 2560, ok, 0, 2560, ok, 1 << 30, nul, nul) == -1
+    assert L.er_linear(ok, 4, ok, 2560, 2560, ok, 0, 2560, ok, 16, nul, nul) == -2
+    assert L.er_linear(nul, 0, nul, 2560, 2560, nul, 0, 2560, nul, 0, nul, nul) == 0
+    assert L.er_launch_count() == before
     # the fused q/k/v + W1-term weights: NULL, unaligned or overlapping buffers are refused
     base = 1 << 40
     qkv_bytes = 12288 * 2560 * 2

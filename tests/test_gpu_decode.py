@@ -424,3 +424,58 @@ def test_rma_off_prefill_matches_oracle_and_decode(sab):
     for n in RMA_ARRAYS:
         assert torch.equal(getattr(st, n), before[n]), n
     assert st.meta[0].tolist() == [t0 + T, 60, 1024, 0]
+
+
+def test_two_caller_streams_run_layer_calls_side_by_side(sab):
+    """Two host threads, each with its own stream, state and workspace, run decode
+    steps (with commits) at the same time: each gets the bits of the same steps run
+    alone.  The library gives each caller stream its own side stream and events,
+    so neither caller's calls wait on the other's."""
+    import threading
+    seed, B, steps, t0 = 88, 8, 6, 4096
+    gw, gdict = H.gpu_weights(seed, 0)
+    fills = [250, 251, 252, 253, 254, 255, 3, 100]  # commits inside the six steps
+    states = []
+    for k in range(2):
+        st = sab.State(B, 1)
+        H.seed_gpu_state(st, 1, t0, fills, seed + k, [gdict])
+        states.append(st)
+    snaps = [st.blob.clone() for st in states]
+    xs = [[wl.make_x(seed + k, 0, s, range(B), device="cuda") for s in range(steps)]
+          for k in range(2)]
+    ids = torch.arange(B, dtype=torch.int32, device="cuda")
+
+    def run(k, stream, outs, start=None):
+        if start is not None:
+            start.wait()
+        ws = torch.empty(sab.decode_workspace_bytes(B), dtype=torch.uint8, device="cuda")
+        with torch.cuda.stream(stream):
+            for s in range(steps):
+                outs.append(sab.swa_rma_decode(states[k], gw, 0, ids, xs[k][s], ws=ws,
+                                               stream=stream))
+                sab.advance(states[k], ids, stream=stream)
+        stream.synchronize()
+
+    alone = [[], []]
+    for k in range(2):
+        run(k, torch.cuda.current_stream(), alone[k])
+    ref_blobs = [st.blob.clone() for st in states]
+    for k in range(2):
+        states[k].blob.copy_(snaps[k])
+    torch.cuda.synchronize()
+    together = [[], []]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    start = threading.Event()
+    threads = [threading.Thread(target=run, args=(k, streams[k], together[k], start))
+               for k in range(2)]
+    for t in threads:
+        t.start()
+    start.set()
+    for t in threads:
+        t.join()
+    torch.cuda.synchronize()
+    for k in range(2):
+        assert sab.last_device_error(states[k]) == 0
+        for s in range(steps):
+            assert torch.equal(together[k][s], alone[k][s]), (k, s)
+        assert torch.equal(states[k].blob, ref_blobs[k]), k
