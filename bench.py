@@ -47,6 +47,8 @@ def parse():
                     help="skip the decode pass with the RMA switched off (the ablation)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph pass (one captured graph per decode step)")
+    ap.add_argument("--no-pool", action="store_true",
+                    help="skip the pooled-layout A/B (decode steps and commits)")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the B=1 (one layer) and B=64 (8 layers) decode configurations")
     ap.add_argument("--prefill-chunks", type=int, default=512,
@@ -74,16 +76,25 @@ def peaks():
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clocks and throttle reasons sampled during the timed region: NVML read
+    every 10 ms from a host thread (read-only queries), else nvidia-smi every
+    200 ms.  Samples outside the timed windows (begin/end) are ignored."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, device=None):
         self.idx = gpu_index
+        self.device = device
         self.proc = None
-        self.lines = []    # (host time, line)
-        self.windows = []  # [t0, t1] spans of timed work; samples outside are ignored
+        self.nvml = None
+        self.samples = []  # (host time, sm MHz, max sm MHz, set of reasons)
+        self.lines = []    # (host time, nvidia-smi line)
+        self.windows = []  # [t0, t1] spans of timed work
+        self.stop_flag = False
 
     def begin(self):
         self.windows.append([time.monotonic(), None])
@@ -91,7 +102,25 @@ class ClockSampler:
     def end(self):
         self.windows[-1][1] = time.monotonic()
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(
+                uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+
     def start(self):
+        try:
+            self.nvml = self._nvml_handle()
+            self.th = threading.Thread(target=self._poll_nvml, daemon=True)
+            self.th.start()
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
@@ -102,13 +131,43 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def _poll_nvml(self):
+        pynvml, h = self.nvml
+        smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop_flag:
+            t = time.monotonic()
+            if self.windows and self.windows[-1][1] is None:
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    bits = pynvml.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+                    rs = {n for n, b in self.REASON_BITS.items() if bits & b}
+                    self.samples.append((t, float(sm), float(smax), rs))
+                except Exception:
+                    pass
+            time.sleep(0.01)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append((time.monotonic(), line.strip()))
 
+    def _timed(self, t):
+        return any(a <= t <= (b if b is not None else float("inf")) for a, b in self.windows)
+
     def stop(self):
+        if self.nvml:
+            self.stop_flag = True
+            self.th.join(timeout=5)
+            sm = [x[1] for x in self.samples if self._timed(x[0])]
+            smax = [x[2] for x in self.samples if self._timed(x[0])]
+            reasons = set()
+            for x in self.samples:
+                if self._timed(x[0]):
+                    reasons |= x[3]
+            return {"sm_mhz": statistics.median(sm) if sm else None,
+                    "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                    "samples": len(sm), "source": "NVML, every 10 ms in the timed loops"}
         if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock query unavailable"]}
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -116,12 +175,8 @@ class ClockSampler:
             self.proc.kill()
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        def timed(t):
-            return not self.windows or any(
-                a <= t <= (b if b is not None else float("inf")) for a, b in self.windows)
-
         for t, ln in self.lines:
-            if not timed(t):
+            if self.windows and not self._timed(t):
                 continue
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
@@ -136,7 +191,7 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvidia-smi, every 200 ms"}
 
 
 # ------------------------------------------------------------ multi-rank
@@ -182,7 +237,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    seed = wl.seed_of(3)
+    seed = wl.seed_of(wl.DECODE_B512)
     weights = [sab.LayerWeights.from_dict(wl.make_weights(seed, l, device=dev))
                for l in range(LAYERS)]
     wdicts = [w.t for w in weights]
@@ -216,7 +271,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     sab.profile_read(reset=True)
     sab.profile_enable(True)
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(local_rank, dev)
     clocks.start()
     n0 = sab.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -389,6 +444,9 @@ def run_ours(args, rank, world, local_rank):
                    "note": "ER_FLAG_RMA_OFF, eager: o_rma = 0, no score, append or commit"}
 
     ms = reduce_max(ms, dev)
+    pool_ab = None
+    if not args.no_pool and rank == 0:
+        pool_ab = pooled_ab(st, weights, ids, xs, dev)  # before the commit workload replaces the state
     cm = None
     if not args.no_commit_bench and rank == 0:
         # the commit microbench reuses the decode state's memory (B=512 x 8 layers)
@@ -398,11 +456,11 @@ def run_ours(args, rank, world, local_rank):
         pf = prefill_bench(dev, args.prefill_chunks)
     cfgs = None
     if not args.no_configs and rank == 0:
-        cfgs = {r["workload"]: r for r in (decode_config_bench(dev, 0),
-                                           decode_config_bench(dev, 2))}
+        cfgs = {r["workload"]: r for r in (decode_config_bench(dev, wl.DECODE_B1),
+                                           decode_config_bench(dev, wl.DECODE_B64))}
     return dict(ms=ms, launches=launches, clocks=clk, attend_ms=attend_ms, attend_n=attend_n,
                 fills=fills, commits=commits, e2e=e2e, commit_microbench=cm, prefill=pf,
-                graph=graph, rma_off=rma_off, configs=cfgs)
+                graph=graph, rma_off=rma_off, configs=cfgs, pool=pool_ab)
 
 
 # ------------------------------------------------------- commit microbench
@@ -419,7 +477,7 @@ def commit_microbench(st, dev, reps=3):
     import torch
     import sliding_window_anchor_b200 as sab
     from synth import workloads as wl
-    seed = wl.seed_of(1)
+    seed = wl.seed_of(wl.COMMIT)
     ids = torch.arange(st.s_max, dtype=torch.int32, device=dev)
     merges = st.s_max * st.n_layers * 4
     times, moved = [], []
@@ -450,6 +508,92 @@ def commit_microbench(st, dev, reps=3):
                                   "workload (i.i.d. scores, ~5% ties)"}
 
 
+def pooled_ab(st, weights, ids, xs, dev, steps=32, reps=3):
+    """The pooled anchor layout (ER_STATE_POOL, a commit that moves no K/V row)
+    against the plain one, measured on the same work: (1) decode steps of the
+    decode workload, each layout starting from the same records, replayed from
+    CUDA graphs; (2) the commit microbench, each repetition's workload copied
+    into the pooled layout (identical records and keys)."""
+    import torch
+    import sliding_window_anchor_b200 as sab
+    from synth import workloads as wl
+    B, L = st.s_max, st.n_layers
+    n_x = len(xs)
+    ws = torch.empty(sab.decode_workspace_bytes(B), dtype=torch.uint8, device=dev)
+    outs = [torch.empty(B, 2560, dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    stream = torch.cuda.current_stream(dev)
+    pool = sab.State(B, L, device=dev, pool=True)
+    pool.pool_from_plain(st)
+    res = {}
+    for name, state in (("pooled", pool), ("plain", st)):
+        def step(s, state=state):
+            for l in range(L):
+                sab.swa_rma_decode(state, weights[l], l, ids, xs[s % n_x][l], out=outs[l], ws=ws)
+            sab.advance(state, ids)
+        step(0)  # the stream's side resources exist before capture
+        torch.cuda.synchronize(dev)
+        stream_g = torch.cuda.Stream(dev)
+        graphs = []
+        for s in range(n_x):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream_g):
+                step(s)
+            graphs.append(g)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for s in range(steps):
+            graphs[(s + 1) % n_x].replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        del graphs
+        if sab.last_device_error(state) != 0:
+            raise RuntimeError(f"device error in the {name} decode pass")
+        ms = e0.elapsed_time(e1) / steps
+        res[name] = {"ms_per_step": ms, "tok_per_s": B / (ms / 1e3)}
+    # the commit microbench in both layouts on the same workloads
+    seed = wl.seed_of(wl.COMMIT)
+    merges = B * L * 4
+    t_plain, t_pool, moved = [], [], []
+    snap_keys = None
+    for rep in range(reps + 1):
+        wl.seed_commit_workload(st.arrays(), range(B), L, T0, seed, rep, dev)
+        pool.pool_from_plain(st)
+        torch.cuda.synchronize(dev)
+        for name, state, acc in (("pooled", pool, t_pool), ("plain", st, t_plain)):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            sab.rma_commit(state, -1, ids)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if sab.last_device_error(state) != 0:
+                raise RuntimeError(f"device error in the {name} commit")
+            if rep > 0:
+                acc.append(e0.elapsed_time(e1))
+        if rep > 0:
+            moved.append(int((st.bank_pos >= T0).sum()))
+    med = lambda v: sorted(v)[len(v) // 2]
+    hbm, kind = peaks()
+    m = med(moved)
+    # bytes a pooled merge must touch: the 1280 keys read, the evicted slots'
+    # position and score written, the 256-entry slot list written (no K/V row)
+    pool_alg = merges * (1280 * 8 + (m / merges) * 8 + 256 * 4)
+    plain_alg = merges * 1280 * 8 + m * (2 * 1024 + 16)
+    res["commit"] = {
+        "workload": f"commit_b{B}_l{L}", "merges": merges, "moved_records_plain": m,
+        "plain_ms": med(t_plain), "pooled_ms": med(t_pool),
+        "plain_merges_per_s": merges / (med(t_plain) / 1e3),
+        "pooled_merges_per_s": merges / (med(t_pool) / 1e3),
+        "plain_alg_bytes": plain_alg, "pooled_alg_bytes": pool_alg,
+        "pooled_frac": pool_alg / (med(t_pool) / 1e3) / 1e9 / hbm, "peak_kind": kind}
+    res["note"] = ("decode: both layouts from the same records, the same inputs, graph-replayed; "
+                   "the pooled read takes all 1280 pool slots per group (free and later ones "
+                   "masked) where the plain one takes the bank and the filled pending slots")
+    del pool
+    torch.cuda.empty_cache()
+    return res
+
+
 def prefill_attention_flops(t0: int, T: int, c: int, p0: int) -> int:
     """Algorithmic FLOPs of one chunk's two reads (QKᵀ and PV, 2 FLOP per
     multiply-add, 16 heads, head dim 256): query i at position t0+i reads
@@ -468,7 +612,7 @@ def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2,
     import torch
     import sliding_window_anchor_b200 as sab
     from synth import workloads as wl
-    seed = wl.seed_of(4)
+    seed = wl.seed_of(wl.PREFILL)
     T = 256
     weights = [sab.LayerWeights.from_dict(wl.make_weights(seed, l, device=dev))
                for l in range(layers)]
@@ -491,8 +635,6 @@ def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2,
     torch.cuda.synchronize(dev)
     sab.state_init(st, seq0)
     torch.cuda.synchronize(dev)
-    sab.profile_read(reset=True)
-    sab.profile_enable(True)
     n0 = sab.launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h0 = time.perf_counter()
@@ -501,12 +643,22 @@ def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2,
     e1.record(stream)
     host_ms = (time.perf_counter() - h0) * 1e3  # submission time on the host
     torch.cuda.synchronize(dev)
-    sab.profile_enable(False)
-    attn_ms, attn_n = sab.profile_read(reset=True)
     launches = sab.launch_count() - n0
     if sab.last_device_error(st) != 0:
         raise RuntimeError("device error in the prefill bench")
     ms = e0.elapsed_time(e1)
+    # the prefill reads' own time: a second eager pass with events around each
+    # read launch (the events cost host time, so this pass is not the one timed)
+    sab.state_init(st, seq0)
+    torch.cuda.synchronize(dev)
+    sab.profile_read(reset=True)
+    sab.profile_enable(True)
+    run(0, chunks)
+    torch.cuda.synchronize(dev)
+    sab.profile_enable(False)
+    attn_ms, attn_n = sab.profile_read(reset=True)
+    if sab.last_device_error(st) != 0:
+        raise RuntimeError("device error in the prefill bench")
     graph_ms = None
     if graph:
         # the same stream replayed from CUDA graphs, one per chunk (all layers + advance)
@@ -553,8 +705,8 @@ def prefill_bench(dev, chunks: int, layers: int = LAYERS, warm_chunks: int = 2,
 WEIGHT_BYTES_PER_LAYER = 13056 * 2560 * 2 + 2560 * 4096 * 2 + 4 * 256 * 4 + 4 * 256 * 2
 
 
-def decode_config_bench(dev, cfg_index: int, n_x: int = 16, warmup: int = 3):
-    """One spec decode configuration end to end on the device: its state
+def decode_config_bench(dev, workload: str, n_x: int = 16, warmup: int = 3):
+    """One named decode workload end to end on the device: its state
     seeded as the tests seed it, then all of its steps (a1-a7 per layer, device-
     gated commits, the advance) replayed from CUDA graphs (one per distinct input
     buffer, inputs resident).  Reports tok/s, ms/step and the fraction of the byte
@@ -563,7 +715,7 @@ def decode_config_bench(dev, cfg_index: int, n_x: int = 16, warmup: int = 3):
     import torch
     import sliding_window_anchor_b200 as sab
     from synth import workloads as wl
-    cfg, seed = wl.CONFIGS[cfg_index], wl.seed_of(cfg_index)
+    cfg, seed = wl.CONFIGS[workload], wl.seed_of(workload)
     Bc, L, steps, t0 = cfg["B"], cfg["n_layers"], cfg["steps"], cfg["t0"]
     weights = [sab.LayerWeights.from_dict(wl.make_weights(seed, l, device=dev))
                for l in range(L)]
@@ -623,7 +775,7 @@ def decode_config_bench(dev, cfg_index: int, n_x: int = 16, warmup: int = 3):
     torch.cuda.synchronize(dev)
     del graphs
     if sab.last_device_error(st) != 0:
-        raise RuntimeError(f"device error in the config {cfg_index} bench")
+        raise RuntimeError(f"device error in the {workload} bench")
     ms = g0.elapsed_time(g1)
     hbm, kind = peaks()
     state_bytes = algorithmic_read_bytes(fills, 0, steps) * L
@@ -656,7 +808,7 @@ def batch_sweep(dev, batches=SWEEP_BATCHES, steps: int = 32, warmup: int = 4):
     import torch
     import sliding_window_anchor_b200 as sab
     from synth import workloads as wl
-    seed = wl.seed_of(3)
+    seed = wl.seed_of(wl.DECODE_B512)
     bmax = max(batches)
     w = sab.LayerWeights.from_dict(wl.make_weights(seed, 0, device=dev))
     st = sab.State(bmax, 1, device=dev)
@@ -797,7 +949,7 @@ def single_kernel(args):
                                                     warm_chunks=1)}
     elif args.kernel == "layer":
         # the decode workload's state for one layer (t0 = 32768, pending U{0..255})
-        seed = wl.seed_of(3)
+        seed = wl.seed_of(wl.DECODE_B512)
         w = sab.LayerWeights.from_dict(wl.make_weights(seed, 0, device=dev))
         st = sab.State(B, 1, device=dev)
         nr = lambda x, g, p: sab.qk_norm_rope(x.contiguous(), g, p.to(torch.int32).contiguous())
@@ -838,7 +990,7 @@ def oracle_tokens_per_s(budget_s=12.0, max_threads=8):
     import oracle
     from synth import workloads as wl
 
-    seed = wl.seed_of(3)
+    seed = wl.seed_of(wl.DECODE_B512)
     threads = max(1, min(max_threads, os.cpu_count() or 1))
     ows = []
     for l in range(LAYERS):
@@ -877,7 +1029,7 @@ def oracle_merges_per_s(budget_s=4.0):
     freshly seeded repetition (as the GPU microbench seeds them)."""
     import oracle
     from synth import workloads as wl
-    seed = wl.seed_of(1)
+    seed = wl.seed_of(wl.COMMIT)
     ost = oracle.OracleState(1, LAYERS)
     arrays = {n: getattr(ost, n) for n in oracle.OracleState.ARRAYS}
     merges, spent, rep = 0, 0.0, 0
@@ -1010,6 +1162,7 @@ def main():
         "prefill": r["prefill"],
         "rma_off": r["rma_off"],
         "configs": r["configs"],
+        "pooled_layout": r["pool"],
         "eager": {"value": whole_job_tokens_per_s(world, B, args.steps, r["ms"]),
                   "ms_per_step": r["ms"] / args.steps, "gpu_launches": r["launches"],
                   "note": "the same steps launched call by call through the binding; "

@@ -28,8 +28,9 @@
  *  - Pointers named in a signature are DEVICE pointers unless marked (host).
  *    The caller allocates and frees all memory (state, weights, inputs,
  *    outputs, workspace); the library never allocates or frees device memory
- *    itself (er_rma_score_noalloc's scratch and the library's error word are
- *    fixed device arrays) and never synchronises the stream,
+ *    itself (cuBLAS keeps its own handle memory; er_rma_score_noalloc's scratch
+ *    and the library's error word are fixed device arrays) and never
+ *    synchronises the stream,
  *    except er_last_device_error and er_last_call_error, which read one word
  *    back.
  *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default).  A
@@ -39,9 +40,9 @@
  *    from and joined back to `stream` inside the call, so everything still
  *    completes in `stream` order and the call can be captured in a CUDA
  *    graph; calls on different caller streams do not wait on each other.
- *    The first layer call on a device creates that device's side streams and
- *    events, and the first call of each kind its kernel attributes: make one
- *    such call on the device before capturing on it.
+ *    The first layer call on a device creates that device's side streams,
+ *    events and cuBLAS handle, and the first call of each kind its kernel
+ *    attributes: make one such call on the device before capturing on it.
  *  - Those per-device resources, and the device addresses of the library's
  *    fixed device arrays, are made once per device and process and are not
  *    made again after cudaDeviceReset: do not call the library on a device
@@ -161,7 +162,7 @@ typedef struct er_state {
  *                             When set, the layer calls take a1 and the W1·x
  *                             product of a3 from ONE GEMM over it (FP32 output;
  *                             the projections are then rounded to BF16, the same
- *                             values a BF16-output er_linear gives) and apply SiLU and
+ *                             values a BF16-output GEMM gives) and apply SiLU and
  *                             W2 in the norm/RoPE kernel, so no separate scorer
  *                             launch runs (calls with ER_FLAG_RMA_OFF score
  *                             nothing and project from w_qkv with BF16 output).
@@ -259,12 +260,17 @@ int er_wait_selftest(const er_state* st, int32_t arrive, er_stream_t stream);
 int er_qk_norm_rope(const er_bf16* x, er_bf16* y, int64_t n_rows, const er_bf16* gain,
                     const int32_t* pos, er_stream_t stream);
 
-/* a1 / a6 — the layer's dense projections on their own [F-arch]: y = x · wᵀ
- * with x BF16 [T][K] and w BF16 [F][K] (row-major, the nn.Linear layout), FP32
- * accumulation on the tensor cores; y is BF16 (y_fp32 = 0, round to nearest
- * even) or FP32 (y_fp32 = 1), [T][ldy] with ldy >= F.  The layer calls use
- * it for x·W_qkvᵀ (F = 12288, or 13056 with the scorer's W1 terms, K = 2560)
- * and for the shared o_proj (F = 2560, K = 4096).  F a multiple of 256, K of
+/* a1 / a6 — a projection of the layer's shapes on its own [F-arch]: y = x · wᵀ
+ * with x BF16 [T][K] and w BF16 [F][K] (row-major, the nn.Linear layout), BF16
+ * products accumulated in FP32 on the tensor cores by this library's own
+ * kernels: up to 32 tokens a weight-streaming kernel (mma.m16n8k16 tiles, the
+ * one the layer calls use for decode batches of up to 8 sequences), above
+ * that a tcgen05 GEMM (CTA pairs, work split over all SMs along K); y is BF16
+ * (y_fp32 = 0, round to nearest even) or FP32 (y_fp32 = 1), [T][ldy] with
+ * ldy >= F.  The shapes are those of x·W_qkvᵀ (F = 12288, or 13056 with the
+ * scorer's W1 terms, K = 2560) and of the shared o_proj (F = 2560, K = 4096).
+ * (For more than 8 tokens the layer calls take these products from cuBLAS,
+ * measured faster at their token counts.)  F a multiple of 256, K of
  * 64, T >= 0; x, w, y 16-byte aligned; ws 256-byte aligned, at least
  * er_linear_workspace_bytes(T, F, K) (0 for bad sizes), reusable by calls
  * ordered on one stream.  The summation order is fixed for given (T, F, K):

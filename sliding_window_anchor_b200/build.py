@@ -36,7 +36,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     """Compile every csrc/*.cu into libedgerock.so; returns the library path."""
     with _lock:
         if force or _stale():
-            cmd = ["nvcc", *NVCC_FLAGS, *extra, "-o", LIB, *sources()]
+            cmd = ["nvcc", *NVCC_FLAGS, *extra, "-o", LIB, *sources(), "-lcublas"]
             if verbose:
                 print(" ".join(cmd))
             subprocess.check_call(cmd)

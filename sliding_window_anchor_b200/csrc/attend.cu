@@ -35,7 +35,9 @@
 // Measured on B200 before this design: the same pipeline with CUDA-core FMAs
 // reached 80% of the measured copy bandwidth, and 105% with the math removed,
 // so the math, not the data path, was the limit.
-// A second kernel merges the splits of both branches when there are several.
+// Small batches split each branch's rows (up to 16 ways, one item per work
+// unit; with no more units than CTAs, CTA i takes unit i and touches no work
+// counter), and a second kernel merges the splits of both branches.
 // Every wait is bounded (≈2 s) and records ER_ETIMEOUT instead of hanging.
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -61,6 +63,7 @@ constexpr int BOX = 64 * 128;           // one 64-row x 64-dim box (8 KB, 128 B 
 constexpr int TILE_BYTES = 4 * BOX;     // a 64-row K (or V) tile: four boxes
 constexpr float kLog2eOver16 = 1.4426950408889634f / 16.0f;
 constexpr int F_FIRST = 1, F_LAST = 2, F_END = 4;  // F_END: no more work for this CTA
+constexpr int kMaxSplits = 16;          // splits of one (query, group, branch) read
 
 struct TileDesc {
   int rows;
@@ -258,18 +261,30 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
   // launched behind the kernel that writes q, the window slot and the pending
   // record (norm/RoPE): nothing above touched them
   grid_dep_wait();
+  grid_dep_trigger();  // the split merge after this read may set itself up (it waits for us)
 
-  // Work is handed out in units of two consecutive items (a (query, group)'s
-  // two branch items when unsplit, read back to back by one CTA): the producer
-  // takes the next unit from a counter in global memory (zeroed before the
-  // launch) when it has issued the last one, so CTAs that meet short items take
-  // more and all finish within about one unit of each other.  Nothing waits on
-  // another CTA.
-  const int n_units = n_items / 2;
+  // Work is handed out in units: two consecutive items when unsplit (a (query,
+  // group)'s two branch items, read back to back by one CTA, which writes their
+  // sum), one item when split (small batches: one or two tiles each, so every
+  // SM gets some).  The producer takes the next unit from a counter in global
+  // memory (zeroed before the launch) when it has issued the last one, so CTAs
+  // that meet short items take more and all finish within about one unit of
+  // each other.  Nothing waits on another CTA.
+  const int upi = P.splits == 1 ? 2 : 1;
+  const int n_units = n_items / upi;
 
   if (warp == NCW) {
     // ------------------------------------------------------------ producer
+    // with no more units than CTAs (small batches) each CTA takes unit blockIdx.x
+    // and no other: the counter's round trips stay off the short critical path
+    const bool fixed = n_units <= (int)gridDim.x;
+    bool first = true;
     auto take_unit = [&]() {
+      if (fixed) {
+        const int u = first ? (int)blockIdx.x : n_units;
+        first = false;
+        return u;
+      }
       int u = 0;
       if (lane == 0) u = atomicAdd(P.sched, 1);
       u = __shfl_sync(0xffffffffu, u, 0);
@@ -277,14 +292,14 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
     };
     TileIter ld;
     int unit = take_unit();
-    ld.init(&P, 2 * unit, 2 * min(unit + 1, n_units));
+    ld.init(&P, upi * unit, upi * min(unit + 1, n_units));
     Tile t;
     uint32_t tc = 0;
     while (true) {
       if (!ld.next(&t)) {
         if (unit >= n_units) break;
         unit = take_unit();
-        ld.init(&P, 2 * unit, 2 * min(unit + 1, n_units));
+        ld.init(&P, upi * unit, upi * min(unit + 1, n_units));
         continue;
       }
       const int stage = tc % STAGES;
@@ -603,30 +618,50 @@ __global__ void __launch_bounds__(NTHREADS, 1) k_attend(const __grid_constant__ 
   }
 }
 
+
 // Merge the splits of both branches for (query, head).
 //  mode 0: o_swa, o_rma FP32 [nq][16][256]; mode 1: o_sum BF16 [nq][4096] = bf16(o_swa + o_rma)
+// Every split's (m, l) and output element is requested before the first is
+// used (the loads of both branches are independent), so a merge costs one
+// round trip to L2 rather than one per split.  A programmatic launch: its
+// blocks wait beside the read's last CTAs (grid_dep_wait).
+template <int SPLITS>
 __global__ void __launch_bounds__(256) k_attend_merge(const float* __restrict__ part_o,
                                                       const float* __restrict__ part_ml,
-                                                      int splits, float* o_swa, float* o_rma,
+                                                      float* o_swa, float* o_rma,
                                                       uint16_t* o_sum) {
   const int qi = blockIdx.x, h = blockIdx.y, d = threadIdx.x;
   const int g = h / HPG, hh = h % HPG;
+  grid_dep_wait();     // the partials come from the read before
+  grid_dep_trigger();  // o_proj may start streaming its weights
+  float m[2][SPLITS], l[2][SPLITS], o[2][SPLITS];
+#pragma unroll
+  for (int br = 0; br < 2; ++br) {
+    const size_t base = (((size_t)qi * NG + g) * 2 + br) * SPLITS;
+#pragma unroll
+    for (int s = 0; s < SPLITS; ++s) {
+      const float2 ml = *reinterpret_cast<const float2*>(part_ml + ((base + s) * HPG + hh) * 2);
+      m[br][s] = ml.x;
+      l[br][s] = ml.y;
+      o[br][s] = part_o[((base + s) * HPG + hh) * D + d];
+    }
+  }
   float ob[2];
 #pragma unroll
   for (int br = 0; br < 2; ++br) {
-    const size_t base = (((size_t)qi * NG + g) * 2 + br) * splits;
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, part_ml[((base + s) * HPG + hh) * 2]);
-    float Ls = 0.f, o = 0.f;
+#pragma unroll
+    for (int s = 0; s < SPLITS; ++s) M = fmaxf(M, m[br][s]);
+    float Ls = 0.f, acc = 0.f;
     if (M != -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float m = part_ml[((base + s) * HPG + hh) * 2];
-        const float f = exp2f(m - M);
-        Ls += part_ml[((base + s) * HPG + hh) * 2 + 1] * f;
-        o += part_o[((base + s) * HPG + hh) * D + d] * f;
+#pragma unroll
+      for (int s = 0; s < SPLITS; ++s) {
+        const float f = exp2f(m[br][s] - M);
+        Ls += l[br][s] * f;
+        acc += o[br][s] * f;
       }
     }
-    ob[br] = Ls > 0.f ? o / Ls : 0.f;
+    ob[br] = Ls > 0.f ? acc / Ls : 0.f;
   }
   if (o_sum) {
     o_sum[(size_t)qi * OIN + h * D + d] = f2bf(ob[0] + ob[1]);
@@ -642,7 +677,7 @@ __global__ void __launch_bounds__(256) k_attend_merge(const float* __restrict__ 
 int attend_splits(int nq) {
   const int items = nq * NG * 2;
   int s = 1;
-  while (items * s < 296 && s < 16) s <<= 1;
+  while (items * s < 296 && s < kMaxSplits) s <<= 1;
   return s;
 }
 
@@ -693,7 +728,7 @@ int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* 
     }
   }
   const int n_items = P.nq * NG * 2 * P.splits;
-  const int grid = min(n_items, num_sms());
+  const int grid = min(P.splits == 1 ? n_items / 2 : n_items, num_sms());
   P.direct = P.splits == 1 ? 1 : 0;
   P.o_swa = o_swa;
   P.o_rma = o_rma;
@@ -720,8 +755,16 @@ int launch_attend(const AttendParams& P0, float* o_swa, float* o_rma, uint16_t* 
   count_launches(1);
   int rc = launch_status();
   if (rc != ER_OK || P.direct) return rc;
-  k_attend_merge<<<dim3(P.nq, NH), 256, 0, st>>>(P.part_o, P.part_ml, P.splits, o_swa, o_rma,
-                                                  o_sum);
+  cfg.gridDim = dim3(P.nq, NH);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  auto merge = P.splits == 2   ? k_attend_merge<2>
+               : P.splits == 4 ? k_attend_merge<4>
+               : P.splits == 8 ? k_attend_merge<8>
+                               : k_attend_merge<16>;
+  if (cudaLaunchKernelEx(&cfg, merge, (const float*)P.part_o, (const float*)P.part_ml, o_swa,
+                         o_rma, o_sum) != cudaSuccess)
+    return ER_ECUDA;
   count_launches(1);
   return launch_status();
 }

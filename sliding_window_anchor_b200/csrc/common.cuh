@@ -28,6 +28,7 @@ constexpr int ROW_BYTES = D * 2;        // one BF16 K or V row
 // The pooled state layout: bank and pending block share 1280 rows per group; a
 // free pool slot holds this position (above every stream position).
 constexpr int POOL = BANK + PEND;       // 1280
+constexpr int kGemvMaxTokensAll = 32;   // largest token count the GEMV kernel takes
 constexpr int32_t FREE_POS = 0x7FFFFFFF;
 
 // Column offsets of the six projections inside one [QKV] projection row.

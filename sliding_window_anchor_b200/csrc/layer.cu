@@ -15,9 +15,12 @@
 
 namespace er {
 
-size_t proj_workspace_bytes(int T, int F, int K);
-int launch_proj(const uint16_t* X, int T, const uint16_t* W, int F, int K, uint16_t* yb,
-                int ldb, int nbf, float* yf, int ldf, void* ws, int32_t* err, cudaStream_t st);
+int gemm_bf16_xwt(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
+                  cudaStream_t st);
+int gemm_bf16_xwt_f32(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K,
+                      int ldy, cudaStream_t st);
+int launch_gemv(const uint16_t* X, int T, const uint16_t* W, int F, int K, void* Y, bool yf32,
+                int ldy, cudaStream_t st);
 int launch_score(const float* w1, const uint16_t* w1_split, const float* w2, const uint16_t* x,
                  int n, float* s, void* scratch, int32_t* err, cudaStream_t st);
 size_t score_scratch_bytes(int n);
@@ -41,9 +44,27 @@ int launch_prefill_attend(const er_state* st, int layer, int seq, int T, const u
 namespace er {
 namespace {
 
+// A batch of at most this many tokens streams the weights through the
+// library's own GEMV kernel (the product is bound by reading the weights);
+// larger ones go to cuBLAS.
+constexpr int kGemvMaxTokens = 8;
+
+// Y[M,N] = X[M,K] · W[N,K]ᵀ, BF16 out (row stride N).
+int project_bf16(const uint16_t* X, const uint16_t* W, uint16_t* Y, int M, int N, int K,
+                 cudaStream_t st) {
+  if (M <= kGemvMaxTokens) return launch_gemv(X, M, W, N, K, Y, false, N, st);
+  return gemm_bf16_xwt(X, W, Y, M, N, K, st);
+}
+
+// The same with FP32 out of row stride ldy.
+int project_f32(const uint16_t* X, const uint16_t* W, float* Y, int M, int N, int K, int ldy,
+                cudaStream_t st) {
+  if (M <= kGemvMaxTokens) return launch_gemv(X, M, W, N, K, Y, true, ldy, st);
+  return gemm_bf16_xwt_f32(X, W, Y, M, N, K, ldy, st);
+}
+
 struct LayerWs {
-  uint16_t* proj;  // BF16 [nq][12288]: the six projections
-  float* w1_sums;  // FP32 [nq][768]: the three W1-term sums (fused weights)
+  void* proj;  // BF16 [nq][12288], or FP32 [nq][13056] with the fused weights
   unsigned char* score_scratch;
   uint16_t *q_swa, *q_rma;
   uint16_t *chunk_k, *chunk_v;
@@ -52,15 +73,13 @@ struct LayerWs {
   float* pf_out;             // prefill: FP32 branch outputs [2][T][4096]
   uint16_t* o_sum;
   MovePlan* plan;            // the commit's move lists, one per (sequence, group)
-  unsigned char* proj_ws;    // the projections' partial sums and flags (one GEMM at a time)
   size_t bytes;
 };
 
 LayerWs carve_ws(void* base, int nq, bool prefill) {
   Carver c(base);
   LayerWs w;
-  w.proj = c.take<uint16_t>((size_t)nq * QKV);
-  w.w1_sums = c.take<float>((size_t)nq * (QKVS - QKV));
+  w.proj = c.take<float>((size_t)nq * QKVS);
   w.score_scratch = c.take<unsigned char>(score_scratch_bytes(nq));
   w.q_swa = c.take<uint16_t>((size_t)nq * NH * D);
   w.q_rma = c.take<uint16_t>((size_t)nq * NH * D);
@@ -73,10 +92,6 @@ LayerWs carve_ws(void* base, int nq, bool prefill) {
   w.o_sum = c.take<uint16_t>((size_t)nq * OIN);
   w.plan = reinterpret_cast<MovePlan*>(
       c.take<unsigned char>(commit_plan_bytes(prefill ? 1 : nq, 1)));
-  size_t pw = proj_workspace_bytes(nq, QKVS, HID);
-  pw = std::max(pw, proj_workspace_bytes(nq, QKV, HID));
-  pw = std::max(pw, proj_workspace_bytes(nq, HID, OIN));
-  w.proj_ws = c.take<unsigned char>(pw);
   w.bytes = c.used();
   return w;
 }
@@ -155,26 +170,20 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   if (!sd) return ER_ECUDA;
   // with the RMA off nothing is scored: the plain BF16 projection is cheaper
   const bool fused = w->w_qkv_score != nullptr && !rma_off;
-  uint16_t* proj_bf = W.proj;
-  int32_t* err = st->dev_error;
+  uint16_t* proj_bf = static_cast<uint16_t*>(W.proj);
+  float* proj_f = static_cast<float*>(W.proj);
   if (fused) {
-    // a1 and a3's W1·x in one GEMM: the projections rounded to BF16, the W1-term
-    // sums kept in FP32
-    if ((rc = launch_proj(x, nq, w->w_qkv_score, QKVS, HID, proj_bf, QKV, QKV, W.w1_sums,
-                          QKVS - QKV, W.proj_ws, err, s)) != ER_OK)
+    // a1 and a3's W1·x in one GEMM, FP32 out
+    if ((rc = project_f32(x, w->w_qkv_score, proj_f, nq, QKVS, HID, QKVS, s)) != ER_OK)
       return rc;
   } else if (rma_off) {
     // a1: all six projections in one GEMM
-    if ((rc = launch_proj(x, nq, w->w_qkv, QKV, HID, proj_bf, QKV, QKV, nullptr, 0, W.proj_ws,
-                          err, s)) != ER_OK)
-      return rc;
+    if ((rc = project_bf16(x, w->w_qkv, proj_bf, nq, QKV, HID, s)) != ER_OK) return rc;
   } else if (!prefill) {
     // a1, then a3 (FP32 scores; the partials stay in the scratch, k_post_proj
     // adds them).  Measured: beside a batch's a1 GEMM, which fills the GPU, the
     // scorer slowed the decode step, so here they run in turn.
-    if ((rc = launch_proj(x, nq, w->w_qkv, QKV, HID, proj_bf, QKV, QKV, nullptr, 0, W.proj_ws,
-                          err, s)) != ER_OK)
-      return rc;
+    if ((rc = project_bf16(x, w->w_qkv, proj_bf, nq, QKV, HID, s)) != ER_OK) return rc;
     if ((rc = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr, W.score_scratch,
                            st->dev_error, s)) != ER_OK)
       return rc;
@@ -186,8 +195,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
       return ER_ECUDA;
     const int rc_score = launch_score(w->w1, w->w1_split, w->w2, x, nq, nullptr,
                                       W.score_scratch, st->dev_error, sd->stream);
-    const int rc_proj =
-        launch_proj(x, nq, w->w_qkv, QKV, HID, proj_bf, QKV, QKV, nullptr, 0, W.proj_ws, err, s);
+    const int rc_proj = project_bf16(x, w->w_qkv, proj_bf, nq, QKV, HID, s);
     if (cudaEventRecord(sd->join, sd->stream) != cudaSuccess ||
         cudaStreamWaitEvent(s, sd->join, 0) != cudaSuccess)
       return ER_ECUDA;
@@ -195,8 +203,8 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
   }
   // a2 + a4: norm/RoPE, window write (decode) or chunk rows (prefill), pending append
   PostParams pp{};
-  pp.proj = proj_bf;
-  pp.w1_sums = fused ? W.w1_sums : nullptr;
+  pp.proj = fused ? nullptr : proj_bf;
+  pp.proj_f32 = fused ? proj_f : nullptr;
   pp.s_part = fused ? nullptr : score_partials(W.score_scratch, nq);
   pp.w2 = w->w2;
   pp.nq = nq;
@@ -258,9 +266,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     rc_read = launch_attend(ap, nullptr, nullptr, W.o_sum, false, s);
   }
   if (rma_off)
-    return rc_read != ER_OK ? rc_read
-                            : launch_proj(W.o_sum, nq, w->w_o, HID, OIN, out, HID, HID,
-                                          nullptr, 0, W.proj_ws, err, s);
+    return rc_read != ER_OK ? rc_read : project_bf16(W.o_sum, w->w_o, out, nq, HID, OIN, s);
   // the moves wait for the reads (they overwrite evicted anchor rows); after a
   // failed launch nothing moves, but the side stream still joins
   int rc_move = ER_OK;
@@ -272,8 +278,7 @@ int run_layer(const er_state* st, const er_layer_weights* w, int layer, const in
     rc_move = launch_commit_move(cp, W.plan, sd->stream);
   const int rc_proj =
       rc_read == ER_OK
-          ? launch_proj(W.o_sum, nq, w->w_o, HID, OIN, out, HID, HID, nullptr, 0, W.proj_ws, err,
-                        s)
+          ? project_bf16(W.o_sum, w->w_o, out, nq, HID, OIN, s)
           : ER_OK;
   // join: the caller's stream waits for the side stream whatever happened above
   joined_ok = cudaEventRecord(sd->join, sd->stream) == cudaSuccess &&

@@ -135,10 +135,41 @@ __global__ void k_norm_rope(const uint16_t* x, uint16_t* y, int64_t n_rows, cons
 // run in series, at half the resident warps).
 namespace {
 
-// One head row: norm + RoPE where it has a gain, then its destination.
+// The retention score of token qi for group g (warp-wide; lane 0's value is
+// the one stored).  It needs no metadata, so k_post_proj forms it before its
+// barrier, beside the metadata loads.
+__device__ __forceinline__ float score_of(const PostParams& P, int qi, int g, int lane) {
+  float sc = 0.f;
+  if (P.proj_f32) {
+    // the score of group g from the fused GEMM: h_j = hi_j + mid_j + lo_j (the
+    // three W1-term sums, smallest first), s_g = sum_j W2[g][j] SiLU(h_j);
+    // lane covers j = 8 lane .. 8 lane + 7, then a fixed-order warp sum
+    const float4* hrow =
+        reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + QKV) + lane * 2;
+    const float4* w2g = reinterpret_cast<const float4*>(P.w2 + g * 256) + lane * 2;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float4 hi = hrow[e], mid = hrow[64 + e], lo = hrow[128 + e], w2 = w2g[e];
+      const float h0 = (lo.x + mid.x) + hi.x, h1 = (lo.y + mid.y) + hi.y;
+      const float h2 = (lo.z + mid.z) + hi.z, h3 = (lo.w + mid.w) + hi.w;
+      sc += w2.x * (h0 / (1.0f + expf(-h0))) + w2.y * (h1 / (1.0f + expf(-h1))) +
+            w2.z * (h2 / (1.0f + expf(-h2))) + w2.w * (h3 / (1.0f + expf(-h3)));
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+  } else if (lane == 0) {
+    // the separate scorer: its 4 quarter partials added in order
+#pragma unroll
+    for (int q = 0; q < 4; ++q) sc += P.s_part[((size_t)q * P.nq + qi) * NG + g];
+  }
+  return sc;
+}
+
+// One head row: norm + RoPE where it has a gain, then its destination (sc: the
+// group's score, for the k_rma rows).
 __device__ __forceinline__ void post_row(const PostParams& P, int hs, int lane, int qi, int seq,
                                          int32_t t, int p_idx, bool state_ok,
-                                         const float2* s_cs, float v[8]) {
+                                         const float2* s_cs, float v[8], float sc) {
   const uint16_t* gain = nullptr;
   if (hs < 16) gain = P.gq_swa;
   else if (hs < 20) gain = P.gk_swa;
@@ -179,29 +210,6 @@ __device__ __forceinline__ void post_row(const PostParams& P, int hs, int lane, 
     dst = ((hs < 44) ? (P.pool ? P.bank_k : P.pend_k) : (P.pool ? P.bank_v : P.pend_v)) +
           rec * D;
     if (hs < 44) {
-      float sc = 0.f;
-      if (P.w1_sums) {
-        // the score of group g from the fused GEMM: h_j = hi_j + mid_j + lo_j (the
-        // three W1-term sums, smallest first), s_g = sum_j W2[g][j] SiLU(h_j);
-        // lane covers j = 8 lane .. 8 lane + 7, then a fixed-order warp sum
-        const float4* hrow =
-            reinterpret_cast<const float4*>(P.w1_sums + (size_t)qi * (QKVS - QKV)) + lane * 2;
-        const float4* w2g = reinterpret_cast<const float4*>(P.w2 + g * 256) + lane * 2;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float4 hi = hrow[e], mid = hrow[64 + e], lo = hrow[128 + e], w2 = w2g[e];
-          const float h0 = (lo.x + mid.x) + hi.x, h1 = (lo.y + mid.y) + hi.y;
-          const float h2 = (lo.z + mid.z) + hi.z, h3 = (lo.w + mid.w) + hi.w;
-          sc += w2.x * (h0 / (1.0f + expf(-h0))) + w2.y * (h1 / (1.0f + expf(-h1))) +
-                w2.z * (h2 / (1.0f + expf(-h2))) + w2.w * (h3 / (1.0f + expf(-h3)));
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
-      } else if (lane == 0) {
-        // the separate scorer: its 4 quarter partials added in order
-#pragma unroll
-        for (int q = 0; q < 4; ++q) sc += P.s_part[((size_t)q * P.nq + qi) * NG + g];
-      }
       if (lane == 0) {
         if (P.pool) {
           P.bank_score[rec] = sc;
@@ -260,7 +268,19 @@ __global__ void __launch_bounds__(256, 8) k_post_proj(PostParams P) {
   // its latency overlaps warp 0's metadata and rotations.
   grid_dep_wait();
   float v[8];
-  load8(P.proj + (size_t)qi * QKV + row_col(hs) + lane * 8, v);
+  const int col = row_col(hs);
+  if (P.proj_f32) {
+    // FP32 sums of the fused GEMM, rounded to BF16 as a BF16-output GEMM would
+    const float4* src =
+        reinterpret_cast<const float4*>(P.proj_f32 + (size_t)qi * QKVS + col) + lane * 2;
+    const float4 a = src[0], b = src[1];
+    v[0] = bf1(f2bf(a.x)); v[1] = bf1(f2bf(a.y)); v[2] = bf1(f2bf(a.z)); v[3] = bf1(f2bf(a.w));
+    v[4] = bf1(f2bf(b.x)); v[5] = bf1(f2bf(b.y)); v[6] = bf1(f2bf(b.z)); v[7] = bf1(f2bf(b.w));
+  } else {
+    load8(P.proj + (size_t)qi * QKV + col + lane * 8, v);
+  }
+  // the k_rma rows' score (no metadata needed)
+  const float sc = (hs >= 40 && hs < 44) ? score_of(P, qi, hs - 40, lane) : 0.f;
   __syncthreads();
   if (!s_tok[3]) {  // the same for the whole block
     if (hs == 0 && lane == 0) set_dev_error(P.err, ER_EINVAL);
@@ -271,7 +291,7 @@ __global__ void __launch_bounds__(256, 8) k_post_proj(PostParams P) {
   const int p_idx = s_tok[2];
   const bool state_ok = p_idx >= 0 && p_idx < PEND && t >= 0;
   if (!state_ok && hs == 40 && lane == 0) set_dev_error(P.err, ER_ECAPACITY);
-  post_row(P, hs, lane, qi, seq, t, p_idx, state_ok, s_cs, v);
+  post_row(P, hs, lane, qi, seq, t, p_idx, state_ok, s_cs, v, sc);
 }
 
 int launch_post_proj(const PostParams& P, bool rma_off, cudaStream_t st) {

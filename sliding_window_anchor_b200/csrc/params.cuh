@@ -9,8 +9,8 @@
 namespace er {
 
 struct PostParams {
-  const uint16_t* proj;      // [nq][12288] BF16: the six projections
-  const float* w1_sums;      // fused scorer: [nq][768] FP32 hi/mid/lo W1-term sums (or NULL)
+  const uint16_t* proj;      // [nq][12288] BF16 (separate scorer), or
+  const float* proj_f32;     // [nq][13056] FP32: q/k/v sums, then hi/mid/lo W1-term sums
   const float* s_part;       // separate scorer: [4 hidden quarters][nq][4] partial scores
   const float* w2;           // fused: W2 [4][256] FP32
   int nq;

@@ -46,6 +46,10 @@ constexpr int PJ_MAXST = 8;
 constexpr int W_BOX_BYTES = 128 * 128;  // 128 features x 64 K of BF16
 constexpr int XBIG = 128, XSMALL = 32, XTINY = 8;  // X box rows
 constexpr int PJ_SMEM_LIMIT = 232448;
+constexpr int EB = 16;                  // tokens per epilogue block
+constexpr int EB_BYTES = EB * 128 * 4;  // one block of 128 FP32 features: 8 KB
+constexpr int PJ_STAGE_OUT = 2 * EB_BYTES;  // the two staging buffers of the stores
+constexpr int PJ_MAXRING = 16;
 constexpr uint64_t kFlagTag = 0xE5C0DE0000000000ull;
 constexpr uint64_t kDrainNs = 200000;
 
@@ -56,12 +60,12 @@ struct ProjPlan {
   int n_tc;      // chunks: ceil(T16 / chunk)
   int T16;       // T rounded up to 16
   int P;         // pairs
-  long U;        // units: n_ft * n_tc * KB
+  int U;         // units: n_ft * n_tc * KB (< 2^17 for every layer shape)
   int max_acc;   // accumulators per chunk (1: chunk <= 256, else 2)
   int x_acc_bytes;  // shared-memory bytes of one accumulator's X rows per CTA
   int stage_bytes, stages;
-  int blk_tok;      // tokens per partial block a finishing pair pulls in (<= 32)
   int nq_max;       // most contributor pairs of one tile
+  int ring;         // a finishing pair's partial-block slots in the idle stage memory
 };
 
 struct ProjParams {
@@ -86,15 +90,16 @@ struct Seg {
   int q_first, q_last;  // SEG_OWNER: the pairs whose partials complete the tile
 };
 
-__host__ __device__ inline long share_begin(const ProjPlan& p, int pair) {
-  return p.U * pair / p.P;
+// First unit of a pair's share (32-bit: U * P stays below 2^31).
+__host__ __device__ inline int share_begin(const ProjPlan& p, int pair) {
+  return (int)((unsigned)p.U * (unsigned)pair / (unsigned)p.P);
 }
 
 // The segments of one pair's share, in order.
 struct SegIter {
   const ProjPlan* p;
   int pair;
-  long cur, end;
+  int cur, end;
   __host__ __device__ void init(const ProjPlan* pl, int pr) {
     p = pl;
     pair = pr;
@@ -103,17 +108,17 @@ struct SegIter {
   }
   __host__ __device__ bool next(Seg& s) {
     if (cur >= end) return false;
-    const long tile = cur / p->KB;
-    const int kb0 = (int)(cur % p->KB);
-    const long tile_end = (tile + 1) * p->KB;
-    const long seg_end = end < tile_end ? end : tile_end;
-    s.ft = (int)(tile / p->n_tc);
-    s.tc = (int)(tile % p->n_tc);
+    const int tile = cur / p->KB;
+    const int kb0 = cur % p->KB;
+    const int tile_end = (tile + 1) * p->KB;
+    const int seg_end = end < tile_end ? end : tile_end;
+    s.ft = tile / p->n_tc;
+    s.tc = tile % p->n_tc;
     s.tok0 = s.tc * p->chunk;
     const int rem = p->T16 - s.tok0;
     s.ntok = rem < p->chunk ? rem : p->chunk;
     s.kb0 = kb0;
-    s.nkb = (int)(seg_end - cur);
+    s.nkb = seg_end - cur;
     s.q_first = s.q_last = -1;
     if (kb0 > 0) {
       s.role = SEG_CONTRIB;
@@ -150,6 +155,11 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   return v;
 }
 
+// Generic-proxy writes to this CTA's shared memory become visible to the TMA.
+__device__ __forceinline__ void fence_async_smem_cta() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // AND of a predicate over the `n` threads that meet at named barrier `id`.
 __device__ __forceinline__ bool bar_and(int id, int n, bool v) {
   uint32_t r;
@@ -170,11 +180,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PJ_THREADS, 1)
   const ProjPlan& pl = P.plan;
   const int NST = pl.stages, SB = pl.stage_bytes;
   struct Bars {
-    uint64_t full[PJ_MAXST], empty[PJ_MAXST], tfull[2], tempty[2], mma_done, pbar[2];
+    uint64_t full[PJ_MAXST], empty[PJ_MAXST], tfull[2], tempty[2], mma_done, pbar[PJ_MAXRING];
     uint32_t tmem_base;
     volatile int failed;
+    int qlist[PJ_MAXRING];  // a finishing pair's contributors (non-empty shares), in K order
   };
-  Bars& B = *reinterpret_cast<Bars*>(base + NST * SB);
+  unsigned char* stg = base + NST * SB;  // two staging buffers for the stores
+  Bars& B = *reinterpret_cast<Bars*>(stg + PJ_STAGE_OUT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = tc::cluster_rank();
   const uint32_t lead = rank & ~1u, peer = rank ^ 1u;
@@ -190,8 +202,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PJ_THREADS, 1)
       mbar_init(&B.tempty[b], 8);  // four epilogue warps of each CTA
     }
     mbar_init(&B.mma_done, 1);
-    mbar_init(&B.pbar[0], 1);
-    mbar_init(&B.pbar[1], 1);
+    for (int r = 0; r < PJ_MAXRING; ++r) mbar_init(&B.pbar[r], 1);
     B.failed = 0;
     fence_mbar_init();
   }
@@ -299,27 +310,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PJ_THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // The four warps take every decision together (bar.red over their 128
-    // threads), so they always meet at the same named barriers.
+    // Blocks of 16 tokens: TMEM -> registers (-> plus the partials of the pairs
+    // that finish this tile) -> a staging buffer (two, alternating) -> 16-byte
+    // stores of whole row segments (the TMA engine stays with the operand
+    // loads; stores queued behind them waited microseconds).  The four warps take
+    // every decision together
+    // (bar.red over their 128 threads), so they always meet at the same named
+    // barriers.
     const uint32_t lane_addr = (uint32_t)(32 * warp) << 16;
     const int fl = 32 * warp + lane;  // this thread's feature within the CTA's 128
     const int ep = threadIdx.x;       // 0..127
-    const int bt = pl.blk_tok;        // tokens per partial block
-    const uint32_t blk_bytes = (uint32_t)bt * 128 * 4;
-    int accn = 0, pk = 0;             // accumulators drained, partial blocks consumed
+    const int R = pl.ring;
+    const uint32_t slot_bytes = (uint32_t)pl.nq_max * EB_BYTES;
+    int accn = 0, pk = 0, nst = 0;    // accumulators drained, partial blocks, stores issued
     bool ok = true;
     while (ok && it.next(sg)) {
       const int na = seg_acc(sg);
-      const int f = 256 * sg.ft + 128 * (int)rank + fl;
+      const int f0 = 256 * sg.ft + 128 * (int)rank;  // the CTA's first feature
+      const bool fp32_y = f0 >= P.nbf;
       int nq = 0;  // contributors (pairs with a non-empty share) of an owner's tile
       if (sg.role == SEG_OWNER) {
         // the pairs holding the tile's later K steps must have left their partials
         bool got = true;
         if (ep == 0) {
           const unsigned long long want = kFlagTag | P.epoch;
-          for (int q = sg.q_first; q <= sg.q_last && got; ++q) {
-            if (share_begin(pl, q) == share_begin(pl, q + 1)) continue;  // an empty share
-            const unsigned long long* fp = P.flags + 2 * q + rank;
+          int n = 0;
+          for (int q = sg.q_first; q <= sg.q_last; ++q)
+            if (share_begin(pl, q) != share_begin(pl, q + 1) && n < PJ_MAXRING) B.qlist[n++] = q;
+          for (int qi = 0; qi < n && got; ++qi) {
+            const unsigned long long* fp = P.flags + 2 * B.qlist[qi] + rank;
             const uint64_t t0 = globaltimer_ns();
             while (ld_acquire_u64(fp) != want) {
               if (globaltimer_ns() - t0 > kWaitLimitNs || B.failed) {
@@ -343,67 +362,81 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PJ_THREADS, 1)
         if (!ok) break;
         tc::fence_after_sync();
         const int nj = acc_n(sg, j);
-        const int nblk = (nj + bt - 1) / bt;
-        // an owner's partial blocks: block k of every contributor into buffer k & 1
-        // (the pipeline's stage memory, idle once this segment's MMAs are done)
+        const int nblk = nj / EB;
+        // an owner's partial blocks: block k of every contributor into ring slot
+        // (pk + k) % R (the stage memory, idle once this segment's MMAs are done)
         auto issue = [&](int k) {
-          const int tl = 256 * j + k * bt;  // first token of the block in the chunk
-          const int ntk = min(bt, nj - k * bt);
-          const int buf = (pk + k) & 1;
-          mbar_arrive_expect_tx(&B.pbar[buf], (uint32_t)(nq * ntk * 128 * 4));
-          int qi = 0;
-          for (int q = sg.q_first; q <= sg.q_last; ++q) {
-            if (share_begin(pl, q) == share_begin(pl, q + 1)) continue;
-            bulk_g2s(base + ((size_t)buf * pl.nq_max + qi) * blk_bytes,
-                     P.part + (((size_t)q * 2 + rank) * pl.chunk + tl) * 128,
-                     (uint32_t)(ntk * 128 * 4), &B.pbar[buf]);
-            ++qi;
-          }
+          const int u = pk + k, slot = u % R;
+          const int tl = 256 * j + k * EB;  // first token of the block in the chunk
+          mbar_arrive_expect_tx(&B.pbar[slot], (uint32_t)(nq * EB_BYTES));
+          for (int qi = 0; qi < nq; ++qi)
+            bulk_g2s(base + (size_t)slot * slot_bytes + (size_t)qi * EB_BYTES,
+                     P.part + (((size_t)B.qlist[qi] * 2 + rank) * pl.chunk + tl) * 128,
+                     EB_BYTES, &B.pbar[slot]);
         };
-        if (sg.role == SEG_OWNER && ep == 0) issue(0);
+        if (sg.role == SEG_OWNER && ep == 0)
+          for (int k = 0; k < R - 1 && k < nblk; ++k) issue(k);
+        uint32_t r[32];
         for (int k = 0; k < nblk; ++k) {
-          if (sg.role == SEG_OWNER && ep == 0 && k + 1 < nblk) issue(k + 1);
-          for (int cbi = 0; cbi < bt; cbi += 32) {
-            if (cbi >= nj - k * bt) break;
-            uint32_t r[32];
-            tc::tmem_ld32(tmem + lane_addr + 256u * b + k * bt + cbi, r);
+          if ((k & 1) == 0) {
+            tc::tmem_ld32(tmem + lane_addr + 256u * b + k * EB, r);
             tc::tmem_wait_ld();
-            const int tl0 = 256 * j + k * bt + cbi;  // the chunk's token in column 0
-            const int nv = min(32, min(bt - cbi, nj - k * bt - cbi));  // valid columns
-            if (sg.role == SEG_OWNER) {
-              const int buf = (pk + k) & 1;
-              if (cbi == 0 &&
-                  !mbar_wait(&B.pbar[buf], ((pk + k) >> 1) & 1, P.err))
-                B.failed = 1;
-              for (int qi = 0; qi < nq; ++qi) {
-                const float* src = reinterpret_cast<const float*>(
-                                       base + ((size_t)buf * pl.nq_max + qi) * blk_bytes) +
-                                   (size_t)cbi * 128 + fl;
+          }
+          float v[EB];
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                  if (c < nv) r[c] = __float_as_uint(__uint_as_float(r[c]) + src[c * 128]);
-              }
+          for (int c = 0; c < EB; ++c) v[c] = __uint_as_float((k & 1) ? r[EB + c] : r[c]);
+          if (sg.role == SEG_OWNER) {
+            const int u = pk + k;
+            if (!mbar_wait(&B.pbar[u % R], (u / R) & 1, P.err)) B.failed = 1;
+            const float* src = reinterpret_cast<const float*>(base + (size_t)(u % R) * slot_bytes);
+            for (int qi = 0; qi < nq; ++qi)
+#pragma unroll
+              for (int c = 0; c < EB; ++c) v[c] += src[qi * (EB * 128) + c * 128 + fl];
+          }
+          // stage the block ([16 tokens][128 features]; a thread writes its
+          // feature's column), then store it with coalesced 16-byte writes
+          unsigned char* sb = stg + (nst & 1) * EB_BYTES;
+          const bool f32 = sg.role == SEG_CONTRIB || fp32_y;
+          if (f32) {
+#pragma unroll
+            for (int c = 0; c < EB; ++c) reinterpret_cast<float*>(sb)[c * 128 + fl] = v[c];
+          } else {
+#pragma unroll
+            for (int c = 0; c < EB; ++c) reinterpret_cast<uint16_t*>(sb)[c * 128 + fl] = f2bf(v[c]);
+          }
+          // the block is staged; the ring slot of the previous block has been read
+          named_bar_sync(1, 128);
+          if (sg.role == SEG_OWNER && ep == 0 && k + R - 1 < nblk) issue(k + R - 1);
+          const int tl = 256 * j + k * EB;  // the chunk's token in row 0 of the block
+          if (sg.role == SEG_CONTRIB) {
+            // 16 x 512 B, contiguous in the pair's partial buffer
+            float4* dst = reinterpret_cast<float4*>(
+                P.part + (((size_t)pair * 2 + rank) * pl.chunk + tl) * 128);
+#pragma unroll
+            for (int i = 0; i < EB * 32 / 128; ++i)
+              __stcg(dst + ep + 128 * i, reinterpret_cast<const float4*>(sb)[ep + 128 * i]);
+          } else if (fp32_y) {
+            // 32 chunks of 16 B per token row
+#pragma unroll
+            for (int i = 0; i < EB * 32 / 128; ++i) {
+              const int ci = ep + 128 * i, row = ci >> 5, col = ci & 31;
+              const int tok = sg.tok0 + tl + row;
+              if (tok < pl.T)
+                *reinterpret_cast<float4*>(P.yf + (size_t)tok * P.ldf + (f0 - P.nbf) + 4 * col) =
+                    reinterpret_cast<const float4*>(sb)[ci];
             }
-            if (sg.role == SEG_CONTRIB) {
-              float* dst = P.part + (((size_t)pair * 2 + rank) * pl.chunk + tl0) * 128 + fl;
+          } else {
+            // 16 chunks of 16 B per token row
 #pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c < nv) __stcg(dst + (size_t)c * 128, __uint_as_float(r[c]));
-            } else if (f < P.nbf) {
-              uint16_t* dst = P.yb + (size_t)(sg.tok0 + tl0) * P.ldb + f;
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c < nv && sg.tok0 + tl0 + c < pl.T)
-                  dst[(size_t)c * P.ldb] = f2bf(__uint_as_float(r[c]));
-            } else {
-              float* dst = P.yf + (size_t)(sg.tok0 + tl0) * P.ldf + (f - P.nbf);
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (c < nv && sg.tok0 + tl0 + c < pl.T) dst[(size_t)c * P.ldf] = __uint_as_float(r[c]);
+            for (int i = 0; i < EB * 16 / 128; ++i) {
+              const int ci = ep + 128 * i, row = ci >> 4, col = ci & 15;
+              const int tok = sg.tok0 + tl + row;
+              if (tok < pl.T)
+                *reinterpret_cast<uint4*>(P.yb + (size_t)tok * P.ldb + f0 + 8 * col) =
+                    reinterpret_cast<const uint4*>(sb)[ci];
             }
           }
-          // every thread is done with buffer (pk + k) & 1 before it is refilled
-          if (sg.role == SEG_OWNER) named_bar_sync(1, 128);
+          ++nst;
         }
         if (sg.role == SEG_OWNER) pk += nblk;
         tc::fence_before_sync();
@@ -456,7 +489,7 @@ double plan_cost(const ProjPlan& p) {
   constexpr double kFlopPerCycle = 7700.0;   // BF16 tensor rate per SM
   constexpr double kHbmBytesPerCycle = 27.0;
   constexpr double kL2BytesPerCycle = 65.0;
-  constexpr double kStoreBytesPerCycle = 64.0;
+  constexpr double kStoreBytesPerCycle = 60.0;
   constexpr double kSegCycles = 1500.0;
   double worst = 0.0;
   for (int pr = 0; pr < p.P; ++pr) {
@@ -493,14 +526,14 @@ ProjPlan make_plan(int T, int F, int K, int pairs, int chunk) {
   p.chunk = chunk;
   p.n_tc = (p.T16 + chunk - 1) / chunk;
   p.P = pairs;
-  p.U = (long)p.n_ft * p.n_tc * p.KB;
+  p.U = p.n_ft * p.n_tc * p.KB;
   p.max_acc = chunk > 256 ? 2 : 1;
   p.x_acc_bytes = x_acc_bytes_for(chunk);
   p.stage_bytes = W_BOX_BYTES + p.max_acc * p.x_acc_bytes;
-  const int room = PJ_SMEM_LIMIT - 1024 - 1024;  // alignment slack, barriers
+  // alignment slack, barriers, the staging buffers of the stores
+  const int room = PJ_SMEM_LIMIT - 2048 - PJ_STAGE_OUT;
   p.stages = room / p.stage_bytes;
   if (p.stages > PJ_MAXST) p.stages = PJ_MAXST;
-  p.blk_tok = chunk < 32 ? chunk : 32;
   p.nq_max = 0;
   for (int pr = 0; pr < p.P; ++pr) {
     SegIter it;
@@ -514,14 +547,20 @@ ProjPlan make_plan(int T, int F, int K, int pairs, int chunk) {
         if (n > p.nq_max) p.nq_max = n;
       }
   }
+  p.ring = 0;
+  if (p.nq_max > 0) {
+    p.ring = (int)((long)p.stages * p.stage_bytes / ((long)p.nq_max * EB_BYTES));
+    if (p.ring > PJ_MAXRING) p.ring = PJ_MAXRING;
+  } else {
+    p.ring = 2;
+  }
   return p;
 }
 
-// The partial blocks of a finishing pair (two buffers of nq_max blocks) must fit
-// in the stage memory they borrow.
+// A finishing pair borrows the stage memory for at least two ring slots of
+// partial blocks.
 bool plan_fits(const ProjPlan& p) {
-  return p.stages >= 2 &&
-         2L * p.nq_max * p.blk_tok * 128 * 4 <= (long)p.stages * p.stage_bytes;
+  return p.stages >= 2 && p.ring >= 2 && p.nq_max <= PJ_MAXRING;
 }
 
 ProjPlan choose_plan(int T, int F, int K, int pairs) {
@@ -609,6 +648,9 @@ std::atomic<uint32_t> g_epoch{1};
 
 }  // namespace
 
+int launch_gemv(const uint16_t* X, int T, const uint16_t* W, int F, int K, void* Y, bool yf32,
+                int ldy, cudaStream_t st);
+
 // Workspace of one projection: the partial sums of the pairs that hand a tile
 // to another (one chunk of 256 features each) and their flags.
 size_t proj_workspace_bytes(int T, int F, int K) {
@@ -639,6 +681,8 @@ int launch_proj(const uint16_t* X, int T, const uint16_t* W, int F, int K, uint1
       !encode_bf16_2d(&P.x_small, X, (uint64_t)K, (uint64_t)T, (uint64_t)K * 2, 64, XSMALL) ||
       !encode_bf16_2d(&P.x_tiny, X, (uint64_t)K, (uint64_t)T, (uint64_t)K * 2, 64, XTINY))
     return ER_ECUDA;
+  if ((nbf > 0 && ((uintptr_t)yb & 15u || ldb % 8)) || (nbf < F && ((uintptr_t)yf & 15u || ldf % 4)))
+    return ER_EINVAL;
   Carver c(ws);
   P.part = c.take<float>((size_t)P.plan.P * 2 * P.plan.chunk * 128);
   P.flags = c.take<unsigned long long>((size_t)P.plan.P * 2);
@@ -649,7 +693,7 @@ int launch_proj(const uint16_t* X, int T, const uint16_t* W, int F, int K, uint1
   P.ldf = ldf;
   P.epoch = g_epoch.fetch_add(1, std::memory_order_relaxed) & 0xFFFFFFu;
   P.err = err;
-  const int smem = P.plan.stages * P.plan.stage_bytes + 2048;
+  const int smem = P.plan.stages * P.plan.stage_bytes + PJ_STAGE_OUT + 2048;
   {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return ER_ECUDA;
@@ -699,6 +743,8 @@ int er_linear(const er_bf16* x, int32_t T, const er_bf16* w, int32_t F, int32_t 
   int32_t* err = dev_error ? dev_error : call_error_word();
   if (!err) return ER_ECUDA;
   const bool bf = y_fp32 == 0;
+  if (T <= kGemvMaxTokensAll)
+    return launch_gemv(x, T, w, F, K, y, !bf, ldy, (cudaStream_t)stream);
   return launch_proj(x, T, w, F, K, bf ? static_cast<uint16_t*>(y) : nullptr, ldy, bf ? F : 0,
                      bf ? nullptr : static_cast<float*>(y), ldy, ws, err, (cudaStream_t)stream);
 }

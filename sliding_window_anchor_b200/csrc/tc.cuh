@@ -252,6 +252,39 @@ __device__ __forceinline__ void tma_load_4d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// A TMA store of one 2-D box from this CTA's shared memory (plain row-major)
+// into the tensor at (x, y); the copy joins the thread's current bulk group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y,
+                                             const void* src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(smem_u32(src))
+      : "memory");
+}
+
+// A bulk store of `bytes` (multiple of 16) from shared memory to global memory.
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Until at most N of this thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Until every bulk group of this thread has completed (its writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 // Arrivals on an mbarrier given by its shared::cluster address (this CTA's or
 // the peer's).  What they publish is tcgen05 work ordered by
 // tcgen05.fence::before_thread_sync, and TMA transaction counts.
@@ -272,6 +305,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar, uint
 // outside the tensor.
 bool encode_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
                  const uint64_t* strides_bytes, const uint32_t* box);
+
+// Host: a 2-D map for TMA stores of [box_rows][box_cols] blocks from plain
+// (unswizzled) row-major shared memory into a BF16 or FP32 matrix of `rows`
+// rows of `cols` elements (row pitch `pitch_bytes`); rows past `rows` are not
+// written.
+bool encode_store_2d(CUtensorMap* m, const void* base, bool fp32, uint64_t cols, uint64_t rows,
+                     uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows);
 
 // Host: encode a 2-D BF16 tensor map over `rows` rows of `cols` elements
 // (row pitch `pitch_bytes`), box `box_cols` x `box_rows`, 128-byte swizzle,

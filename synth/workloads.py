@@ -33,19 +33,28 @@ D, HIDDEN, NG, NH, WIN, BANK, PEND = 256, 2560, 4, 16, 1024, 1024, 256
 QKV = 12288
 BASE_SEED = 20261202
 
+# The workloads, by name: sizes, state recipe and the offset of their seed.
+DECODE_B1 = "decode_b1_l1_t4096"
+COMMIT = "commit_b512_l8"
+DECODE_B64 = "decode_b64_l8_t32768"
+DECODE_B512 = "decode_b512_l8_t32768"
+PREFILL = "prefill_b1_l8_131072"
 CONFIGS = {
-    0: dict(name="decode_b1_l1_t4096", B=1, n_layers=1, t0=4096, pend="zero", steps=256),
-    1: dict(name="commit_b512_l8", B=512, n_layers=8, t0=32768, pend="full", steps=0),
-    2: dict(name="decode_b64_l8_t32768", B=64, n_layers=8, t0=32768, pend="uniform", steps=1024),
-    3: dict(name="decode_b512_l8_t32768", B=512, n_layers=8, t0=32768, pend="uniform",
-            steps=2048),
-    4: dict(name="prefill_b1_l8_131072", B=1, n_layers=8, t0=0, pend="zero", tokens=131072,
-            chunk=256),
+    DECODE_B1: dict(name=DECODE_B1, B=1, n_layers=1, t0=4096, pend="zero", steps=256,
+                    seed_offset=0),
+    COMMIT: dict(name=COMMIT, B=512, n_layers=8, t0=32768, pend="full", steps=0, seed_offset=1),
+    DECODE_B64: dict(name=DECODE_B64, B=64, n_layers=8, t0=32768, pend="uniform", steps=1024,
+                     seed_offset=2),
+    DECODE_B512: dict(name=DECODE_B512, B=512, n_layers=8, t0=32768, pend="uniform",
+                      steps=2048, seed_offset=3),
+    PREFILL: dict(name=PREFILL, B=1, n_layers=8, t0=0, pend="zero", tokens=131072, chunk=256,
+                  seed_offset=4),
 }
 
 
-def seed_of(cfg_index: int) -> int:
-    return BASE_SEED + int(cfg_index)
+def seed_of(workload: str) -> int:
+    """The base seed of a named workload (CONFIGS)."""
+    return BASE_SEED + CONFIGS[workload]["seed_offset"]
 
 
 # --------------------------------------------------------------- weights

@@ -62,7 +62,7 @@ def download_row(st, row):
 
 
 def tol_ok(gpu, ref, atol=1e-2, rtol=1e-2):
-    """Spec tolerance for attention/layer outputs: |Δ| <= atol + rtol·|ref|."""
+    """The stated tolerance for attention/layer outputs: |Δ| <= atol + rtol·|ref|."""
     g = gpu.double().cpu()
     r = ref.double().cpu()
     return bool(((g - r).abs() <= atol + rtol * r.abs()).all())

@@ -39,7 +39,7 @@ def _run_oracle_seq(ow_list, ost, row, steps, layers, seed, gseq, x_of):
 
 def test_decode_single_layer_256_steps_with_commit(sab):
     """B=1, one layer, state at 4096, empty pending: 256 steps, one commit at the last."""
-    cfg, seed = wl.CONFIGS[0], wl.seed_of(0)
+    cfg, seed = wl.CONFIGS[wl.DECODE_B1], wl.seed_of(wl.DECODE_B1)
     L = cfg["n_layers"]
     ow, wdict = H.oracle_weights(seed, 0)
     gw, gdict = H.gpu_weights(seed, 0)
@@ -60,7 +60,7 @@ def test_decode_single_layer_256_steps_with_commit(sab):
         ost.advance(0)
         assert H.tol_ok(gouts[step][0], ref), (step, H.max_err(gouts[step][0], ref))
         worst = max(worst, H.max_err(gouts[step][0], ref) / float(ref.double().abs().max()))
-    print(f"config0 worst |Δ|/max|ref| = {worst:.3e}")
+    print(f"{wl.DECODE_B1} worst |Δ|/max|ref| = {worst:.3e}")
     assert worst < 2e-2
     grow, orow = H.download_row(st, 0), {n: getattr(ost, n)[0] for n in oracle.OracleState.ARRAYS}
     assert torch.equal(grow["meta"], orow["meta"])
@@ -85,20 +85,21 @@ def _pick_sequences(fills, steps, n_commit, n_other):
     return chosen
 
 
-# config 3 (B=512): the oracle follows 8 sequences for 64 steps, 6 of them committing at
-# different steps; config 2 (B=64): 300 steps, so every sequence crosses its commit
-# (staggered by its fill) and the fullest ones a second one
-BATCHED = {2: dict(steps=300, n_commit=6, n_other=0), 3: dict(steps=64, n_commit=6, n_other=2)}
+# the B=512 decode batch: the oracle follows 8 sequences for 64 steps, 6 of them
+# committing at different steps; the B=64 batch: 300 steps, so every followed sequence
+# crosses its commit (staggered by its fill) and the fullest ones a second one
+BATCHED = {wl.DECODE_B64: dict(steps=300, n_commit=6, n_other=0),
+           wl.DECODE_B512: dict(steps=64, n_commit=6, n_other=2)}
 
 
-@pytest.mark.parametrize("cfg_index", [2, 3])
-def test_decode_batched_sampled_sequences(sab, cfg_index):
+@pytest.mark.parametrize("workload", [wl.DECODE_B64, wl.DECODE_B512])
+def test_decode_batched_sampled_sequences(sab, workload):
     """Full batch on the device (B=64 or 512, 8 layers, t0=32768, random fills); the
     oracle follows sampled sequences through staggered, device-gated commits.  Every
     layer output of every step within the stated tolerance; metadata equal and kept
     anchor sets equal (up to boundary near-ties) at the end."""
-    cfg, seed = wl.CONFIGS[cfg_index], wl.seed_of(cfg_index)
-    plan = BATCHED[cfg_index]
+    cfg, seed = wl.CONFIGS[workload], wl.seed_of(workload)
+    plan = BATCHED[workload]
     B, L, steps = cfg["B"], cfg["n_layers"], plan["steps"]
     gws, gdicts = zip(*[H.gpu_weights(seed, l) for l in range(L)])
     st = sab.State(B, L)
@@ -146,7 +147,7 @@ def test_graph_replayed_steps_equal_eager_steps_and_oracle(sab):
     some sequences commit and others do not: the same bits as the same steps run
     call by call on a copy of the state, outputs and every state array; sampled
     sequences (one committing, one not) within tolerance of the oracle."""
-    cfg, seed = wl.CONFIGS[2], wl.seed_of(2)
+    cfg, seed = wl.CONFIGS[wl.DECODE_B64], wl.seed_of(wl.DECODE_B64)
     B, L = cfg["B"], cfg["n_layers"]
     gws, gdicts = zip(*[H.gpu_weights(seed, l) for l in range(L)])
     st_g = sab.State(B, L)
@@ -236,7 +237,7 @@ def test_prefill_chunks_match_oracle_and_decode(sab, case):
     prefill and against the same tokens replayed one by one through the decode path
     (state row 1); states and kept anchor sets must agree afterwards."""
     cfg = PREFILL_CASES[case]
-    seed = wl.seed_of(4)
+    seed = wl.seed_of(wl.PREFILL)
     L = 1
     ow, wdict = H.oracle_weights(seed, 0)
     gw, gdict = H.gpu_weights(seed, 0, prepare=cfg.get("prepare", True))

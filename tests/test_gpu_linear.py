@@ -4,9 +4,12 @@ y = x·wᵀ with BF16 operands and FP32 accumulation, at the layer's shapes
 (F = 13056 / 12288 rows of the fused q/k/v (+ W1 terms) weight, K = 2560;
 F = 2560, K = 4096 for o_proj) and token counts from one decode token to a
 512-sequence batch, ragged counts included (they leave part of a 16-token
-group and of a tile empty).  The kernel splits the work between CTA pairs so
-that some tiles are finished from partial sums of other pairs; every shape
-below exercises that path at some token count.
+group and of a tile empty).  Up to 32 tokens the call runs the weight-
+streaming kernel the layer calls use for small batches (1, 2 or 4 tiles of 8
+tokens, K split between the warps of a block); above, the tcgen05 GEMM, which
+splits the work between CTA pairs so that some tiles are finished from
+partial sums of other pairs; every shape below exercises that path at some
+token count.
 
 Bars:
   FP32 output: |Δ| <= 2^-17·Σ_k |x_k·w_k| against a float64 matmul (FP32
@@ -53,7 +56,7 @@ def bf16_exact(a):
 
 
 @pytest.mark.parametrize("F,K", [(13056, 2560), (12288, 2560), (2560, 4096)])
-@pytest.mark.parametrize("T", [1, 7, 16, 100, 256, 300, 512])
+@pytest.mark.parametrize("T", [1, 7, 9, 16, 24, 32, 33, 100, 256, 300, 512])
 def test_linear_fp32_matches_float64(sab, F, K, T):
     w = _weights(F, K, 11 + F)
     x = _x(T, K, 13 + T)
@@ -68,7 +71,7 @@ def test_linear_fp32_matches_float64(sab, F, K, T):
     assert torch.equal(got, again)
 
 
-@pytest.mark.parametrize("T", [1, 16, 64, 77, 256, 512])
+@pytest.mark.parametrize("T", [1, 5, 16, 31, 64, 77, 256, 512])
 def test_linear_bf16_matches_single_rounding(sab, T):
     F, K = 2560, 4096
     w = _weights(F, K, 5)

@@ -71,7 +71,7 @@ def check_slot_list(st, row, n_layers):
 def test_pool_explicit_commit_matches_oracle_and_moves_nothing(sab):
     """The commit workload (bank and pending full, ~5% exact score ties) in the pooled
     layout: the kept records equal the oracle's bit for bit, no K/V row changes."""
-    seed, n, L, t0 = wl.seed_of(1), 16, 2, 32768
+    seed, n, L, t0 = wl.seed_of(wl.COMMIT), 16, 2, 32768
     plain = sab.State(n, L)
     wl.seed_commit_workload(plain.arrays(), range(n), L, t0, seed, 0, "cuda")
     st = pooled_copy(sab, plain)
@@ -80,7 +80,7 @@ def test_pool_explicit_commit_matches_oracle_and_moves_nothing(sab):
     assert sab.last_device_error(st) == 0
     assert torch.equal(st.bank_k, k_before) and torch.equal(st.bank_v, v_before)
     for seq in (0, 5, 15):
-        ost = oracle.OracleState(1, L, kv=False)
+        ost = oracle.OracleState(1, L)
         wl.seed_commit_workload({k: getattr(ost, k) for k in oracle.OracleState.ARRAYS}, [seq],
                                 L, t0, seed, 0, "cpu")
         ost.commit(-1, 0)
@@ -154,7 +154,7 @@ def plain_view(st, row):
 def test_pool_stream_start_prefill_and_decode_match_oracle(sab):
     """From an empty pooled state: two prefill chunks (256, then a ragged 77, so the
     first commit keeps every record), then decode steps, against the oracle."""
-    seed = wl.seed_of(4)
+    seed = wl.seed_of(wl.PREFILL)
     gw, gdict = H.gpu_weights(seed, 0)
     ow, wdict = H.oracle_weights(seed, 0)
     st = sab.State(1, 1, pool=True)

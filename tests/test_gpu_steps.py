@@ -264,7 +264,7 @@ def test_commit_full_size_workload_matches_oracle(sab):
     oracle on the same seeded rows: every state array after repetition 0; the scores,
     positions and metadata (which records are kept and in which slot) after the later
     ones; and each later merge moves about 205 records on average."""
-    seed, n, L, t0 = wl.seed_of(1), 512, 8, 32768
+    seed, n, L, t0 = wl.seed_of(wl.COMMIT), 512, 8, 32768
     st = sab.State(n, L)
     ids = torch.arange(n, dtype=torch.int32, device="cuda")
     keys = ("bank_score", "pend_score", "bank_pos", "pend_pos", "meta")

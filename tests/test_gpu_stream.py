@@ -49,8 +49,8 @@ def _layer_slice(row, l):
 
 
 def test_prefill_stream_131072_tokens_8_layers(sab):
-    seed = wl.seed_of(4)
-    cfg = wl.CONFIGS[4]
+    seed = wl.seed_of(wl.PREFILL)
+    cfg = wl.CONFIGS[wl.PREFILL]
     assert cfg["tokens"] == CHUNK * N_CHUNKS and cfg["n_layers"] == L and cfg["chunk"] == CHUNK
     gws, gdicts = zip(*[H.gpu_weights(seed, l) for l in range(L)])
     w1 = [d["w1"].double() for d in gdicts]

@@ -42,7 +42,7 @@ def test_affine_and_integer_fills():
 
 
 def test_workload_weights_shapes():
-    w = wl.make_weights(wl.seed_of(0), 0)
+    w = wl.make_weights(wl.seed_of(wl.DECODE_B1), 0)
     assert w["w_qkv"].shape == (12288, 2560) and w["w_qkv"].dtype == torch.bfloat16
     assert w["w_o"].shape == (2560, 4096)
     assert w["w1"].shape == (256, 2560) and w["w1"].dtype == torch.float32
