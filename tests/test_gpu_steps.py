@@ -251,6 +251,13 @@ def test_attend_mixed_batch(sab):
     _attend_case(sab, 4, [4096, 4096, 3, 300], [0, 254, 0, 0])
 
 
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_attend_every_split_count(sab, B):
+    # B = 8, 16, 32 split each branch 8, 4 and 2 ways (B = 1 and 4: 16 ways), each
+    # merged by its own instance of the split merge; ragged pending fills
+    _attend_case(sab, B, [4096] * B, [(53 * b + 11) % 250 for b in range(B)])
+
+
 def test_attend_many_queries_one_split(sab):
     B = 40  # 320 items: one split per branch
     _attend_case(sab, B, [4096] * B, [(37 * b) % 250 for b in range(B)])
