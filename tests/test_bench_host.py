@@ -97,3 +97,82 @@ def test_reference_arm_other_ranks_exit_quietly():
     r = _run_reference({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert not any(l.startswith("{") for l in r.stdout.splitlines())
+
+
+class _FakeNvml:
+    """Read-only NVML stand-in: a scripted SM clock and clock-event-reason bits."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, script):
+        self.script = list(script)  # (sm MHz, reason bits) per query
+        self.i = 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        return "h"
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.script[min(self.i, len(self.script) - 1)][0]
+
+    def nvmlDeviceGetCurrentClocksThrottleReasons(self, h):
+        v = self.script[min(self.i, len(self.script) - 1)][1]
+        self.i += 1
+        return v
+
+
+def test_clock_sampler_keeps_only_timed_samples_and_names_reasons():
+    """The bench's clock record: samples outside begin/end are dropped, the median
+    SM clock and the union of the reasons seen inside are reported (0x4 is
+    sw_power_cap, 0x8 hw_slowdown, 0x20 sw_thermal_slowdown, 0x40
+    hw_thermal_slowdown)."""
+    import time
+    fake = _FakeNvml([(1965, 0x0), (1800, 0x4), (1700, 0x4 | 0x40)])
+    cs = bench.ClockSampler(0)
+    cs.nvml = (fake, "h")
+    t = time.monotonic()
+    cs.windows = [[t, t + 1.0]]
+    cs.samples = [(t - 0.5, 1200.0, 1965.0, {"hw_slowdown"}),  # before the window
+                  (t + 0.1, 1965.0, 1965.0, set()),
+                  (t + 0.2, 1800.0, 1965.0, {"sw_power_cap"}),
+                  (t + 0.3, 1700.0, 1965.0, {"sw_power_cap", "hw_thermal_slowdown"}),
+                  (t + 2.0, 900.0, 1965.0, {"sw_thermal_slowdown"})]  # after it
+    cs.stop_flag = False
+
+    class _Done:
+        def join(self, timeout=None):
+            pass
+    cs.th = _Done()
+    rec = cs.stop()
+    assert rec["samples"] == 3
+    assert rec["sm_mhz"] == 1800.0
+    assert rec["sm_max_mhz"] == 1965.0
+    assert rec["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+
+
+def test_clock_sampler_polls_nvml_only_inside_a_window():
+    """The polling thread reads NVML while a window is open and not after."""
+    import time
+    fake = _FakeNvml([(1900, 0x4)])
+    cs = bench.ClockSampler(0)
+    cs.nvml = (fake, "h")
+    import threading
+    cs.th = threading.Thread(target=cs._poll_nvml, daemon=True)
+    cs.th.start()
+    time.sleep(0.05)
+    assert not cs.samples          # no window yet
+    cs.begin()
+    time.sleep(0.1)
+    cs.end()
+    n = len(cs.samples)
+    time.sleep(0.05)
+    rec = cs.stop()
+    assert n >= 3 and len(cs.samples) == n
+    assert rec["sm_mhz"] == 1900.0 and rec["reasons"] == ["sw_power_cap"]
