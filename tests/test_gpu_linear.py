@@ -92,10 +92,12 @@ def test_linear_bf16_matches_single_rounding(sab, T):
             assert torch.equal(oracle.linear_bf16(w, x[t]), ref[t])
 
 
-def test_linear_row_stride_and_zero_tokens(sab):
+@pytest.mark.parametrize("T", [7, 40])
+def test_linear_row_stride_and_zero_tokens(sab, T):
     """Output rows with a stride above F (the fused projection's layout) leave the
-    columns past F untouched; T = 0 launches nothing."""
-    F, K, T = 2560, 2560, 40
+    columns past F untouched, in both kernels (7 tokens: the weight-streaming one,
+    40: the tcgen05 GEMM); T = 0 launches nothing."""
+    F, K = 2560, 2560
     w = _weights(F, K, 21)
     x = _x(T, K, 22)
     out = torch.full((T, F + 256), 7.0, dtype=torch.float32, device="cuda")
